@@ -1,0 +1,10 @@
+"""fp64 CPU oracle for DCP absorbed-MLA decode (test infrastructure only).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline legs of
+``bench.py`` may import this package.  The CUDA path never does.
+"""
+from .mla_decode import (  # noqa: F401
+    BF16_ROW_BYTES, FP8_ROW_BYTES, LATENT_DIM, ROPE_DIM, ROW_DIM,
+    attention_with_lse, dcp_decode, dcp_merge, decode_bf16, decode_e4m3,
+    decode_rows, e4m3_value, fetch_rows, local_positions, mla_decode_partial,
+)
