@@ -1,0 +1,441 @@
+"""Benchmark: emulated DCP MLA decode steps on B200, one JSON line on rank 0.
+
+A step is the whole hot path for one batch: the N shard partial-attention
+calls (``mla_decode_partial``, each a partial kernel plus its split combine)
+and the LSE merge (``dcp_merge``).  The default workload is the
+agentic-trace-shaped batch (64 requests, 64 heads, fp8 rows, lengths
+lognormal with median 67,000 clipped to [4,096, 200,000], N = 8 shards): the
+configuration the metric "KV-read GB/s and % of HBM peak at >= 64K context"
+is quoted on.  ``value`` is KV bytes read per step / device time per step,
+with the cache resident in HBM; the cache (3.4+ GB) is larger than L2, so no
+flush is needed between steps.
+
+``--impl reference`` times the fp64 CPU oracle instead (bounded samples of
+the same workload on the host cores), for the driver's reference arm.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MLA decode KV-read GB/s and % of HBM peak; decode steps/s at 64K context"
+UNIT = "GB/s"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="agentic",
+                    choices=["agentic", "dense", "million", "sparse", "tiny"])
+    ap.add_argument("--kernel", default="auto", choices=["auto", "simt", "tc"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    return ap.parse_args()
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def kv_bytes(prob) -> int:
+    """KV bytes one step must read: every cached (or, sparse, every selected) row once."""
+    from long_context_decode_mla_b200.workload import ROW_BYTES
+    rb = ROW_BYTES[prob.kv_dtype]
+    if prob.sparse_idx is None:
+        return int(prob.seq_lens.long().sum()) * rb
+    idx = prob.sparse_idx.long().cpu()
+    lens = prob.seq_lens.long().cpu()[:, None]
+    return int(((idx >= 0) & (idx < lens)).sum()) * rb
+
+
+def shard_kv_bytes(prob, s) -> int:
+    from long_context_decode_mla_b200.workload import ROW_BYTES
+    rb = ROW_BYTES[prob.kv_dtype]
+    N = prob.num_shards
+    lens = prob.seq_lens.long().cpu()
+    if prob.sparse_idx is None:
+        n = ((lens - s - 1).clamp(min=-1) // N + 1).clamp(min=0)
+        return int(n.sum()) * rb
+    idx = prob.sparse_idx.long().cpu()
+    ok = (idx >= 0) & (idx < lens[:, None]) & (idx % N == s)
+    return int(ok.sum()) * rb
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "long_context_decode_mla_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str, kernel: str):
+    """DRAM traffic per launch from a committed ncu summary, if it is current."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    e = d.get(f"{workload}/{kernel}")
+    if not e or e.get("source_hash") != kernel_source_hash():
+        return None
+    return e.get("bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled in the background."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index, self.samples, self.proc = index, [], None
+        self.t_on = self.t_off = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        threading.Thread(target=self._read, daemon=True).start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.samples.append((time.time(), line.strip()))
+
+    def mark(self, on: bool):
+        if on:
+            self.t_on = time.time()
+        else:
+            self.t_off = time.time()
+
+    def stop(self):
+        if self.proc:
+            time.sleep(0.12)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = [s for t, s in self.samples if self.t_on and self.t_off and
+                self.t_on <= t <= self.t_off + 0.06]
+        window = "timed region"
+        if not rows:
+            rows = [s for _, s in self.samples]
+            window = "whole run (timed region shorter than the sampling interval)"
+        mhz, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            f = [x.strip() for x in r.split(",")]
+            try:
+                mhz.append(float(f[0]))
+                mx = float(f[1])
+            except (ValueError, IndexError):
+                continue
+            for name, v in zip(names, f[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(mhz), "window": window}
+
+
+# ------------------------------------------------------------------ ours ----
+
+def run_ours(args, rank, world, local):
+    import torch
+    import torch.distributed as dist
+
+    from long_context_decode_mla_b200 import dcpmla, workload
+
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", device_id=torch.device("cuda", local),
+                                timeout=__import__("datetime").timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+    # weak scaling: every rank decodes its own batch (distinct seed), no collectives
+    cfg = dict(workload.CONFIGS[args.workload])
+    prob = workload.make_problem(args.workload, device=dev, kv_device=dev,
+                                 seed=cfg["seed"] + 1000 * rank)
+    N, B, H = prob.num_shards, prob.batch, prob.heads
+    topk = 0 if prob.sparse_idx is None else prob.sparse_idx.shape[1]
+    long_single = args.workload == "million"
+    streams = [torch.cuda.Stream(device=dev) for _ in range(N)] if long_single else None
+    splits = max(1, dcpmla.device_sm_count() // N) if long_single else 0
+    dec = dcpmla.DcpDecoder(B, H, N, topk=topk, num_splits=splits, device=dev,
+                            impl=args.kernel, streams=streams)
+    stream = torch.cuda.current_stream(dev)
+    kvb = kv_bytes(prob)
+    per_shard_kv = [shard_kv_bytes(prob, s) for s in range(N)]
+    other_per_launch = B * H * 576 * 2 + B * H * 513 * 4
+
+    # events around every shard call of every timed step (same stream): the
+    # partial kernel's average launch duration for the roofline
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(N)] for _ in range(args.steps)]
+
+    def step(k=None):
+        if streams:
+            dec.step(prob, stream)
+            return
+        for s in range(N):
+            if k is not None:
+                ev[k][s][0].record(stream)
+            dcpmla.mla_decode_partial(prob.q, prob.kv_cache, prob.kv_dtype, prob.block_tables[s],
+                                      prob.seq_lens, s, N, prob.sparse_idx, prob.softmax_scale,
+                                      dec.partials[s], dec.lses[s], dec.workspaces[s],
+                                      splits, args.kernel, stream)
+            if k is not None:
+                ev[k][s][1].record(stream)
+        dcpmla.dcp_merge(dec.partials, dec.lses, dec.out, dec.out_lse, stream)
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize(dev)
+    assert dec.flags() == 0, "device flags set during warm-up"
+
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    sampler.mark(True)
+    t0.record(stream)
+    for k in range(args.steps):
+        step(k)
+    t1.record(stream)
+    t1.synchronize()
+    sampler.mark(False)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    ms_step = t0.elapsed_time(t1) / args.steps
+    launch_ms = [0.0] * N
+    if not streams:
+        for k in range(args.steps):
+            for s in range(N):
+                launch_ms[s] += ev[k][s][0].elapsed_time(ev[k][s][1]) / args.steps
+
+    # end to end through the public API, host buffers in pinned memory
+    h_q = prob.q.cpu().pin_memory()
+    h_lens = prob.seq_lens.cpu().pin_memory()
+    h_tables = prob.block_tables.cpu().pin_memory()
+    h_idx = None if prob.sparse_idx is None else prob.sparse_idx.cpu().pin_memory()
+    h_out = torch.empty_like(dec.out, device="cpu").pin_memory()
+    h_lse = torch.empty_like(dec.out_lse, device="cpu").pin_memory()
+    e_steps = max(3, args.steps // 4)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def e2e_step():
+        prob.q.copy_(h_q, non_blocking=True)
+        prob.seq_lens.copy_(h_lens, non_blocking=True)
+        prob.block_tables.copy_(h_tables, non_blocking=True)
+        if h_idx is not None:
+            prob.sparse_idx.copy_(h_idx, non_blocking=True)
+        dec.step(prob, stream)
+        h_out.copy_(dec.out, non_blocking=True)
+        h_lse.copy_(dec.out_lse, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(e_steps):
+        e2e_step()
+    e1.record(stream)
+    e1.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e_steps
+    h2d = h_q.numel() * 2 + h_lens.numel() * 4 + h_tables.numel() * 4 + \
+        (0 if h_idx is None else h_idx.numel() * 4)
+    d2h = h_out.numel() * 4 + h_lse.numel() * 4
+    assert dec.flags() == 0, "device flags set"
+    sampler.stop()
+
+    times = torch.tensor([ms_step, e2e_ms], device=dev)
+    if world > 1:
+        dist.all_reduce(times, op=dist.ReduceOp.MAX)
+    ms_step, e2e_ms = times.tolist()
+    gpu_launches = args.steps * (N * (1 if (prob.sparse_idx is not None) else 2) + 1)
+    peak, peak_kind = measured_peaks()
+    result = None
+    if rank == 0:
+        value = world * kvb / (ms_step * 1e-3) / 1e9
+        if launch_ms[0] > 0:
+            alg = [per_shard_kv[s] + other_per_launch for s in range(N)]
+            achieved = sum(alg) / (sum(launch_ms) * 1e-3) / 1e9
+        else:   # concurrent shard streams: attribute the step to the partial kernels
+            achieved = (kvb + N * other_per_launch) / (ms_step * 1e-3) / 1e9
+        traffic = recorded_traffic(args.workload, args.kernel)
+        clocks = sampler.summary()
+        result = {
+            "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": round(ms_step, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if args.kernel != "simt" else "f32",
+            "data": "synthetic (seeded; no public trace or checkpoint available)",
+            "config": {
+                "workload": describe(args.workload, prob), "global_batch": B * world,
+                "heads": H, "shards": N, "kv_dtype": prob.kv_dtype,
+                "seq_len_median": int(prob.seq_lens.float().median()),
+                "kv_bytes_per_step_per_gpu": kvb, "kernel": args.kernel,
+                "parallelism": f"{world} independent replicas, {N} DCP shards emulated per GPU",
+                "l2": "no flush: the KV read per step is larger than the 126 MB L2",
+            },
+            "steps_per_s": round(1e3 / ms_step, 2),
+            "pct_hbm_peak_kv": round(100 * value / world / peak, 1),
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+                         "unit": "GB/s", "frac": round(achieved / peak, 4),
+                         "traffic": traffic, "peak_source": peak_kind,
+                         "kernel": "mla_decode_partial (partial + split combine)"},
+            "e2e": {"value": round(world * kvb / (e2e_ms * 1e-3) / 1e9, 1), "unit": UNIT,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": round(e2e_ms, 4),
+                    "note": "per step: q, lengths, block tables (and indices) host->device; "
+                            "merged O and LSE device->host; the KV cache is resident state"},
+            "gpu_launches": gpu_launches,
+            "clocks": clocks,
+        }
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return result, prob
+
+
+def describe(name, prob):
+    lens = prob.seq_lens
+    return (f"{name}: batch {prob.batch}, {prob.heads} heads, {prob.kv_dtype} rows, "
+            f"lengths {int(lens.min())}..{int(lens.max())} (median {int(lens.float().median())}), "
+            f"{prob.num_shards} round-robin shards + LSE merge")
+
+
+# ------------------------------------------------------------------ oracle --
+
+def oracle_sample_step(prob_np, b):
+    import oracle
+    return oracle.dcp_decode(prob_np["q"], prob_np["kv_cache"], prob_np["kv_dtype"],
+                             prob_np["block_tables"], prob_np["seq_lens"],
+                             prob_np["num_shards"], prob_np["softmax_scale"],
+                             prob_np["sparse_idx"], prob_np["block_size"], [b])
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        return max((i.get("num_threads", 1) for i in info), default=1)
+    except Exception:
+        return 1
+
+
+def cpu_sample_problem(workload_name, target_len):
+    """One request of the workload's shape (same heads, row format, shards) on the CPU."""
+    from long_context_decode_mla_b200 import workload
+    cfg = workload.CONFIGS[workload_name]
+    over = dict(batch=1, seq_len=[target_len])
+    if cfg.get("topk"):
+        over["topk"] = cfg["topk"]
+    return workload.make_problem(workload_name, **over)
+
+
+def time_oracle(workload_name, seconds_budget, sample_len=None):
+    """Time the oracle on single-request samples until the budget is spent."""
+    from long_context_decode_mla_b200 import workload
+    cfg = workload.CONFIGS[workload_name]
+    if sample_len is None:
+        sample_len = 16384 if cfg["seq_len"] == "lognormal" else min(int(cfg["seq_len"]), 16384)
+    prob = cpu_sample_problem(workload_name, sample_len)
+    ni = prob.numpy_inputs()
+    kvb = kv_bytes(prob)
+    n, t0 = 0, time.perf_counter()
+    while True:
+        oracle_sample_step(ni, 0)
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= seconds_budget:
+            break
+    return {"value": round(n * kvb / el / 1e9, 4), "unit": UNIT, "cores": blas_threads(),
+            "kind": "oracle",
+            "sample": (f"{n} x one request of the {workload_name} workload "
+                       f"(L={sample_len}, {prob.heads} heads, {prob.kv_dtype}, "
+                       f"{prob.num_shards} shards + merge), {el:.1f} s of fp64 numpy")}, el / n
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    from long_context_decode_mla_b200 import workload
+    cfg = workload.CONFIGS[args.workload]
+    sample_len = 16384 if cfg["seq_len"] == "lognormal" else min(int(cfg["seq_len"]), 16384)
+    prob = cpu_sample_problem(args.workload, sample_len)
+    ni = prob.numpy_inputs()
+    kvb = kv_bytes(prob)
+    for _ in range(max(3, args.warmup)):
+        oracle_sample_step(ni, 0)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_sample_step(ni, 0)
+    el = time.perf_counter() - t0
+    value = kvb * args.steps / el / 1e9
+    cpu = {"value": round(value, 4), "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+           "sample": (f"each step: one request of the {args.workload} workload (L={sample_len}, "
+                      f"{prob.heads} heads, {prob.kv_dtype}, {prob.num_shards} shards + merge)")}
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": max(3, args.warmup),
+        "ms_per_step": round(1e3 * el / args.steps, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": describe(args.workload, prob) + " (one-request CPU sample)"},
+        "cpu_baseline": cpu,
+        "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse()
+    rank, world, local = dist_env()
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+    res, prob = run_ours(args, rank, world, local)
+    if rank == 0:
+        if not args.no_cpu_baseline:
+            res["cpu_baseline"], _ = time_oracle(args.workload, args.cpu_seconds)
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

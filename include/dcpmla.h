@@ -1,0 +1,165 @@
+/*
+ * dcpmla.h - C ABI of libdcpmla.so: decode-context-parallel (DCP) absorbed-MLA
+ * decode on NVIDIA B200 (sm_100a).
+ *
+ * What the calls compute (cited by page title and section):
+ *
+ *  - "GLM-5.2 vLLM Decode Context Parallelism", section "See why vLLM 0.26.0
+ *    fails": under DCP each rank computes a partial attention output over its
+ *    own part of the cache, and the partial outputs are combined with the
+ *    softmax normalisation, which needs the decode log-sum-exp (LSE).
+ *  - same page, section "Separate the backend merge from stable": the LSE is
+ *    returned per (token, head); global sparse top-K indices are localised to
+ *    the rank that owns each position; a row with no selected local token
+ *    returns the neutral pair (O = 0, LSE = -inf) and drops out of the merge.
+ *  - "How vLLM Serves GLM-5.3 with Million-Token Contexts on 16 H200s",
+ *    section "The core design": cache tokens are distributed round-robin, so
+ *    each of N ranks holds 1/N of them.  Here token t belongs to shard t mod N
+ *    and sits at local index t div N of that shard.
+ *  - "The Final Verification: Confirming a 200k Context Deployment on GLM-5",
+ *    section "The Decision-Making Process Visible in the Reasoning": one MLA
+ *    cache row per token and layer holds kv_lora_rank + qk_rope_head_dim =
+ *    512 + 64 values (1,152 bytes in bf16).
+ *
+ * Readings used where the pages are silent:
+ *  - Absorbed MLA: the query row (576 values) is already in the latent space,
+ *    every query head attends to the one shared latent row, scores are
+ *    softmax_scale * <q, k> over all 576 values, and the value is the first
+ *    512 values of the same row.  The output is the 512-wide latent result.
+ *  - LSE is the natural logarithm of sum_t exp(score_t), scale included.
+ *  - fp8 rows ("fp8_ds_mla"-like, 656 bytes): 512 OCP E4M3 codes, then 4
+ *    little-endian fp32 scales (latent values [128g, 128g+128) use scale g),
+ *    then 64 bf16 rope values.  bf16 rows: 576 bf16 values (1,152 bytes).
+ *  - Each shard has its own block table over its local indices; block size
+ *    is 64 rows.
+ *
+ * Conventions for every entry point:
+ *  - All array pointers are DEVICE pointers owned by the caller.  The library
+ *    allocates no memory, never synchronises, and only enqueues work on
+ *    `stream` (a cudaStream_t; NULL means the legacy default stream).  The
+ *    call returns once the work is enqueued.
+ *  - Arguments are checked on the host, before anything is launched; a
+ *    failed check returns a negative DCPMLA_ERR_* code and launches nothing
+ *    (fail closed: nothing is clamped or guessed).  Device-side contents
+ *    (block-table entries, sparse indices, lengths) are range-checked in the
+ *    kernels: an out-of-range entry is skipped, never dereferenced, and sets
+ *    a bit in the workspace's device flag word (see below).
+ *  - Asynchronous CUDA faults surface at the caller's next synchronisation;
+ *    launch failures are returned as DCPMLA_ERR_CUDA.
+ */
+#ifndef DCPMLA_H
+#define DCPMLA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Cache row formats. */
+#define DCPMLA_KV_BF16 0     /* 1,152-byte rows: 576 bf16 */
+#define DCPMLA_KV_FP8 1      /* 656-byte rows: 512 e4m3 + 4 fp32 scales + 64 bf16 rope */
+
+/* Kernel selection for mla_decode_partial. */
+#define DCPMLA_IMPL_AUTO 0   /* fastest available for the arguments */
+#define DCPMLA_IMPL_SIMT 1   /* plain CUDA-core kernel (any H <= 64) */
+#define DCPMLA_IMPL_TC 2     /* tcgen05 / TMEM tensor-core kernel */
+
+/* Return codes. */
+#define DCPMLA_OK 0
+#define DCPMLA_ERR_INVALID_ARGUMENT (-1)   /* null pointer, bad size, shard id out of range ... */
+#define DCPMLA_ERR_UNSUPPORTED (-2)        /* valid but not implemented (e.g. H > 64, block != 64) */
+#define DCPMLA_ERR_WORKSPACE (-3)          /* workspace missing or smaller than required */
+#define DCPMLA_ERR_ALIGNMENT (-4)          /* a pointer is not 16-byte aligned */
+#define DCPMLA_ERR_CUDA (-5)               /* a CUDA runtime call or launch failed */
+
+/* Bits the kernels OR into the workspace flag word (int32 at byte 0). */
+#define DCPMLA_FLAG_BAD_BLOCK 1      /* a block-table entry was outside [0, num_blocks) */
+#define DCPMLA_FLAG_BAD_LENGTH 2     /* a length was negative or needs more blocks than the table row has */
+
+#define DCPMLA_HEAD_DIM 576          /* 512 latent + 64 rope */
+#define DCPMLA_V_DIM 512
+#define DCPMLA_BLOCK_SIZE 64
+#define DCPMLA_MAX_HEADS 64
+
+/*
+ * Bytes of workspace that mla_decode_partial needs for these sizes.
+ *
+ *   batch, num_heads: as passed to mla_decode_partial.
+ *   num_splits: as passed to mla_decode_partial (0 = automatic, which uses
+ *               the SM count of the current device).
+ *   topk: length of each sparse index list, 0 for dense decode.
+ *   bytes: receives the size.
+ *
+ * Layout: a 256-byte header (int32 flag word at byte 0, the rest reserved),
+ * then per-split partial results.  The flag word is OR-ed by the kernels and
+ * never cleared by the library: zero it before the first call if you read it.
+ * Returns DCPMLA_OK or a negative code.
+ */
+int mla_decode_workspace_size(int batch, int num_heads, int num_splits, int topk,
+                              size_t* bytes);
+
+/*
+ * Partial attention of one DCP shard, with its LSE, for every request.
+ *
+ *   q            [batch][num_heads][576] bf16, 16-byte aligned.
+ *   kv_cache     [num_blocks][64][row bytes] raw rows in format `kv_dtype`,
+ *                16-byte aligned.
+ *   block_table  [batch][block_table_stride] int32: this shard's table; entry
+ *                k of request b is the physical block holding local rows
+ *                [64k, 64k+64).
+ *   seq_lens     [batch] int32 GLOBAL cached lengths L_b.  The shard's local
+ *                length is the number of t in [0, L_b) with t mod N = shard_id.
+ *   shard_id, num_shards: 0 <= shard_id < num_shards.
+ *   sparse_idx   NULL for dense decode, else [batch][topk] int32 global token
+ *                positions; entries outside [0, L_b) are skipped (-1 pads);
+ *                entries owned by other shards are skipped.
+ *   softmax_scale  multiplies <q, k> before the softmax.
+ *   out_partial  [batch][num_heads][512] fp32: sum_t softmax_t * v_t over
+ *                this shard's tokens (0 for a request with none).
+ *   out_lse      [batch][num_heads] fp32: natural-log LSE (-inf if none).
+ *   workspace, workspace_bytes: at least mla_decode_workspace_size(...).
+ *   num_splits   CTAs to spread the work over (0 = automatic: the SM count).
+ *   impl         DCPMLA_IMPL_* (AUTO picks the tensor-core kernel when it
+ *                supports the arguments).
+ *   stream       cudaStream_t to enqueue on.
+ *
+ * Returns DCPMLA_OK or a negative DCPMLA_ERR_* code.
+ */
+int mla_decode_partial(const void* q, const void* kv_cache, int kv_dtype, int64_t num_blocks,
+                       int block_size, const int32_t* block_table, int block_table_stride,
+                       const int32_t* seq_lens, int batch, int num_heads, int shard_id,
+                       int num_shards, const int32_t* sparse_idx, int topk,
+                       float softmax_scale, float* out_partial, float* out_lse,
+                       void* workspace, size_t workspace_bytes, int num_splits, int impl,
+                       void* stream);
+
+/*
+ * LSE-weighted merge of N shard partials into the full-context result.
+ *
+ *   partials  [num_shards][batch][num_heads][512] fp32 (16-byte aligned).
+ *   lses      [num_shards][batch][num_heads] fp32.
+ *   out       [batch][num_heads][512] fp32: with M = max_i lse_i and
+ *             w_i = exp(lse_i - M), out = sum_i w_i partial_i / sum_i w_i.
+ *             Shards with lse = -inf weigh exactly 0; if all are -inf the
+ *             result is 0.
+ *   out_lse   [batch][num_heads] fp32 merged LSE M + ln sum_i w_i (-inf if all
+ *             are -inf), or NULL if not wanted.
+ *
+ * Returns DCPMLA_OK or a negative code.
+ */
+int dcp_merge(const float* partials, const float* lses, int num_shards, int batch,
+              int num_heads, float* out, float* out_lse, void* stream);
+
+/* Static description of a return code (never NULL). */
+const char* dcpmla_error_string(int code);
+
+/* Number of SMs of the current device (what num_splits = 0 uses). */
+int dcpmla_device_sm_count(int* sm_count);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DCPMLA_H */

@@ -1,0 +1,168 @@
+// C ABI of libdcpmla.so: argument checks, work decomposition and launches.
+// The entry points are declared (and their contracts stated) in dcpmla.h.
+#include "dcpmla.h"
+
+#include <cmath>
+#include <cstdint>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace dcpmla {
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int sm_count_current(int* out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return DCPMLA_ERR_CUDA;
+  static int cache[64] = {0};
+  if (dev >= 0 && dev < 64 && cache[dev] > 0) {
+    *out = cache[dev];
+    return DCPMLA_OK;
+  }
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+    return DCPMLA_ERR_CUDA;
+  if (dev >= 0 && dev < 64) cache[dev] = n;
+  *out = n;
+  return DCPMLA_OK;
+}
+
+// CTAs sharing one shard's dense tile space.
+int resolve_ctas(int num_splits, int* ctas) {
+  if (num_splits > 0) {
+    *ctas = num_splits;
+    return DCPMLA_OK;
+  }
+  return sm_count_current(ctas);
+}
+
+// Index-list chunks per request in sparse mode: enough CTAs to cover the
+// device when the batch is small, and chunks short enough for the kernels'
+// on-chip selection lists.
+int sparse_parts_for(int batch, int topk, int ctas) {
+  const int cap = simt_sparse_chunk_max();
+  int p = (topk + cap - 1) / cap;
+  int fill = batch > 0 ? ctas / batch : 1;
+  if (fill > p) p = fill;
+  if (p > topk) p = topk;
+  return p < 1 ? 1 : p;
+}
+
+long long slots_for(int batch, int topk, int ctas) {
+  if (topk > 0) return (long long)batch * sparse_parts_for(batch, topk, ctas);
+  return (long long)ctas + batch;
+}
+
+}  // namespace
+}  // namespace dcpmla
+
+using namespace dcpmla;
+
+extern "C" {
+
+const char* dcpmla_error_string(int code) {
+  switch (code) {
+    case DCPMLA_OK: return "ok";
+    case DCPMLA_ERR_INVALID_ARGUMENT: return "invalid argument";
+    case DCPMLA_ERR_UNSUPPORTED: return "unsupported argument combination";
+    case DCPMLA_ERR_WORKSPACE: return "workspace missing or too small";
+    case DCPMLA_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+    case DCPMLA_ERR_CUDA: return "CUDA runtime error";
+    default: return "unknown error code";
+  }
+}
+
+int dcpmla_device_sm_count(int* sm_count) {
+  if (!sm_count) return DCPMLA_ERR_INVALID_ARGUMENT;
+  return sm_count_current(sm_count);
+}
+
+int mla_decode_workspace_size(int batch, int num_heads, int num_splits, int topk,
+                              size_t* bytes) {
+  if (!bytes || batch < 0 || num_heads < 1 || num_splits < 0 || topk < 0)
+    return DCPMLA_ERR_INVALID_ARGUMENT;
+  if (num_heads > kMaxHeads) return DCPMLA_ERR_UNSUPPORTED;
+  int ctas = 0;
+  int rc = resolve_ctas(num_splits, &ctas);
+  if (rc != DCPMLA_OK) return rc;
+  *bytes = ws_total(slots_for(batch, topk, ctas), num_heads);
+  return DCPMLA_OK;
+}
+
+int mla_decode_partial(const void* q, const void* kv_cache, int kv_dtype, int64_t num_blocks,
+                       int block_size, const int32_t* block_table, int block_table_stride,
+                       const int32_t* seq_lens, int batch, int num_heads, int shard_id,
+                       int num_shards, const int32_t* sparse_idx, int topk,
+                       float softmax_scale, float* out_partial, float* out_lse,
+                       void* workspace, size_t workspace_bytes, int num_splits, int impl,
+                       void* stream) {
+  // ---- scalar checks (fail closed, nothing launched on error) ----
+  if (batch < 0 || num_heads < 1 || num_shards < 1 || shard_id < 0 || shard_id >= num_shards ||
+      block_size < 1 || block_table_stride < 1 || num_blocks < 1 || num_splits < 0 ||
+      topk < 0 || (sparse_idx && topk < 1) || !std::isfinite(softmax_scale))
+    return DCPMLA_ERR_INVALID_ARGUMENT;
+  if (kv_dtype != DCPMLA_KV_BF16 && kv_dtype != DCPMLA_KV_FP8) return DCPMLA_ERR_INVALID_ARGUMENT;
+  if (impl != DCPMLA_IMPL_AUTO && impl != DCPMLA_IMPL_SIMT && impl != DCPMLA_IMPL_TC)
+    return DCPMLA_ERR_INVALID_ARGUMENT;
+  if (num_heads > kMaxHeads || block_size != kBlock) return DCPMLA_ERR_UNSUPPORTED;
+  if (batch == 0) return DCPMLA_OK;
+  if (!q || !kv_cache || !block_table || !seq_lens || !out_partial || !out_lse)
+    return DCPMLA_ERR_INVALID_ARGUMENT;
+  if (!aligned16(q) || !aligned16(kv_cache) || !aligned16(out_partial) || !aligned16(out_lse) ||
+      (workspace && !aligned16(workspace)))
+    return DCPMLA_ERR_ALIGNMENT;
+  const int eff_topk = sparse_idx ? topk : 0;
+  int ctas = 0;
+  int rc = resolve_ctas(num_splits, &ctas);
+  if (rc != DCPMLA_OK) return rc;
+  const long long slots = slots_for(batch, eff_topk, ctas);
+  if (!workspace || workspace_bytes < ws_total(slots, num_heads)) return DCPMLA_ERR_WORKSPACE;
+
+  PartialParams p{};
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.kv = static_cast<const uint8_t*>(kv_cache);
+  p.num_blocks = num_blocks;
+  p.block_table = block_table;
+  p.bt_stride = block_table_stride;
+  p.seq_lens = seq_lens;
+  p.batch = batch;
+  p.heads = num_heads;
+  p.shard = shard_id;
+  p.nshards = num_shards;
+  p.sparse_idx = sparse_idx;
+  p.topk = eff_topk;
+  p.sparse_parts = sparse_idx ? sparse_parts_for(batch, topk, ctas) : 1;
+  p.scale = softmax_scale;
+  p.out = out_partial;
+  p.out_lse = out_lse;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  p.flags = reinterpret_cast<int*>(ws);
+  p.ws_o = reinterpret_cast<float*>(ws + ws_o_offset());
+  p.ws_lse = reinterpret_cast<float*>(ws + ws_lse_offset(slots, num_heads));
+  p.num_ctas = ctas;
+
+  const bool tc_ok = tc_supports(p, kv_dtype);
+  if (impl == DCPMLA_IMPL_TC && !tc_ok) return DCPMLA_ERR_UNSUPPORTED;
+  const bool use_tc = impl == DCPMLA_IMPL_TC || (impl == DCPMLA_IMPL_AUTO && tc_ok);
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = use_tc ? launch_partial_tc(p, kv_dtype, st) : launch_partial_simt(p, kv_dtype, st);
+  if (e != cudaSuccess) return DCPMLA_ERR_CUDA;
+  e = launch_split_combine(p, st);
+  return e == cudaSuccess ? DCPMLA_OK : DCPMLA_ERR_CUDA;
+}
+
+int dcp_merge(const float* partials, const float* lses, int num_shards, int batch,
+              int num_heads, float* out, float* out_lse, void* stream) {
+  if (num_shards < 1 || batch < 0 || num_heads < 1) return DCPMLA_ERR_INVALID_ARGUMENT;
+  if (batch == 0) return DCPMLA_OK;
+  if (!partials || !lses || !out) return DCPMLA_ERR_INVALID_ARGUMENT;
+  if (!aligned16(partials) || !aligned16(out)) return DCPMLA_ERR_ALIGNMENT;
+  cudaError_t e = launch_dcp_merge(partials, lses, num_shards, batch, num_heads, out, out_lse,
+                                   static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? DCPMLA_OK : DCPMLA_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,187 @@
+"""ctypes binding of libdcpmla.so (argument marshalling only).
+
+The functions keep the C names (``mla_decode_partial``, ``dcp_merge``,
+``mla_decode_workspace_size``, ``dcpmla_error_string``); they take torch
+tensors for device memory, pass raw pointers and sizes, and raise
+:class:`DcpMlaError` on a negative return code.  All arithmetic happens in the
+library's CUDA kernels.  :class:`DcpDecoder` strings the calls together for a
+whole emulated DCP step (N shard partials, then the merge).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libdcpmla.so")
+
+KV_DTYPES = {"bf16": 0, "fp8": 1}
+IMPLS = {"auto": 0, "simt": 1, "tc": 2}
+HEAD_DIM, V_DIM, BLOCK_SIZE, MAX_HEADS = 576, 512, 64, 64
+FLAG_BAD_BLOCK, FLAG_BAD_LENGTH = 1, 2
+
+_lib = None
+
+
+class DcpMlaError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        super().__init__(f"{where} failed: {error_string(code)} (code {code})")
+        self.code = code
+
+
+def lib() -> ctypes.CDLL:
+    """Load libdcpmla.so (once).  Raises if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(
+            f"{LIB_PATH} is missing: build it with `python -m long_context_decode_mla_b200.build`"
+            " (the decode path has no fallback)")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i32, i64, f32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+    L.mla_decode_workspace_size.argtypes = [i32, i32, i32, i32, ctypes.POINTER(sz)]
+    L.mla_decode_workspace_size.restype = i32
+    L.mla_decode_partial.argtypes = [vp, vp, i32, i64, i32, vp, i32, vp, i32, i32, i32, i32, vp,
+                                     i32, f32, vp, vp, vp, sz, i32, i32, vp]
+    L.mla_decode_partial.restype = i32
+    L.dcp_merge.argtypes = [vp, vp, i32, i32, i32, vp, vp, vp]
+    L.dcp_merge.restype = i32
+    L.dcpmla_error_string.argtypes = [i32]
+    L.dcpmla_error_string.restype = ctypes.c_char_p
+    L.dcpmla_device_sm_count.argtypes = [ctypes.POINTER(i32)]
+    L.dcpmla_device_sm_count.restype = i32
+    _lib = L
+    return L
+
+
+def error_string(code: int) -> str:
+    return lib().dcpmla_error_string(int(code)).decode()
+
+
+dcpmla_error_string = error_string
+
+
+def _check(code: int, where: str):
+    if code != 0:
+        raise DcpMlaError(code, where)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def padded_heads(num_heads: int) -> int:
+    """Query-head envelope of the tensor-core kernel (heads padded to 64 rows).
+
+    Mirrors the fp8 sparse-MLA head envelope ("GLM-5.2 vLLM Decode Context
+    Parallelism", "Calculate the GLM-5.2 head envelope"): 8 local or up to 64
+    gathered heads all land in the 64-row envelope; more than 64 would need
+    the 128 envelope, which this library does not take.
+    """
+    if num_heads < 1:
+        raise ValueError("num_heads must be >= 1")
+    return 64 if num_heads <= 64 else 128
+
+
+def device_sm_count() -> int:
+    n = ctypes.c_int(0)
+    _check(lib().dcpmla_device_sm_count(ctypes.byref(n)), "dcpmla_device_sm_count")
+    return n.value
+
+
+def mla_decode_workspace_size(batch: int, num_heads: int, num_splits: int = 0,
+                              topk: int = 0) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().mla_decode_workspace_size(batch, num_heads, num_splits, topk, ctypes.byref(n)),
+           "mla_decode_workspace_size")
+    return n.value
+
+
+def mla_decode_partial(q, kv_cache, kv_dtype, block_table, seq_lens, shard_id, num_shards,
+                       sparse_idx, softmax_scale, out_partial, out_lse, workspace,
+                       num_splits: int = 0, impl: str | int = "auto", stream=None,
+                       block_size: int = BLOCK_SIZE, num_blocks: int | None = None):
+    """One shard's partial attention + LSE (see include/dcpmla.h)."""
+    B, H = q.shape[0], q.shape[1]
+    kvd = KV_DTYPES[kv_dtype] if isinstance(kv_dtype, str) else int(kv_dtype)
+    nb = kv_cache.shape[0] if num_blocks is None else num_blocks
+    topk = 0 if sparse_idx is None else sparse_idx.shape[1]
+    impl_code = IMPLS[impl] if isinstance(impl, str) else int(impl)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = lib().mla_decode_partial(
+        _ptr(q), _ptr(kv_cache), kvd, nb, block_size, _ptr(block_table), block_table.shape[-1],
+        _ptr(seq_lens), B, H, shard_id, num_shards, _ptr(sparse_idx), topk,
+        float(softmax_scale), _ptr(out_partial), _ptr(out_lse), _ptr(workspace), ws_bytes,
+        num_splits, impl_code, _stream(stream))
+    _check(rc, "mla_decode_partial")
+
+
+def dcp_merge(partials, lses, out, out_lse=None, stream=None):
+    """LSE-weighted merge of [N, B, H, 512] partials (see include/dcpmla.h)."""
+    N, B, H = partials.shape[0], partials.shape[1], partials.shape[2]
+    rc = lib().dcp_merge(_ptr(partials), _ptr(lses), N, B, H, _ptr(out), _ptr(out_lse),
+                         _stream(stream))
+    _check(rc, "dcp_merge")
+
+
+class DcpDecoder:
+    """Buffers and calls for whole emulated DCP decode steps on one GPU.
+
+    Holds the outputs ([N, B, H, 512] partials, [N, B, H] LSEs, merged
+    [B, H, 512] and [B, H]) and one workspace per shard, so shards issued on
+    different streams never share scratch memory.
+    """
+
+    def __init__(self, batch, heads, num_shards, topk=0, num_splits=0, device="cuda",
+                 impl="auto", streams=None):
+        self.batch, self.heads, self.num_shards = batch, heads, num_shards
+        self.num_splits, self.impl, self.topk = num_splits, impl, topk
+        dev = torch.device(device)
+        self.partials = torch.empty(num_shards, batch, heads, V_DIM, device=dev)
+        self.lses = torch.empty(num_shards, batch, heads, device=dev)
+        self.out = torch.empty(batch, heads, V_DIM, device=dev)
+        self.out_lse = torch.empty(batch, heads, device=dev)
+        nbytes = mla_decode_workspace_size(batch, heads, num_splits, topk)
+        self.workspaces = [torch.zeros(nbytes, dtype=torch.uint8, device=dev)
+                           for _ in range(num_shards)]
+        self.streams = streams
+
+    def flags(self) -> int:
+        """OR of the device flag words of all shard workspaces (syncs)."""
+        v = 0
+        for w in self.workspaces:
+            v |= int(w[:4].view(torch.int32).item())
+        return v
+
+    def step(self, prob, stream=None):
+        """All N shard partials, then the merge, for a DecodeProblem on the GPU."""
+        base = torch.cuda.current_stream() if stream is None else stream
+        streams = self.streams
+        if streams:
+            ev = torch.cuda.Event()
+            ev.record(base)
+        for s in range(self.num_shards):
+            st = streams[s % len(streams)] if streams else base
+            if streams:
+                st.wait_event(ev)
+            mla_decode_partial(prob.q, prob.kv_cache, prob.kv_dtype, prob.block_tables[s],
+                               prob.seq_lens, s, self.num_shards, prob.sparse_idx,
+                               prob.softmax_scale, self.partials[s], self.lses[s],
+                               self.workspaces[s], self.num_splits, self.impl, st,
+                               prob.block_size)
+        if streams:
+            for st in streams:
+                e2 = torch.cuda.Event()
+                e2.record(st)
+                base.wait_event(e2)
+        dcp_merge(self.partials, self.lses, self.out, self.out_lse, base)
+        return self.out, self.out_lse

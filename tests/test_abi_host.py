@@ -1,0 +1,118 @@
+"""Host-side checks of the C ABI: exported symbols and fail-closed argument checks.
+
+None of these calls reaches a kernel launch: every case returns an error code
+from the host-side checks, so they run without a GPU (and are harmless with
+one).
+"""
+import ctypes
+import json
+import os
+import re
+
+import pytest
+
+from long_context_decode_mla_b200 import dcpmla
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "dcpmla.h")
+
+OK, EINVAL, EUNSUP, EWS, EALIGN, ECUDA = 0, -1, -2, -3, -4, -5
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return set(re.findall(r"^\s*(?:const\s+)?\w+\**\s+\**(\w+)\s*\(", text, flags=re.M))
+
+
+def test_header_declares_the_entry_points():
+    names = _declared_functions()
+    assert {"mla_decode_partial", "dcp_merge", "mla_decode_workspace_size",
+            "dcpmla_error_string", "dcpmla_device_sm_count"} <= names
+
+
+def test_library_exports_every_declared_symbol():
+    L = dcpmla.lib()
+    for name in _declared_functions():
+        assert hasattr(L, name), name
+
+
+def test_error_strings():
+    for code in (OK, EINVAL, EUNSUP, EWS, EALIGN, ECUDA, -99):
+        assert isinstance(dcpmla.error_string(code), str) and dcpmla.error_string(code)
+
+
+def test_workspace_size_grows_with_splits_and_batch():
+    a = dcpmla.mla_decode_workspace_size(64, 64, 148)
+    b = dcpmla.mla_decode_workspace_size(64, 64, 296)
+    c = dcpmla.mla_decode_workspace_size(128, 64, 148)
+    assert 256 < a < b and a < c
+    # (G + B) slots of H x 512 fp32 plus LSEs plus the 256-byte header
+    assert a >= 256 + (148 + 64) * 64 * 513 * 4
+    s = dcpmla.mla_decode_workspace_size(128, 64, 148, topk=2048)
+    assert s >= 256 + 128 * 64 * 513 * 4
+
+
+def test_workspace_size_rejects_bad_arguments():
+    L = dcpmla.lib()
+    n = ctypes.c_size_t(0)
+    assert L.mla_decode_workspace_size(-1, 64, 1, 0, ctypes.byref(n)) == EINVAL
+    assert L.mla_decode_workspace_size(1, 0, 1, 0, ctypes.byref(n)) == EINVAL
+    assert L.mla_decode_workspace_size(1, 65, 1, 0, ctypes.byref(n)) == EUNSUP
+    assert L.mla_decode_workspace_size(1, 8, 1, 0, None) == EINVAL
+
+
+FAKE = 0x10000          # aligned, never dereferenced: every call below fails before launch
+
+
+def _call(**kw):
+    a = dict(q=FAKE, kv=FAKE, kv_dtype=0, num_blocks=16, block_size=64, bt=FAKE, bt_stride=4,
+             lens=FAKE, batch=2, heads=8, shard=0, nshards=2, idx=None, topk=0, scale=0.07,
+             out=FAKE, lse=FAKE, ws=FAKE, ws_bytes=0, splits=4, impl=0, stream=None)
+    a.update(kw)
+    return dcpmla.lib().mla_decode_partial(
+        a["q"], a["kv"], a["kv_dtype"], a["num_blocks"], a["block_size"], a["bt"], a["bt_stride"],
+        a["lens"], a["batch"], a["heads"], a["shard"], a["nshards"], a["idx"], a["topk"],
+        a["scale"], a["out"], a["lse"], a["ws"], a["ws_bytes"], a["splits"], a["impl"],
+        a["stream"])
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(shard=2), EINVAL), (dict(shard=-1), EINVAL), (dict(nshards=0), EINVAL),
+    (dict(batch=-1), EINVAL), (dict(heads=0), EINVAL), (dict(heads=65), EUNSUP),
+    (dict(heads=128), EUNSUP), (dict(block_size=16), EUNSUP), (dict(block_size=0), EINVAL),
+    (dict(kv_dtype=2), EINVAL), (dict(num_blocks=0), EINVAL), (dict(bt_stride=0), EINVAL),
+    (dict(splits=-1), EINVAL), (dict(impl=7), EINVAL), (dict(scale=float("nan")), EINVAL),
+    (dict(scale=float("inf")), EINVAL), (dict(idx=FAKE, topk=0), EINVAL),
+    (dict(q=None), EINVAL), (dict(kv=None), EINVAL), (dict(bt=None), EINVAL),
+    (dict(lens=None), EINVAL), (dict(out=None), EINVAL), (dict(lse=None), EINVAL),
+    (dict(q=FAKE + 8), EALIGN), (dict(kv=FAKE + 4), EALIGN), (dict(out=FAKE + 4), EALIGN),
+    (dict(ws=None), EWS), (dict(ws_bytes=1024), EWS),
+])
+def test_partial_fails_closed(kw, code):
+    assert _call(**kw) == code
+
+
+def test_empty_batch_is_a_no_op():
+    assert _call(batch=0, q=None, kv=None, bt=None, lens=None, out=None, lse=None) == OK
+
+
+def test_merge_fails_closed():
+    L = dcpmla.lib()
+    assert L.dcp_merge(FAKE, FAKE, 0, 1, 8, FAKE, None, None) == EINVAL
+    assert L.dcp_merge(FAKE, FAKE, 2, -1, 8, FAKE, None, None) == EINVAL
+    assert L.dcp_merge(FAKE, FAKE, 2, 1, 0, FAKE, None, None) == EINVAL
+    assert L.dcp_merge(None, FAKE, 2, 1, 8, FAKE, None, None) == EINVAL
+    assert L.dcp_merge(FAKE, FAKE, 2, 1, 8, None, None, None) == EINVAL
+    assert L.dcp_merge(FAKE + 4, FAKE, 2, 1, 8, FAKE, None, None) == EALIGN
+    assert L.dcp_merge(FAKE, FAKE, 2, 0, 8, FAKE, None, None) == OK
+
+
+def test_head_envelope_matches_the_page_table():
+    with open(os.path.join(ROOT, "tests", "golden", "head_envelope.json")) as f:
+        g = json.load(f)
+    for row in g["rows"]:
+        assert row["local"] == g["global_heads"] // g["tp"]
+        assert row["gathered"] == row["local"] * row["dcp"]
+        assert dcpmla.padded_heads(row["local"]) == row["local_pad"]
+        assert dcpmla.padded_heads(row["gathered"]) == row["gathered_pad"]

@@ -1,0 +1,250 @@
+"""GPU-vs-oracle parity of the whole emulated DCP step, through the C ABI.
+
+Tolerances (stated by the target, applied to every shard's partials and to the
+merged result): bf16 cache max|dO| <= 2e-3 * max|O| and |dLSE| <= 1e-4; fp8
+cache max|dO| <= 2e-2 * max|O| and |dLSE| <= 1e-3 (the LSE bound for fp8 is a
+reading: the target states none).  Empty shards must return exactly (0, -inf).
+Addressing and sparse selection are checked bit-exactly with id-coded rows.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from long_context_decode_mla_b200 import dcpmla
+from long_context_decode_mla_b200 import workload as wl
+
+pytestmark = pytest.mark.gpu
+
+TOL = {"bf16": (2e-3, 1e-4), "fp8": (2e-2, 1e-3)}
+IMPLS = ["simt", "auto"]
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    dcpmla.lib()
+    torch.cuda.set_device(0)
+
+
+def _run(prob, impl="auto", num_splits=0, streams=None):
+    dp = prob.to("cuda")
+    topk = 0 if prob.sparse_idx is None else prob.sparse_idx.shape[1]
+    dec = dcpmla.DcpDecoder(prob.batch, prob.heads, prob.num_shards, topk=topk,
+                            num_splits=num_splits, impl=impl, streams=streams)
+    dec.step(dp)
+    torch.cuda.synchronize()
+    assert dec.flags() == 0
+    return (dec.partials.double().cpu().numpy(), dec.lses.double().cpu().numpy(),
+            dec.out.double().cpu().numpy(), dec.out_lse.double().cpu().numpy())
+
+
+def _oracle(prob, batch_ids=None):
+    ni = prob.numpy_inputs()
+    return oracle.dcp_decode(ni["q"], ni["kv_cache"], ni["kv_dtype"], ni["block_tables"],
+                             ni["seq_lens"], ni["num_shards"], ni["softmax_scale"],
+                             ni["sparse_idx"], ni["block_size"], batch_ids)
+
+
+def _compare(o, l, o_ref, l_ref, kv_dtype, what):
+    rel_o, abs_l = TOL[kv_dtype]
+    fin = np.isfinite(l_ref)
+    assert np.array_equal(fin, np.isfinite(l)), f"{what}: -inf pattern differs"
+    assert np.all(np.isneginf(l[~fin])), f"{what}: empty rows must have LSE -inf"
+    empty_rows = ~fin
+    assert not o[empty_rows].any(), f"{what}: empty rows must have O == 0"
+    if not fin.any():
+        return 0.0, 0.0
+    scale = np.abs(o_ref).max()
+    eo = np.abs(o - o_ref).max() / scale
+    el = np.abs(l[fin] - l_ref[fin]).max()
+    assert eo <= rel_o, f"{what}: max|dO|/max|O| = {eo:.3g} > {rel_o}"
+    assert el <= abs_l, f"{what}: max|dLSE| = {el:.3g} > {abs_l}"
+    return eo, el
+
+
+def _check_problem(prob, impl="auto", batch_ids=None, num_splits=0, streams=None):
+    parts, lses, out, lse = _run(prob, impl, num_splits, streams)
+    rp, rl, ro, rlse = _oracle(prob, batch_ids)
+    ids = list(range(prob.batch)) if batch_ids is None else list(batch_ids)
+    for s in range(prob.num_shards):
+        _compare(parts[s, ids], lses[s, ids], rp[s], rl[s], prob.kv_dtype, f"shard {s}")
+    return _compare(out[ids], lse[ids], ro, rlse, prob.kv_dtype, "merged")
+
+
+# --------------------------------------------------------------- small ------
+
+@pytest.mark.parametrize("impl", IMPLS)
+@pytest.mark.parametrize("N", [1, 2, 4, 8])
+def test_tiny_config(impl, N):
+    _check_problem(wl.make_problem("tiny", num_shards=N), impl)
+
+
+@pytest.mark.parametrize("impl", IMPLS)
+@pytest.mark.parametrize("kv_dtype", ["bf16", "fp8"])
+@pytest.mark.parametrize("N", [1, 3, 8])
+def test_ragged_lengths_and_empty_shards(impl, kv_dtype, N):
+    lens = [0, 1, N - 1, N, 63, 64, 65, 130, 1000, 4097]
+    prob = wl.make_problem("dense", num_shards=N, batch=len(lens), heads=64, seq_len=lens,
+                           kv_dtype=kv_dtype, seed=77)
+    _check_problem(prob, impl)
+
+
+@pytest.mark.parametrize("impl", IMPLS)
+@pytest.mark.parametrize("heads", [1, 8, 17, 64])
+def test_head_counts(impl, heads):
+    prob = wl.make_problem("dense", num_shards=2, batch=3, heads=heads, seq_len=[700, 64, 3],
+                           seed=5)
+    _check_problem(prob, impl)
+
+
+@pytest.mark.parametrize("impl", IMPLS)
+@pytest.mark.parametrize("splits", [1, 3, 148, 400])
+def test_split_counts_agree(impl, splits):
+    prob = wl.make_problem("agentic", num_shards=4, batch=5,
+                           seq_len=[9000, 200, 64, 20000, 5], seed=9)
+    _check_problem(prob, impl, num_splits=splits)
+
+
+@pytest.mark.parametrize("impl", IMPLS)
+@pytest.mark.parametrize("N", [1, 2, 8])
+def test_sparse_small(impl, N):
+    prob = wl.make_problem("sparse", num_shards=N, batch=6, seq_len=3000, topk=300, seed=4)
+    idx = prob.sparse_idx
+    idx[1] = -1                                   # empty list
+    idx[2, :] = (torch.arange(300) * N) % 3000    # everything on shard 0
+    idx[3, :150] = torch.arange(150) + 3000       # half out of range
+    _check_problem(prob, impl)
+
+
+# --------------------------------------------------------------- addressing -
+
+def _id_expect(ids):
+    return [sum((t >> d) & 1 for t in ids) for d in range(21)]
+
+
+@pytest.mark.parametrize("impl", IMPLS)
+@pytest.mark.parametrize("kv_dtype", ["bf16", "fp8"])
+@pytest.mark.parametrize("N", [1, 2, 3, 4, 8])
+def test_block_table_addressing_is_exact(impl, kv_dtype, N):
+    lens = [1, max(1, N - 1), N, 63, 64, 65, 1000, 5000]
+    prob = wl.id_coded_problem(lens, N, kv_dtype, heads=8, seed=N)
+    parts, lses, out, lse = _run(prob, impl)
+    for b, L in enumerate(lens):
+        for s in range(N):
+            ids = [t for t in range(L) if t % N == s]
+            if not ids:
+                assert np.all(np.isneginf(lses[s, b])) and not parts[s, b].any()
+                continue
+            n = len(ids)
+            assert np.abs(lses[s, b] - math.log(n)).max() < 1e-5
+            counts = np.rint(parts[s, b, :, :21] * n)
+            assert np.all(np.abs(parts[s, b, :, :21] * n - counts) < 1e-3)
+            assert all(counts[h].tolist() == _id_expect(ids) for h in range(8))
+            assert not parts[s, b, :, 21:].any()
+
+
+@pytest.mark.parametrize("impl", IMPLS)
+@pytest.mark.parametrize("N", [1, 2, 4, 8])
+def test_sparse_selection_is_exact(impl, N):
+    L = 6000
+    rng = np.random.default_rng(N)
+    idx = np.full((5, 512), -1, dtype=np.int32)
+    idx[0] = rng.choice(L, 512, replace=False)
+    idx[1, :64] = np.arange(64) * N + (N - 1)      # all on the last shard
+    idx[2, :4] = [L, -5, 10 * L, -1]               # nothing valid
+    idx[3, :300] = rng.choice(L, 300, replace=False)
+    idx[4, :] = rng.choice(L, 512, replace=False)
+    prob = wl.id_coded_problem([L] * 5, N, "fp8", heads=8, seed=N, sparse_idx=idx)
+    parts, lses, out, lse = _run(prob, impl)
+    for b in range(5):
+        for s in range(N):
+            ids = [int(t) for t in idx[b] if 0 <= t < L and t % N == s]
+            if not ids:
+                assert np.all(np.isneginf(lses[s, b])) and not parts[s, b].any()
+                continue
+            n = len(ids)
+            assert np.abs(lses[s, b] - math.log(n)).max() < 1e-5
+            counts = np.rint(parts[s, b, :, :21] * n)
+            assert all(counts[h].tolist() == _id_expect(ids) for h in range(8))
+    assert np.all(np.isneginf(lse[2])) and not out[2].any()
+
+
+# --------------------------------------------------------------- merge ------
+
+def test_dcp_merge_kernel_matches_oracle():
+    rng = np.random.default_rng(7)
+    N, B, H = 8, 5, 64
+    parts = rng.standard_normal((N, B, H, 512)).astype(np.float32)
+    lses = (rng.standard_normal((N, B, H)) * 4).astype(np.float32)
+    lses[2, 1] = -np.inf
+    lses[:, 3] = -np.inf                     # every shard empty
+    parts[:, 3] = 0
+    lses[1:, 4] = -np.inf                    # only shard 0 contributes
+    o = torch.empty(B, H, 512, device="cuda")
+    ol = torch.empty(B, H, device="cuda")
+    dcpmla.dcp_merge(torch.from_numpy(parts).cuda(), torch.from_numpy(lses).cuda(), o, ol)
+    torch.cuda.synchronize()
+    ro, rl = oracle.dcp_merge(parts.astype(np.float64), lses.astype(np.float64))
+    o, ol = o.double().cpu().numpy(), ol.double().cpu().numpy()
+    assert np.array_equal(np.isneginf(ol), np.isneginf(rl))
+    assert not o[3].any()
+    fin = np.isfinite(rl)
+    assert np.abs(o - ro).max() < 1e-5 * np.abs(ro).max()
+    assert np.abs(ol[fin] - rl[fin]).max() < 1e-5
+
+
+# --------------------------------------------------------------- faults -----
+
+def test_bad_block_entry_is_flagged_not_read():
+    prob = wl.make_problem("tiny", num_shards=2).to("cuda")
+    prob.block_tables[1, 0, 2] = 10 ** 6           # outside the pool
+    prob.block_tables[0, 0, 0] = -7
+    dec = dcpmla.DcpDecoder(1, 8, 2, impl="simt")
+    dec.step(prob)
+    torch.cuda.synchronize()
+    assert dec.flags() & dcpmla.FLAG_BAD_BLOCK
+
+
+def test_length_beyond_table_is_flagged():
+    prob = wl.make_problem("tiny", num_shards=2).to("cuda")
+    prob.seq_lens[0] = 10 ** 6                       # needs more blocks than the row has
+    dec = dcpmla.DcpDecoder(1, 8, 2, impl="simt")
+    dec.step(prob)
+    torch.cuda.synchronize()
+    assert dec.flags() & dcpmla.FLAG_BAD_LENGTH
+
+
+# --------------------------------------------------------------- full size --
+
+def _sample(prob, k=3):
+    lens = prob.seq_lens.tolist()
+    order = sorted(range(len(lens)), key=lambda b: lens[b])
+    return sorted(set([order[0], order[-1], order[len(order) // 2]][:k]))
+
+
+@pytest.mark.parametrize("N", [1, 2, 4, 8])
+def test_dense_config_full_size(N):
+    prob = wl.make_problem("dense", num_shards=N, kv_device="cuda")
+    _check_problem(prob, "auto", batch_ids=[0, 13, 31])
+
+
+@pytest.mark.parametrize("N", [1, 2, 4, 8])
+def test_agentic_config_full_size(N):
+    prob = wl.make_problem("agentic", num_shards=N, kv_device="cuda")
+    _check_problem(prob, "auto", batch_ids=_sample(prob))
+
+
+@pytest.mark.parametrize("N", [1, 2, 4, 8])
+def test_million_config_full_size(N):
+    prob = wl.make_problem("million", num_shards=N, kv_device="cuda")
+    streams = [torch.cuda.Stream() for _ in range(N)]
+    _check_problem(prob, "auto", batch_ids=[0], num_splits=max(1, 148 // N), streams=streams)
+
+
+@pytest.mark.parametrize("N", [1, 2, 4, 8])
+def test_sparse_config_full_size(N):
+    prob = wl.make_problem("sparse", num_shards=N, kv_device="cuda")
+    _check_problem(prob, "auto", batch_ids=[0, 64, 127])
