@@ -43,6 +43,7 @@ struct PartialParams {
   int* flags;                 // workspace flag word
   float* ws_o;                // [slots][H][512]
   float* ws_lse;              // [slots][H]
+  int* ws_list;               // sparse mode: per-CTA lists of selected local rows
   int num_ctas;               // G: CTAs sharing the dense tile space
 };
 
@@ -187,9 +188,14 @@ __host__ __device__ __forceinline__ size_t ws_o_offset() { return kWsHeader; }
 __host__ __device__ __forceinline__ size_t ws_lse_offset(long long slots, int heads) {
   return kWsHeader + (size_t)slots * heads * kVDim * sizeof(float);
 }
-__host__ __device__ __forceinline__ size_t ws_total(long long slots, int heads) {
+__host__ __device__ __forceinline__ size_t ws_list_offset(long long slots, int heads) {
   size_t lse_bytes = ((size_t)slots * heads * sizeof(float) + 255) & ~(size_t)255;
   return ws_lse_offset(slots, heads) + lse_bytes;
+}
+// `list_ints` = CTAs x index-list chunk for sparse mode, 0 for dense.
+__host__ __device__ __forceinline__ size_t ws_total(long long slots, int heads,
+                                                   long long list_ints = 0) {
+  return ws_list_offset(slots, heads) + (((size_t)list_ints * sizeof(int) + 255) & ~(size_t)255);
 }
 
 }  // namespace dcpmla

@@ -55,6 +55,14 @@ long long slots_for(int batch, int topk, int ctas) {
   return (long long)ctas + batch;
 }
 
+// Sparse mode: room for every CTA's list of selected local rows.
+long long list_ints_for(int batch, int topk, int ctas) {
+  if (topk <= 0) return 0;
+  const int parts = sparse_parts_for(batch, topk, ctas);
+  const long long chunk = (topk + parts - 1) / parts;
+  return (long long)batch * parts * chunk;
+}
+
 }  // namespace
 }  // namespace dcpmla
 
@@ -87,7 +95,7 @@ int mla_decode_workspace_size(int batch, int num_heads, int num_splits, int topk
   int ctas = 0;
   int rc = resolve_ctas(num_splits, &ctas);
   if (rc != DCPMLA_OK) return rc;
-  *bytes = ws_total(slots_for(batch, topk, ctas), num_heads);
+  *bytes = ws_total(slots_for(batch, topk, ctas), num_heads, list_ints_for(batch, topk, ctas));
   return DCPMLA_OK;
 }
 
@@ -110,7 +118,7 @@ int mla_decode_partial(const void* q, const void* kv_cache, int kv_dtype, int64_
   if (batch == 0) return DCPMLA_OK;
   if (!q || !kv_cache || !block_table || !seq_lens || !out_partial || !out_lse)
     return DCPMLA_ERR_INVALID_ARGUMENT;
-  if (!aligned16(q) || !aligned16(kv_cache) || !aligned16(out_partial) || !aligned16(out_lse) ||
+  if (!aligned16(q) || !aligned16(kv_cache) || !aligned16(out_partial) ||
       (workspace && !aligned16(workspace)))
     return DCPMLA_ERR_ALIGNMENT;
   const int eff_topk = sparse_idx ? topk : 0;
@@ -118,7 +126,9 @@ int mla_decode_partial(const void* q, const void* kv_cache, int kv_dtype, int64_
   int rc = resolve_ctas(num_splits, &ctas);
   if (rc != DCPMLA_OK) return rc;
   const long long slots = slots_for(batch, eff_topk, ctas);
-  if (!workspace || workspace_bytes < ws_total(slots, num_heads)) return DCPMLA_ERR_WORKSPACE;
+  const long long list_ints = list_ints_for(batch, eff_topk, ctas);
+  if (!workspace || workspace_bytes < ws_total(slots, num_heads, list_ints))
+    return DCPMLA_ERR_WORKSPACE;
 
   PartialParams p{};
   p.q = static_cast<const __nv_bfloat16*>(q);
@@ -141,6 +151,7 @@ int mla_decode_partial(const void* q, const void* kv_cache, int kv_dtype, int64_
   p.flags = reinterpret_cast<int*>(ws);
   p.ws_o = reinterpret_cast<float*>(ws + ws_o_offset());
   p.ws_lse = reinterpret_cast<float*>(ws + ws_lse_offset(slots, num_heads));
+  p.ws_list = list_ints ? reinterpret_cast<int*>(ws + ws_list_offset(slots, num_heads)) : nullptr;
   p.num_ctas = ctas;
 
   const bool tc_ok = tc_supports(p, kv_dtype);

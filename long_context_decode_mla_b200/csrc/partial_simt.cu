@@ -292,10 +292,18 @@ __global__ void __launch_bounds__(kThreads, 1) partial_simt_sparse(PartialParams
 }
 
 template <class K>
-cudaError_t launch(K kernel, int grid, const PartialParams& p, cudaStream_t st) {
+cudaError_t launch(K kernel, int slot, int grid, const PartialParams& p, cudaStream_t st) {
   const int smem = (int)sizeof(SimtSmem);
-  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  // Raise the shared-memory limit once per kernel and device (graph-capture safe afterwards).
+  static int configured[4][64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
+  if (!configured[slot][dev & 63]) {
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    configured[slot][dev & 63] = 1;
+  }
   kernel<<<grid, kThreads, smem, st>>>(p);
   return cudaGetLastError();
 }
@@ -305,11 +313,11 @@ cudaError_t launch(K kernel, int grid, const PartialParams& p, cudaStream_t st) 
 cudaError_t launch_partial_simt(const PartialParams& p, int kv_dtype, cudaStream_t st) {
   if (p.sparse_idx) {
     const int grid = p.batch * p.sparse_parts;
-    return kv_dtype == kKvBf16 ? launch(partial_simt_sparse<kKvBf16>, grid, p, st)
-                               : launch(partial_simt_sparse<kKvFp8>, grid, p, st);
+    return kv_dtype == kKvBf16 ? launch(partial_simt_sparse<kKvBf16>, 0, grid, p, st)
+                               : launch(partial_simt_sparse<kKvFp8>, 1, grid, p, st);
   }
-  return kv_dtype == kKvBf16 ? launch(partial_simt_dense<kKvBf16>, p.num_ctas, p, st)
-                             : launch(partial_simt_dense<kKvFp8>, p.num_ctas, p, st);
+  return kv_dtype == kKvBf16 ? launch(partial_simt_dense<kKvBf16>, 2, p.num_ctas, p, st)
+                             : launch(partial_simt_dense<kKvFp8>, 3, p.num_ctas, p, st);
 }
 
 int simt_sparse_chunk_max() { return kSparseChunkMax; }

@@ -1,13 +1,616 @@
-// Tensor-core (tcgen05 / TMEM) kernel for one shard's partial attention.
+// Tensor-core kernel (tcgen05 / TMEM, sm_100a) for one shard's partial
+// attention with its LSE.
+//
+// What it computes is the same as the CUDA-core kernel: for each request, the
+// softmax over this shard's tokens of scale * <q_h, k_t> (576 values) applied
+// to the first 512 values of the rows, plus LSE = ln sum_t exp(score)
+// ("GLM-5.2 vLLM Decode Context Parallelism", sections "See why vLLM 0.26.0
+// fails" and "Separate the backend merge from stable"; round-robin ownership
+// from "How vLLM Serves GLM-5.3 with Million-Token Contexts on 16 H200s",
+// "The core design").
+//
+// How (per CTA, one per SM, persistent over its slice of the tile space):
+//  * Q of the current request (64 heads padded, 576 bf16) sits in shared
+//    memory, 128-byte swizzled, as the A operand of S = Q K^T.
+//  * A tile is 128 local tokens (two cache blocks).  Its rows are brought into
+//    nine 16 KB shared-memory chunk slots (8 latent chunks of 64 values, then
+//    rope), swizzled for the tensor core.  bf16 rows are copied with
+//    cp.async; fp8 rows are read into registers, decoded (e4m3 * scale ->
+//    bf16) and stored, so raw fp8 never occupies shared memory.
+//  * S = Q K^T: 36 weight-stationary MMAs (M = 64 heads, N = 128 tokens,
+//    K = 16) into TMEM; the 2x2 data path puts head h at TMEM lane h for
+//    tokens 0..63 and lane 64 + h for tokens 64..127.
+//  * Four softmax warps (one TMEM lane each) run the online softmax in base 2
+//    with a lazily updated running max (the output is only rescaled when the
+//    max grows by more than 2^8), write P (bf16) into the rope slot, which
+//    the scores no longer need, and keep the running sum.
+//  * O += P V: 16 MMAs (M = 64, N = 256 dims, K = 16 tokens) reading V from
+//    the same chunk slots as an MN-major operand; O (64 x 512 fp32) stays in
+//    TMEM for the whole request and is normalised in the epilogue.
+//  * Slots are released per half of the PV step so the next tile's first
+//    chunks can be filled while the second half still runs.
+#include <cuda_fp8.h>
+#include <math_constants.h>
+
 #include "common.cuh"
 #include "kernels.h"
+#include "tc_ptx.cuh"
 
 namespace dcpmla {
+namespace {
 
-bool tc_supports(const PartialParams&, int) { return false; }
+constexpr int kThreads = 384;          // 12 warps: 4 softmax (thread 0 issues MMAs), 8 converters
+constexpr int kConvBase = 128;         // first converter thread
+constexpr int kConvThreads = 256;
+constexpr int kTileTok = 128;
+constexpr int kSlotBytes = 16384;
+constexpr int kNumSlots = 9;
+constexpr int kRopeSlot = 8;
+constexpr int kQBytes = 9 * 8192;
+constexpr int kMaxSeg = 128;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColS = 256;        // S: columns [256, 320); O: columns [0, 256)
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kRescaleThreshold = 8.f;
+constexpr int kFlagTimeout = 4;
 
-cudaError_t launch_partial_tc(const PartialParams&, int, cudaStream_t) {
-  return cudaErrorNotSupported;
+struct TcCtl {
+  uint64_t full[kNumSlots];
+  uint64_t empty[kNumSlots];
+  uint64_t q_full, q_empty, s_full, p_full, o_full;
+  uint32_t tmem_base;
+  int abort;
+  uint32_t row_mask[4];
+  float red[2][2][64];
+  float lred[2][64];
+  int nseg;
+  int sel_count;
+  int warp_sums[16];
+  Segment seg[kMaxSeg];
+};
+
+constexpr size_t kSmemBytes = kQBytes + (size_t)kNumSlots * kSlotBytes + sizeof(TcCtl) + 1024;
+
+struct SegView {
+  int b;
+  int row_begin;   // first local row (dense) or list offset (sparse)
+  int nrows;
+  int ntiles;
+  bool whole;
+};
+
+__device__ __forceinline__ uint32_t swz(int row, int unit) {
+  return (uint32_t)((row >> 3) * 1024 + (row & 7) * 128 + ((unit ^ (row & 7)) << 4));
 }
+
+__device__ __forceinline__ SegView seg_view(const PartialParams& p, const TcCtl& c, int k) {
+  SegView v;
+  if (p.sparse_idx) {
+    v.b = blockIdx.x / p.sparse_parts;
+    v.row_begin = 0;
+    v.nrows = c.sel_count;
+    v.whole = p.sparse_parts == 1;
+  } else {
+    const Segment s = c.seg[k];
+    v.b = s.b;
+    v.row_begin = s.t0 * kBlock;
+    v.nrows = min(s.n_rows, s.t1 * kBlock) - v.row_begin;
+    v.whole = s.t0 == 0 && s.t1 == s.nt;
+  }
+  v.ntiles = (v.nrows + kTileTok - 1) / kTileTok;
+  return v;
+}
+
+// Address of local tile row r of the segment, or nullptr if it is past the
+// end or its block-table entry is out of range (flagged).
+template <int KV>
+__device__ __forceinline__ const uint8_t* tile_row(const PartialParams& p, const SegView& v,
+                                                  const int* list, int tile, int r) {
+  constexpr int kRowBytes = KV == kKvBf16 ? kRowBytesBf16 : kRowBytesFp8;
+  const int i = tile * kTileTok + r;
+  if (i >= v.nrows) return nullptr;
+  const int j = p.sparse_idx ? list[i] : v.row_begin + i;   // written by this CTA: no __ldg
+  const int blk = tile_block(p, v.b, j >> 6);
+  if (blk < 0) return nullptr;
+  return p.kv + ((size_t)blk * kBlock + (j & 63)) * kRowBytes;
+}
+
+// 16 e4m3 codes times `sc` -> 16 bf16 (two 16-byte units, dims in order).
+__device__ __forceinline__ void decode16(const uint4 v, float sc, uint4& lo, uint4& hi) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t o[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+#pragma unroll
+    for (int hw = 0; hw < 2; ++hw) {
+      const __nv_fp8x2_storage_t pair = (__nv_fp8x2_storage_t)((w[i] >> (16 * hw)) & 0xFFFFu);
+      const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3);
+      __half2 h2;
+      *reinterpret_cast<__half2_raw*>(&h2) = hr;
+      const float2 f = __half22float2(h2);
+      const __nv_bfloat162 b2 = __floats2bfloat162_rn(f.x * sc, f.y * sc);
+      o[2 * i + hw] = *reinterpret_cast<const uint32_t*>(&b2);
+    }
+  }
+  lo = make_uint4(o[0], o[1], o[2], o[3]);
+  hi = make_uint4(o[4], o[5], o[6], o[7]);
+}
+
+// ------------------------------------------------------------- segments ----
+
+// Collect this CTA's dense segments number [first, first + kMaxSeg) in request
+// order into c.seg.  Returns the total number of segments of the CTA.
+__device__ int collect_segments(const PartialParams& p, int lo, int hi, int first, TcCtl& c) {
+  int off = 0, seen = 0;
+  for (int base = 0; base < p.batch && off < hi; base += blockDim.x) {
+    const int b = base + threadIdx.x;
+    int n = 0, nt = 0;
+    if (b < p.batch) nt = request_tiles(p, b, &n);
+    int tot;
+    const int start = off + block_exclusive_scan(nt, c.warp_sums, &tot);
+    const int inter = (nt > 0 && start < hi && start + nt > lo) ? 1 : 0;
+    int tot_inter;
+    const int idx = seen + block_exclusive_scan(inter, c.warp_sums, &tot_inter);
+    if (inter && idx >= first && idx < first + kMaxSeg) {
+      Segment s;
+      s.b = b;
+      s.t0 = max(lo, start) - start;
+      s.t1 = min(hi, start + nt) - start;
+      s.n_rows = n;
+      s.nt = nt;
+      c.seg[idx - first] = s;
+    }
+    seen += tot_inter;
+    off += tot;
+  }
+  __syncthreads();
+  return seen;
+}
+
+// Sparse mode: this CTA's chunk of the index list, filtered to the positions
+// this shard owns, as local indices (in list order) into `list`.
+__device__ int compact_sparse(const PartialParams& p, int* list, TcCtl& c) {
+  const int b = blockIdx.x / p.sparse_parts, part = blockIdx.x % p.sparse_parts;
+  const int chunk = (p.topk + p.sparse_parts - 1) / p.sparse_parts;
+  const int i0 = part * chunk, i1 = min(p.topk, i0 + chunk);
+  int L = __ldg(p.seq_lens + b);
+  if (L < 0) {
+    if (threadIdx.x == 0 && p.flags) atomicOr(p.flags, kFlagBadLength);
+    L = 0;
+  }
+  int count = 0;
+  for (int base = i0; base < i1; base += blockDim.x) {
+    const int i = base + threadIdx.x;
+    int sel = 0, j = 0;
+    if (i < i1) {
+      const int t = __ldg(p.sparse_idx + (size_t)b * p.topk + i);
+      if (t >= 0 && t < L && t % p.nshards == p.shard) {
+        j = t / p.nshards;
+        if ((j >> 6) < p.bt_stride) {
+          sel = 1;
+        } else if (p.flags) {
+          atomicOr(p.flags, kFlagBadLength);
+        }
+      }
+    }
+    int tot;
+    const int pos = count + block_exclusive_scan(sel, c.warp_sums, &tot);
+    if (sel) list[pos] = j;
+    count += tot;
+  }
+  __syncthreads();
+  return count;
+}
+
+// ------------------------------------------------------------- roles -------
+
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, TcCtl& c) {
+  return ptx::mbar_wait(bar, parity, &c.abort);
+}
+
+// MMA issue (one thread): S = Q K^T for tile t.
+__device__ __forceinline__ bool issue_qk(TcCtl& c, uint32_t q0, uint32_t s0, uint32_t tau) {
+  constexpr uint32_t kIdQK = ptx::idesc_bf16(64, 128, false);
+  for (int s = 0; s < kNumSlots; ++s)
+    if (!wait_or_abort(&c.full[s], tau & 1, c)) return false;
+  ptx::tc_fence_after();
+#pragma unroll 4
+  for (int ks = 0; ks < 36; ++ks) {
+    const uint64_t a = ptx::sdesc_sw128(q0 + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024);
+    const uint64_t b = ptx::sdesc_sw128(s0 + (ks >> 2) * kSlotBytes + (ks & 3) * 32, 16, 1024);
+    ptx::mma_ws_f16(c.tmem_base + kColS, a, b, kIdQK, ks > 0);
+  }
+  ptx::mma_commit(&c.s_full);
+  return true;
+}
+
+// MMA issue (one thread): O (+)= P V for tile t; releases the slots per half.
+__device__ __forceinline__ void issue_pv(TcCtl& c, uint32_t s0, bool first_tile) {
+  constexpr uint32_t kIdPV = ptx::idesc_bf16(64, 256, true);
+  const uint32_t pbase = s0 + kRopeSlot * kSlotBytes;
+#pragma unroll
+  for (int hf = 0; hf < 2; ++hf) {
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+      const uint64_t a = ptx::sdesc_sw128(pbase + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
+      const uint64_t b = ptx::sdesc_sw128(s0 + 4 * hf * kSlotBytes + kk * 2048, kSlotBytes, 1024);
+      ptx::mma_ws_f16(c.tmem_base + hf * 128, a, b, kIdPV, (!first_tile || kk > 0) ? 1u : 0u);
+    }
+    if (hf == 0) {
+      for (int s = 0; s < 4; ++s) ptx::mma_commit(&c.empty[s]);
+    } else {
+      for (int s = 4; s < kNumSlots; ++s) ptx::mma_commit(&c.empty[s]);
+    }
+  }
+}
+
+// Online softmax, P, and the epilogue (128 threads, one TMEM lane each).
+__device__ void softmax_role(const PartialParams& p, TcCtl& c, uint8_t* sq, uint8_t* sslot,
+                             int nseg, uint32_t& tau, uint32_t& sigma) {
+  const int L = threadIdx.x;                 // 0..127
+  const bool issuer = L == 0;
+  const uint32_t q0 = ptx::smem_addr(sq), s0 = ptx::smem_addr(sslot);
+  const int h = L & 63, half = L >> 6;
+  const int warp = L >> 5;
+  const uint32_t lane_base = c.tmem_base + ((uint32_t)(warp * 32) << 16);
+  const float sl2 = p.scale * kLog2e;
+  uint8_t* pslot = sslot + kRopeSlot * kSlotBytes + half * 8192;
+  for (int k = 0; k < nseg; ++k) {
+    const SegView v = seg_view(p, c, k);
+    const size_t slot = v.whole ? (size_t)v.b
+                                : (p.sparse_idx ? (size_t)blockIdx.x : (size_t)blockIdx.x + v.b);
+    float* o_base = (v.whole ? p.out : p.ws_o) + (slot * p.heads + h) * kVDim;
+    float* l_base = (v.whole ? p.out_lse : p.ws_lse) + slot * p.heads + h;
+    if (v.ntiles == 0) {
+      if (h < p.heads) {
+        float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int i = half; i < kVDim / 4; i += 2) reinterpret_cast<float4*>(o_base)[i] = z;
+        if (half == 0) *l_base = -CUDART_INF_F;
+      }
+      continue;
+    }
+    float m_used = -CUDART_INF_F, l = 0.f;
+    // The issuing thread never leaves before the warp re-converges: on a
+    // failed wait it stops issuing, and the whole group then fails together
+    // on the scores barrier that can no longer complete.
+    bool issuing = issuer && wait_or_abort(&c.q_full, sigma & 1, c);
+    for (int t = 0; t < v.ntiles; ++t, ++tau) {
+      if (issuing) {
+        issuing = issue_qk(c, q0, s0, tau);
+        if (issuing && t == v.ntiles - 1) ptx::mma_commit(&c.q_empty);
+      }
+      __syncwarp();
+      if (!wait_or_abort(&c.s_full, tau & 1, c)) return;
+      if (!wait_or_abort(&c.full[kRopeSlot], tau & 1, c)) return;
+      __syncwarp();
+      ptx::tc_fence_after();
+      uint32_t sa[32], sb[32];
+      ptx::tmem_ld32(lane_base + kColS, sa);
+      ptx::tmem_ld32(lane_base + kColS + 32, sb);
+      ptx::tmem_wait_ld();
+      const uint32_t mw0 = c.row_mask[half * 2], mw1 = c.row_mask[half * 2 + 1];
+      float x[64];
+      float mloc = -CUDART_INF_F;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        x[j] = ((mw0 >> j) & 1u) ? __uint_as_float(sa[j]) * sl2 : -CUDART_INF_F;
+        x[32 + j] = ((mw1 >> j) & 1u) ? __uint_as_float(sb[j]) * sl2 : -CUDART_INF_F;
+        mloc = fmaxf(mloc, fmaxf(x[j], x[32 + j]));
+      }
+      const int par = tau & 1;
+      c.red[par][half][h] = mloc;
+      ptx::named_bar(1, 128);
+      const float mnew = fmaxf(mloc, c.red[par][half ^ 1][h]);
+      // Lazy rescale.  The TMEM loads/stores below are warp-collective, so the
+      // decision is made per warp: if any head of the warp needs a new max,
+      // every lane moves to max(m_used, mnew).  The partner warp (the other
+      // token half) holds the same 32 heads and decides identically.
+      const bool first = m_used == -CUDART_INF_F;
+      const bool need = !first && mnew > m_used + kRescaleThreshold;
+      const bool any_need = __any_sync(0xffffffffu, need);
+      float alpha = 1.f;
+      if (first) {
+        m_used = mnew;
+      } else if (any_need) {
+        const float m2 = fmaxf(m_used, mnew);
+        alpha = exp2f(m_used - m2);
+        m_used = m2;
+        l *= alpha;
+      }
+      if (any_need) {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          uint32_t r[32];
+          const uint32_t addr = lane_base + (q >> 2) * 128 + (q & 3) * 32;
+          ptx::tmem_ld32(addr, r);
+          ptx::tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+          ptx::tmem_st32(addr, r);
+        }
+        ptx::tmem_wait_st();
+      }
+      float sum = 0.f;
+      uint32_t pk[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const float p0 = m_used == -CUDART_INF_F ? 0.f : exp2f(x[2 * j] - m_used);
+        const float p1 = m_used == -CUDART_INF_F ? 0.f : exp2f(x[2 * j + 1] - m_used);
+        sum += p0 + p1;
+        const __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
+        pk[j] = *reinterpret_cast<const uint32_t*>(&b2);
+      }
+      l += sum;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        *reinterpret_cast<uint4*>(pslot + swz(h, u)) =
+            make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+      }
+      ptx::fence_proxy_async();
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(&c.p_full);
+      if (issuing) {
+        issuing = wait_or_abort(&c.p_full, tau & 1, c);
+        if (issuing) {
+          ptx::tc_fence_after();
+          issue_pv(c, s0, t == 0);
+          if (t == v.ntiles - 1) ptx::mma_commit(&c.o_full);
+        }
+      }
+      __syncwarp();
+    }
+    // epilogue: O / l and the LSE
+    if (!wait_or_abort(&c.o_full, sigma & 1, c)) return;
+    __syncwarp();
+    ptx::tc_fence_after();
+    c.lred[half][h] = l;
+    ptx::named_bar(1, 128);
+    const float ltot = l + c.lred[half ^ 1][h];
+    const float inv = ltot > 0.f ? 1.f / ltot : 0.f;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      uint32_t r[32];
+      ptx::tmem_ld32(lane_base + (q >> 2) * 128 + (q & 3) * 32, r);
+      ptx::tmem_wait_ld();
+      if (h < p.heads) {
+        float4* dst = reinterpret_cast<float4*>(o_base + (q >> 2) * 256 + half * 128 + (q & 3) * 32);
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          dst[e] = make_float4(__uint_as_float(r[4 * e]) * inv, __uint_as_float(r[4 * e + 1]) * inv,
+                               __uint_as_float(r[4 * e + 2]) * inv, __uint_as_float(r[4 * e + 3]) * inv);
+      }
+    }
+    if (h < p.heads && half == 0)
+      *l_base = ltot > 0.f ? (m_used + log2f(ltot)) * kLn2 : -CUDART_INF_F;
+    ptx::tc_fence_before();
+    ptx::named_bar(1, 128);
+    ++sigma;
+  }
+}
+
+// Fills Q and the chunk slots (256 threads).
+template <int KV>
+__device__ void convert_role(const PartialParams& p, TcCtl& c, uint8_t* sq, uint8_t* sslot,
+                             const int* list, int nseg, uint32_t& tau, uint32_t& sigma) {
+  const int ct = threadIdx.x - kConvBase;      // 0..255
+  const int cw = ct >> 5, cl = ct & 31;
+  const uint32_t q0 = ptx::smem_addr(sq), s0 = ptx::smem_addr(sslot);
+  for (int k = 0; k < nseg; ++k) {
+    const SegView v = seg_view(p, c, k);
+    if (v.ntiles == 0) continue;
+    // ---- Q of request b: 64 rows x 72 units, heads >= H zero-filled ----
+    if (sigma > 0 && !wait_or_abort(&c.q_empty, (sigma - 1) & 1, c)) return;
+    const uint8_t* qb = reinterpret_cast<const uint8_t*>(p.q + (size_t)v.b * p.heads * kHeadDim);
+    for (int i = 0; i < 18; ++i) {
+      const int U = i * kConvThreads + ct;
+      const int row = U / 72, u = U % 72;
+      const bool ok = row < p.heads;
+      ptx::cp_async16(q0 + (u >> 3) * 8192 + swz(row, u & 7),
+                      ok ? qb + ((size_t)row * kHeadDim + u * 8) * 2 : qb, ok ? 16u : 0u);
+    }
+    ptx::cp_async_arrive(&c.q_full);
+    for (int t = 0; t < v.ntiles; ++t, ++tau) {
+      if constexpr (KV == kKvFp8) {
+        // rows 16 j + 2 cw + rsel, latent units u0 (half 0) and 16 + u0 (half 1)
+        const int rsel = (cl >> 2) & 1;
+        const int u0 = (cl & 3) + 4 * (cl >> 3);
+        uint4 c0[8], c1[8];
+        float sc0[8], sc1[8];
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) {
+          const int r = 16 * jj + 2 * cw + rsel;
+          const uint8_t* row = tile_row<KV>(p, v, list, t, r);
+          if (row) {
+            c0[jj] = __ldg(reinterpret_cast<const uint4*>(row) + u0);
+            c1[jj] = __ldg(reinterpret_cast<const uint4*>(row) + 16 + u0);
+            sc0[jj] = __ldg(reinterpret_cast<const float*>(row + 512) + (u0 >> 3));
+            sc1[jj] = __ldg(reinterpret_cast<const float*>(row + 512) + 2 + (u0 >> 3));
+          } else {
+            c0[jj] = c1[jj] = make_uint4(0, 0, 0, 0);
+            sc0[jj] = sc1[jj] = 0.f;
+          }
+        }
+        if (tau > 0)
+          for (int s = 0; s < 4; ++s)
+            if (!wait_or_abort(&c.empty[s], (tau - 1) & 1, c)) return;
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) {
+          const int r = 16 * jj + 2 * cw + rsel;
+          uint4 lo, hi;
+          decode16(c0[jj], sc0[jj], lo, hi);
+          uint8_t* dst = sslot + (u0 >> 2) * kSlotBytes;
+          *reinterpret_cast<uint4*>(dst + swz(r, (u0 & 3) * 2)) = lo;
+          *reinterpret_cast<uint4*>(dst + swz(r, (u0 & 3) * 2 + 1)) = hi;
+        }
+        ptx::fence_proxy_async();
+        for (int s = 0; s < 4; ++s) ptx::mbar_arrive(&c.full[s]);
+        if (tau > 0)
+          for (int s = 4; s < kNumSlots; ++s)
+            if (!wait_or_abort(&c.empty[s], (tau - 1) & 1, c)) return;
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) {
+          const int r = 16 * jj + 2 * cw + rsel;
+          uint4 lo, hi;
+          decode16(c1[jj], sc1[jj], lo, hi);
+          uint8_t* dst = sslot + (4 + (u0 >> 2)) * kSlotBytes;
+          *reinterpret_cast<uint4*>(dst + swz(r, (u0 & 3) * 2)) = lo;
+          *reinterpret_cast<uint4*>(dst + swz(r, (u0 & 3) * 2 + 1)) = hi;
+        }
+        // rope: 128 rows x 8 units of bf16, copied as is
+        for (int i = 0; i < 4; ++i) {
+          const int U = i * kConvThreads + ct;
+          const int r = U >> 3, u = U & 7;
+          const uint8_t* row = tile_row<KV>(p, v, list, t, r);
+          ptx::cp_async16(s0 + kRopeSlot * kSlotBytes + swz(r, u), row ? row + 528 + 16 * u : p.kv,
+                          row ? 16u : 0u);
+        }
+      } else {
+        if (tau > 0)
+          for (int s = 0; s < kNumSlots; ++s)
+            if (!wait_or_abort(&c.empty[s], (tau - 1) & 1, c)) return;
+        for (int i = 0; i < 36; ++i) {
+          const int U = i * kConvThreads + ct;
+          const int r = U / 72, u = U % 72;
+          const uint8_t* row = tile_row<KV>(p, v, list, t, r);
+          ptx::cp_async16(s0 + (u >> 3) * kSlotBytes + swz(r, u & 7), row ? row + 16 * u : p.kv,
+                          row ? 16u : 0u);
+        }
+      }
+      // valid-row mask of the tile, published with the rope slot
+      if (ct < 128) {
+        const bool ok = tile_row<KV>(p, v, list, t, ct) != nullptr;
+        const uint32_t m = __ballot_sync(0xffffffffu, ok);
+        if (cl == 0) c.row_mask[cw] = m;
+      }
+      ptx::fence_proxy_async();
+      if constexpr (KV == kKvFp8) {
+        for (int s = 4; s < 8; ++s) ptx::mbar_arrive(&c.full[s]);
+        ptx::cp_async_arrive(&c.full[kRopeSlot]);
+      } else {
+        for (int s = 0; s < kNumSlots; ++s) ptx::cp_async_arrive(&c.full[s]);
+      }
+      if (ct < 128 && cl == 0) ptx::mbar_arrive(&c.full[kRopeSlot]);
+    }
+    ++sigma;
+  }
+}
+
+template <int KV>
+__global__ void __launch_bounds__(kThreads, 1) partial_tc_kernel(PartialParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sq = base;
+  uint8_t* sslot = base + kQBytes;
+  TcCtl& c = *reinterpret_cast<TcCtl*>(base + kQBytes + kNumSlots * kSlotBytes);
+  const int warp = threadIdx.x >> 5;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kNumSlots; ++s) {
+      // fp8: 256 converter arrivals on every slot; the rope slot also gets the
+      // 4 row-mask writers.  bf16: the same counts.
+      ptx::mbar_init(&c.full[s], kConvThreads + (s == kRopeSlot ? 4 : 0));
+      ptx::mbar_init(&c.empty[s], 1);
+    }
+    ptx::mbar_init(&c.q_full, kConvThreads);
+    ptx::mbar_init(&c.q_empty, 1);
+    ptx::mbar_init(&c.s_full, 1);
+    ptx::mbar_init(&c.p_full, 128);
+    ptx::mbar_init(&c.o_full, 1);
+    c.abort = 0;
+  }
+  if (warp == 0) ptx::tmem_alloc(&c.tmem_base, kTmemCols);
+  ptx::fence_proxy_async();
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+
+  const int* list = nullptr;
+  int lo = 0, hi = 0;
+  if (p.sparse_idx) {
+    const int chunk = (p.topk + p.sparse_parts - 1) / p.sparse_parts;
+    int* my_list = p.ws_list + (size_t)blockIdx.x * chunk;
+    const int n = blockIdx.x < p.batch * p.sparse_parts ? compact_sparse(p, my_list, c) : 0;
+    if (threadIdx.x == 0) c.sel_count = n;
+    list = my_list;
+  } else {
+    const int T = total_tiles(p, c.warp_sums);
+    const int tpc = T > 0 ? (T + p.num_ctas - 1) / p.num_ctas : 0;
+    lo = blockIdx.x * tpc;
+    hi = min(T, lo + tpc);
+  }
+  __syncthreads();
+
+  uint32_t tau = 0, sigma = 0;
+  uint32_t tau_issuer = 0, sigma_issuer = 0;
+  int first = 0;
+  while (true) {
+    int nseg, total;
+    if (p.sparse_idx) {
+      nseg = total = 1;
+    } else {
+      total = lo < hi ? collect_segments(p, lo, hi, first, c) : 0;
+      nseg = min(kMaxSeg, total - first);
+    }
+    if (nseg <= 0) break;
+    if (warp < 4) {
+      softmax_role(p, c, sq, sslot, nseg, tau, sigma);
+      tau_issuer = tau;
+      sigma_issuer = sigma;
+    } else {
+      convert_role<KV>(p, c, sq, sslot, list, nseg, tau, sigma);
+    }
+    __syncthreads();
+    if (c.abort) break;
+    first += kMaxSeg;
+    if (p.sparse_idx || total <= first) break;
+  }
+  // Drain: every tcgen05.commit arrives on its mbarrier asynchronously.  The
+  // last tile's slot releases and the last segment's Q release are never
+  // waited on by the pipeline, so wait for them here; otherwise an arrival
+  // could land after this CTA exits, on the barriers the next CTA on this SM
+  // has just initialised at the same shared-memory offsets.
+  if (threadIdx.x == 0) {
+    if (tau_issuer > 0)
+      for (int s = 0; s < kNumSlots; ++s) wait_or_abort(&c.empty[s], (tau_issuer - 1) & 1, c);
+    if (sigma_issuer > 0) wait_or_abort(&c.q_empty, (sigma_issuer - 1) & 1, c);
+  }
+  if (c.abort && threadIdx.x == 0 && p.flags) atomicOr(p.flags, kFlagTimeout);
+  ptx::cp_async_wait_all();
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  if (warp == 0) ptx::tmem_dealloc(c.tmem_base, kTmemCols);
+}
+
+}  // namespace
+
+bool tc_supports(const PartialParams& p, int kv_dtype) {
+  (void)kv_dtype;
+  return p.heads >= 1 && p.heads <= kMaxHeads;
+}
+
+cudaError_t launch_partial_tc(const PartialParams& p, int kv_dtype, cudaStream_t st) {
+  const int grid = p.sparse_idx ? p.batch * p.sparse_parts : p.num_ctas;
+  const int smem = (int)kSmemBytes;
+  auto kernel = kv_dtype == kKvBf16 ? partial_tc_kernel<kKvBf16> : partial_tc_kernel<kKvFp8>;
+  // Raise the shared-memory limit once per kernel and device, so that later
+  // launches (including ones captured into a CUDA graph) are plain launches.
+  static int configured[2][64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  int& done = configured[kv_dtype == kKvBf16 ? 0 : 1][dev & 63];
+  if (!done) {
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    done = 1;
+  }
+  kernel<<<grid, kThreads, smem, st>>>(p);
+  return cudaGetLastError();
+}
+
+size_t tc_smem_bytes() { return kSmemBytes; }
 
 }  // namespace dcpmla

@@ -162,7 +162,7 @@ class DcpDecoder:
             v |= int(w[:4].view(torch.int32).item())
         return v
 
-    def step(self, prob, stream=None):
+    def step(self, prob, stream=None, merge=True):
         """All N shard partials, then the merge, for a DecodeProblem on the GPU."""
         base = torch.cuda.current_stream() if stream is None else stream
         streams = self.streams
@@ -183,5 +183,24 @@ class DcpDecoder:
                 e2 = torch.cuda.Event()
                 e2.record(st)
                 base.wait_event(e2)
-        dcp_merge(self.partials, self.lses, self.out, self.out_lse, base)
+        if merge:
+            dcp_merge(self.partials, self.lses, self.out, self.out_lse, base)
         return self.out, self.out_lse
+
+    def capture(self, prob, merge=True):
+        """Record one whole step (or only the shard partials) into a CUDA graph.
+
+        The graph reads the problem's buffers in place: refill ``prob.q``,
+        ``prob.seq_lens``, ``prob.block_tables`` (and ``prob.sparse_idx``) and
+        call ``graph.replay()`` for the next step; results land in
+        ``self.out`` / ``self.out_lse`` (and ``self.partials`` / ``self.lses``).
+        """
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            self.step(prob, side, merge)         # resolve lazy state before capture
+        torch.cuda.current_stream().wait_stream(side)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=side):
+            self.step(prob, side, merge)
+        return g
