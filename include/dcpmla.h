@@ -77,6 +77,8 @@ extern "C" {
 /* Bits the kernels OR into the workspace flag word (int32 at byte 0). */
 #define DCPMLA_FLAG_BAD_BLOCK 1      /* a block-table entry was outside [0, num_blocks) */
 #define DCPMLA_FLAG_BAD_LENGTH 2     /* a length was negative or needs more blocks than the table row has */
+#define DCPMLA_FLAG_TIMEOUT 4        /* a tensor-core kernel pipeline wait gave up (about 2 s); outputs invalid */
+#define DCPMLA_FLAG_RANGE 8          /* a q or cache value beyond +-65504 was clamped by the fp16 tensor-core path */
 
 #define DCPMLA_HEAD_DIM 576          /* 512 latent + 64 rope */
 #define DCPMLA_V_DIM 512

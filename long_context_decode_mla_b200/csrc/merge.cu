@@ -75,11 +75,14 @@ __global__ void __launch_bounds__(kMergeWarps * 32) dcp_merge_kernel(
              out_lse ? out_lse + row : nullptr);
 }
 
-// Combine of the split pieces of each request (grid: one CTA per request).
+// Combine of the split pieces of each request.  Grid: one CTA per
+// (request, group of 8 heads), one warp per head.
 __global__ void __launch_bounds__(256) split_combine_kernel(PartialParams p) {
   __shared__ int warp_sums[8];
-  const int b = blockIdx.x;
-  const int warp = threadIdx.x >> 5;
+  __shared__ int sh_start, sh_nt;
+  const int hgroups = (p.heads + 7) / 8;
+  const int b = blockIdx.x / hgroups;
+  const int h = (blockIdx.x % hgroups) * 8 + (threadIdx.x >> 5);
   int first_slot, count;
   if (p.sparse_idx) {
     if (p.sparse_parts == 1) return;          // written directly by the partial kernel
@@ -87,7 +90,6 @@ __global__ void __launch_bounds__(256) split_combine_kernel(PartialParams p) {
     count = p.sparse_parts;
   } else {
     // start tile of request b and the total, with the partial kernel's schedule
-    __shared__ int sh_start, sh_nt;
     int T = 0;
     for (int base = 0; base < p.batch; base += blockDim.x) {
       const int r = base + threadIdx.x;
@@ -104,7 +106,7 @@ __global__ void __launch_bounds__(256) split_combine_kernel(PartialParams p) {
     __syncthreads();
     const int start = sh_start, nt_b = sh_nt;
     if (nt_b == 0) {
-      for (int h = warp; h < p.heads; h += 8) {
+      if (h < p.heads) {
         float* o = p.out + ((size_t)b * p.heads + h) * kVDim;
         for (int i = threadIdx.x & 31; i < kVDim; i += 32) o[i] = 0.f;
         if ((threadIdx.x & 31) == 0) p.out_lse[(size_t)b * p.heads + h] = -CUDART_INF_F;
@@ -117,10 +119,9 @@ __global__ void __launch_bounds__(256) split_combine_kernel(PartialParams p) {
     first_slot = c_first + b;
     count = c_last - c_first + 1;
   }
-  for (int h = warp; h < p.heads; h += 8) {
+  if (h < p.heads)
     merge_warp(p.ws_o, p.ws_lse, (size_t)first_slot * p.heads + h, p.heads, count,
                p.out + ((size_t)b * p.heads + h) * kVDim, p.out_lse + (size_t)b * p.heads + h);
-  }
 }
 
 }  // namespace
@@ -136,7 +137,8 @@ cudaError_t launch_dcp_merge(const float* partials, const float* lses, int num_s
 
 cudaError_t launch_split_combine(const PartialParams& p, cudaStream_t st) {
   if (p.sparse_idx && p.sparse_parts == 1) return cudaSuccess;
-  split_combine_kernel<<<p.batch, 256, 0, st>>>(p);
+  const int hgroups = (p.heads + 7) / 8;
+  split_combine_kernel<<<p.batch * hgroups, 256, 0, st>>>(p);
   return cudaGetLastError();
 }
 

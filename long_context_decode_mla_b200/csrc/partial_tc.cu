@@ -10,13 +10,18 @@
 // "The core design").
 //
 // How (per CTA, one per SM, persistent over its slice of the tile space):
-//  * Q of the current request (64 heads padded, 576 bf16) sits in shared
+//  * The tensor-core operands are fp16 with fp32 accumulation: bf16 cache
+//    values convert to fp16 exactly (within +-65504), e4m3 * scale rounds to
+//    11 significant bits (8x finer than bf16), and P keeps 11 bits too.
+//    Values beyond the fp16 range are clamped and flagged.
+//  * Q of the current request (64 heads padded, 576 values) sits in shared
 //    memory, 128-byte swizzled, as the A operand of S = Q K^T.
 //  * A tile is 128 local tokens (two cache blocks).  Its rows are brought into
 //    nine 16 KB shared-memory chunk slots (8 latent chunks of 64 values, then
-//    rope), swizzled for the tensor core.  bf16 rows are copied with
-//    cp.async; fp8 rows are read into registers, decoded (e4m3 * scale ->
-//    bf16) and stored, so raw fp8 never occupies shared memory.
+//    rope), swizzled for the tensor core.  Eight converter warps load each
+//    tile's rows into registers one tile ahead (global-memory latency stays
+//    off the critical path), then decode and store them once the slots are
+//    free; raw cache bytes never occupy shared memory.
 //  * S = Q K^T: 36 weight-stationary MMAs (M = 64 heads, N = 128 tokens,
 //    K = 16) into TMEM; the 2x2 data path puts head h at TMEM lane h for
 //    tokens 0..63 and lane 64 + h for tokens 64..127.
@@ -54,6 +59,8 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.f;
 constexpr int kFlagTimeout = 4;
+constexpr int kFlagRange = 8;
+constexpr float kF16Max = 65504.f;
 
 struct TcCtl {
   uint64_t full[kNumSlots];
@@ -116,8 +123,16 @@ __device__ __forceinline__ const uint8_t* tile_row(const PartialParams& p, const
   return p.kv + ((size_t)blk * kBlock + (j & 63)) * kRowBytes;
 }
 
-// 16 e4m3 codes times `sc` -> 16 bf16 (two 16-byte units, dims in order).
-__device__ __forceinline__ void decode16(const uint4 v, float sc, uint4& lo, uint4& hi) {
+// fp32 pair -> fp16 pair (lo in the low half), rounded to nearest, clamped
+// to +-65504.
+__device__ __forceinline__ uint32_t f16x2_sat(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// 16 e4m3 codes times `sc` -> 16 fp16 (two 16-byte units, dims in order).
+__device__ __forceinline__ void e4m3x16_to_f16(const uint4 v, float sc, uint4& lo, uint4& hi) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
   uint32_t o[8];
 #pragma unroll
@@ -129,12 +144,24 @@ __device__ __forceinline__ void decode16(const uint4 v, float sc, uint4& lo, uin
       __half2 h2;
       *reinterpret_cast<__half2_raw*>(&h2) = hr;
       const float2 f = __half22float2(h2);
-      const __nv_bfloat162 b2 = __floats2bfloat162_rn(f.x * sc, f.y * sc);
-      o[2 * i + hw] = *reinterpret_cast<const uint32_t*>(&b2);
+      o[2 * i + hw] = f16x2_sat(f.x * sc, f.y * sc);
     }
   }
   lo = make_uint4(o[0], o[1], o[2], o[3]);
   hi = make_uint4(o[4], o[5], o[6], o[7]);
+}
+
+// 8 bf16 -> 8 fp16; `amax` collects the largest magnitude seen.
+__device__ __forceinline__ uint4 bf16x8_to_f16(const uint4 v, float& amax) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t o[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float a = __uint_as_float(w[i] << 16), b = __uint_as_float(w[i] & 0xFFFF0000u);
+    amax = fmaxf(amax, fmaxf(fabsf(a), fabsf(b)));
+    o[i] = f16x2_sat(a, b);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
 // ------------------------------------------------------------- segments ----
@@ -211,15 +238,21 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, Tc
 
 // MMA issue (one thread): S = Q K^T for tile t.
 __device__ __forceinline__ bool issue_qk(TcCtl& c, uint32_t q0, uint32_t s0, uint32_t tau) {
-  constexpr uint32_t kIdQK = ptx::idesc_bf16(64, 128, false);
-  for (int s = 0; s < kNumSlots; ++s)
-    if (!wait_or_abort(&c.full[s], tau & 1, c)) return false;
-  ptx::tc_fence_after();
+  constexpr uint32_t kIdQK = ptx::idesc_f16(64, 128, false);
+  // chunks 0..3 (K-steps 0..15) first: they are filled while the previous
+  // tile's second PV half still runs
+  for (int half = 0; half < 2; ++half) {
+    const int s_lo = half ? 4 : 0, s_hi = half ? kNumSlots : 4;
+    for (int s = s_lo; s < s_hi; ++s)
+      if (!wait_or_abort(&c.full[s], tau & 1, c)) return false;
+    ptx::tc_fence_after();
+    const int k_lo = half ? 16 : 0, k_hi = half ? 36 : 16;
 #pragma unroll 4
-  for (int ks = 0; ks < 36; ++ks) {
-    const uint64_t a = ptx::sdesc_sw128(q0 + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024);
-    const uint64_t b = ptx::sdesc_sw128(s0 + (ks >> 2) * kSlotBytes + (ks & 3) * 32, 16, 1024);
-    ptx::mma_ws_f16(c.tmem_base + kColS, a, b, kIdQK, ks > 0);
+    for (int ks = k_lo; ks < k_hi; ++ks) {
+      const uint64_t a = ptx::sdesc_sw128(q0 + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024);
+      const uint64_t b = ptx::sdesc_sw128(s0 + (ks >> 2) * kSlotBytes + (ks & 3) * 32, 16, 1024);
+      ptx::mma_ws_f16(c.tmem_base + kColS, a, b, kIdQK, ks > 0);
+    }
   }
   ptx::mma_commit(&c.s_full);
   return true;
@@ -227,7 +260,7 @@ __device__ __forceinline__ bool issue_qk(TcCtl& c, uint32_t q0, uint32_t s0, uin
 
 // MMA issue (one thread): O (+)= P V for tile t; releases the slots per half.
 __device__ __forceinline__ void issue_pv(TcCtl& c, uint32_t s0, bool first_tile) {
-  constexpr uint32_t kIdPV = ptx::idesc_bf16(64, 256, true);
+  constexpr uint32_t kIdPV = ptx::idesc_f16(64, 256, true);
   const uint32_t pbase = s0 + kRopeSlot * kSlotBytes;
 #pragma unroll
   for (int hf = 0; hf < 2; ++hf) {
@@ -338,8 +371,8 @@ __device__ void softmax_role(const PartialParams& p, TcCtl& c, uint8_t* sq, uint
         const float p0 = m_used == -CUDART_INF_F ? 0.f : exp2f(x[2 * j] - m_used);
         const float p1 = m_used == -CUDART_INF_F ? 0.f : exp2f(x[2 * j + 1] - m_used);
         sum += p0 + p1;
-        const __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
-        pk[j] = *reinterpret_cast<const uint32_t*>(&b2);
+        const __half2 h2 = __floats2half2_rn(p0, p1);
+        pk[j] = *reinterpret_cast<const uint32_t*>(&h2);
       }
       l += sum;
 #pragma unroll
@@ -389,111 +422,225 @@ __device__ void softmax_role(const PartialParams& p, TcCtl& c, uint8_t* sq, uint
   }
 }
 
-// Fills Q and the chunk slots (256 threads).
+// Rows of one tile held in a converter thread's registers between the
+// global loads and the shared-memory stores.
+template <int KV>
+struct Stage;
+
+// fp8: latent units u0 (dims 16 u0 ..) and 16 + u0 of rows 16 j + 2 cw + rsel,
+// their groups' scales, and four 16-byte rope units.
+template <>
+struct Stage<kKvFp8> {
+  uint4 c0[8], c1[8];
+  float s0[8], s1[8];
+  uint4 rope[4];
+};
+
+// bf16: latent dims 0..255 (unit = lane) of rows 8 i + cw; the second half
+// (dims 256..511 and rope) is loaded when the first half has been stored.
+template <>
+struct Stage<kKvBf16> {
+  uint4 a[16];   // latent dims 0..255
+  uint4 b[20];   // latent dims 256..511 and rope (loaded after a[] is stored)
+};
+
+// Loads the rows of tile t of segment v that this thread stores (fp8).
+__device__ __forceinline__ void stage_load(const PartialParams& p, const SegView& v,
+                                           const int* list, int t, int ct, Stage<kKvFp8>& st,
+                                           bool& range_bad) {
+  const int cw = ct >> 5, cl = ct & 31;
+  const int rsel = (cl >> 2) & 1, u0 = (cl & 3) + 4 * (cl >> 3);
+#pragma unroll
+  for (int jj = 0; jj < 8; ++jj) {
+    const uint8_t* row = tile_row<kKvFp8>(p, v, list, t, 16 * jj + 2 * cw + rsel);
+    if (row) {
+      st.c0[jj] = __ldg(reinterpret_cast<const uint4*>(row) + u0);
+      st.c1[jj] = __ldg(reinterpret_cast<const uint4*>(row) + 16 + u0);
+      st.s0[jj] = __ldg(reinterpret_cast<const float*>(row + 512) + (u0 >> 3));
+      st.s1[jj] = __ldg(reinterpret_cast<const float*>(row + 512) + 2 + (u0 >> 3));
+    } else {
+      st.c0[jj] = st.c1[jj] = make_uint4(0, 0, 0, 0);
+      st.s0[jj] = st.s1[jj] = 0.f;
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int U = i * kConvThreads + ct;
+    const uint8_t* row = tile_row<kKvFp8>(p, v, list, t, U >> 3);
+    st.rope[i] = row ? __ldg(reinterpret_cast<const uint4*>(row + 528) + (U & 7))
+                     : make_uint4(0, 0, 0, 0);
+  }
+  (void)range_bad;
+}
+
+__device__ __forceinline__ void stage_load(const PartialParams& p, const SegView& v,
+                                           const int* list, int t, int ct, Stage<kKvBf16>& st,
+                                           bool& range_bad) {
+  const int cw = ct >> 5, cl = ct & 31;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const uint8_t* row = tile_row<kKvBf16>(p, v, list, t, 8 * i + cw);
+    st.a[i] = row ? __ldg(reinterpret_cast<const uint4*>(row) + cl) : make_uint4(0, 0, 0, 0);
+  }
+  (void)range_bad;
+}
+
+// Stores the first half (latent chunks 0..3) of a staged tile.
+__device__ __forceinline__ void stage_store_half0(uint8_t* sslot, int ct, const Stage<kKvFp8>& st,
+                                                  bool& range_bad) {
+  const int cw = ct >> 5, cl = ct & 31;
+  const int rsel = (cl >> 2) & 1, u0 = (cl & 3) + 4 * (cl >> 3);
+  uint8_t* dst = sslot + (u0 >> 2) * kSlotBytes;
+#pragma unroll
+  for (int jj = 0; jj < 8; ++jj) {
+    const int r = 16 * jj + 2 * cw + rsel;
+    uint4 lo, hi;
+    e4m3x16_to_f16(st.c0[jj], st.s0[jj], lo, hi);
+    range_bad |= st.s0[jj] * 448.f > kF16Max;
+    *reinterpret_cast<uint4*>(dst + swz(r, (u0 & 3) * 2)) = lo;
+    *reinterpret_cast<uint4*>(dst + swz(r, (u0 & 3) * 2 + 1)) = hi;
+  }
+}
+
+__device__ __forceinline__ void stage_store_half0(uint8_t* sslot, int ct, const Stage<kKvBf16>& st,
+                                                  bool& range_bad) {
+  const int cw = ct >> 5, cl = ct & 31;
+  float amax = 0.f;
+  uint8_t* dst = sslot + (cl >> 3) * kSlotBytes;
+#pragma unroll
+  for (int i = 0; i < 16; ++i)
+    *reinterpret_cast<uint4*>(dst + swz(8 * i + cw, cl & 7)) = bf16x8_to_f16(st.a[i], amax);
+  range_bad |= amax > kF16Max;
+}
+
+// Loads the second half (latent dims 256..511 and rope) where it is not
+// staged yet: bf16 rows, 20 units per thread.  fp8 staged it with the first.
+__device__ __forceinline__ void stage_load_half1(const PartialParams&, const SegView&, const int*,
+                                                 int, int, Stage<kKvFp8>&) {}
+
+__device__ __forceinline__ void stage_load_half1(const PartialParams& p, const SegView& v,
+                                                 const int* list, int t, int ct,
+                                                 Stage<kKvBf16>& st) {
+#pragma unroll
+  for (int i = 0; i < 20; ++i) {
+    const int U = i * kConvThreads + ct;
+    const uint8_t* row = tile_row<kKvBf16>(p, v, list, t, U / 40);
+    st.b[i] = row ? __ldg(reinterpret_cast<const uint4*>(row) + 32 + U % 40)
+                  : make_uint4(0, 0, 0, 0);
+  }
+}
+
+// Stores the second half (latent chunks 4..7 and the rope slot).
+__device__ __forceinline__ void stage_store_half1(uint8_t* sslot, int ct, const Stage<kKvFp8>& st,
+                                                  bool& range_bad) {
+  const int cw = ct >> 5, cl = ct & 31;
+  const int rsel = (cl >> 2) & 1, u0 = (cl & 3) + 4 * (cl >> 3);
+  uint8_t* dst = sslot + (4 + (u0 >> 2)) * kSlotBytes;
+#pragma unroll
+  for (int jj = 0; jj < 8; ++jj) {
+    const int r = 16 * jj + 2 * cw + rsel;
+    uint4 lo, hi;
+    e4m3x16_to_f16(st.c1[jj], st.s1[jj], lo, hi);
+    range_bad |= st.s1[jj] * 448.f > kF16Max;
+    *reinterpret_cast<uint4*>(dst + swz(r, (u0 & 3) * 2)) = lo;
+    *reinterpret_cast<uint4*>(dst + swz(r, (u0 & 3) * 2 + 1)) = hi;
+  }
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int U = i * kConvThreads + ct;
+    *reinterpret_cast<uint4*>(sslot + kRopeSlot * kSlotBytes + swz(U >> 3, U & 7)) =
+        bf16x8_to_f16(st.rope[i], amax);
+  }
+  range_bad |= amax > kF16Max;
+}
+
+__device__ __forceinline__ void stage_store_half1(uint8_t* sslot, int ct, const Stage<kKvBf16>& st,
+                                                  bool& range_bad) {
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 20; ++i) {
+    const int U = i * kConvThreads + ct;
+    const int r = U / 40, u = 32 + U % 40;
+    *reinterpret_cast<uint4*>(sslot + (u >> 3) * kSlotBytes + swz(r, u & 7)) =
+        bf16x8_to_f16(st.b[i], amax);
+  }
+  range_bad |= amax > kF16Max;
+}
+
+// Q of request b into the Q region: 64 rows x 72 units of fp16, heads >= H
+// zero.
+__device__ __forceinline__ void load_q(const PartialParams& p, int b, uint8_t* sq, int ct,
+                                       bool& range_bad) {
+  const uint4* qb = reinterpret_cast<const uint4*>(p.q + (size_t)b * p.heads * kHeadDim);
+  float amax = 0.f;
+#pragma unroll 6
+  for (int i = 0; i < 18; ++i) {
+    const int U = i * kConvThreads + ct;
+    const int row = U / 72, u = U % 72;
+    const uint4 v = row < p.heads ? __ldg(qb + (size_t)row * 72 + u) : make_uint4(0, 0, 0, 0);
+    *reinterpret_cast<uint4*>(sq + (u >> 3) * 8192 + swz(row, u & 7)) = bf16x8_to_f16(v, amax);
+  }
+  range_bad |= amax > kF16Max;
+}
+
+// Fills Q and the chunk slots (256 threads), one tile ahead in registers.
 template <int KV>
 __device__ void convert_role(const PartialParams& p, TcCtl& c, uint8_t* sq, uint8_t* sslot,
                              const int* list, int nseg, uint32_t& tau, uint32_t& sigma) {
   const int ct = threadIdx.x - kConvBase;      // 0..255
   const int cw = ct >> 5, cl = ct & 31;
-  const uint32_t q0 = ptx::smem_addr(sq), s0 = ptx::smem_addr(sslot);
-  for (int k = 0; k < nseg; ++k) {
-    const SegView v = seg_view(p, c, k);
-    if (v.ntiles == 0) continue;
-    // ---- Q of request b: 64 rows x 72 units, heads >= H zero-filled ----
-    if (sigma > 0 && !wait_or_abort(&c.q_empty, (sigma - 1) & 1, c)) return;
-    const uint8_t* qb = reinterpret_cast<const uint8_t*>(p.q + (size_t)v.b * p.heads * kHeadDim);
-    for (int i = 0; i < 18; ++i) {
-      const int U = i * kConvThreads + ct;
-      const int row = U / 72, u = U % 72;
-      const bool ok = row < p.heads;
-      ptx::cp_async16(q0 + (u >> 3) * 8192 + swz(row, u & 7),
-                      ok ? qb + ((size_t)row * kHeadDim + u * 8) * 2 : qb, ok ? 16u : 0u);
-    }
-    ptx::cp_async_arrive(&c.q_full);
-    for (int t = 0; t < v.ntiles; ++t, ++tau) {
-      if constexpr (KV == kKvFp8) {
-        // rows 16 j + 2 cw + rsel, latent units u0 (half 0) and 16 + u0 (half 1)
-        const int rsel = (cl >> 2) & 1;
-        const int u0 = (cl & 3) + 4 * (cl >> 3);
-        uint4 c0[8], c1[8];
-        float sc0[8], sc1[8];
-#pragma unroll
-        for (int jj = 0; jj < 8; ++jj) {
-          const int r = 16 * jj + 2 * cw + rsel;
-          const uint8_t* row = tile_row<KV>(p, v, list, t, r);
-          if (row) {
-            c0[jj] = __ldg(reinterpret_cast<const uint4*>(row) + u0);
-            c1[jj] = __ldg(reinterpret_cast<const uint4*>(row) + 16 + u0);
-            sc0[jj] = __ldg(reinterpret_cast<const float*>(row + 512) + (u0 >> 3));
-            sc1[jj] = __ldg(reinterpret_cast<const float*>(row + 512) + 2 + (u0 >> 3));
-          } else {
-            c0[jj] = c1[jj] = make_uint4(0, 0, 0, 0);
-            sc0[jj] = sc1[jj] = 0.f;
-          }
-        }
-        if (tau > 0)
-          for (int s = 0; s < 4; ++s)
-            if (!wait_or_abort(&c.empty[s], (tau - 1) & 1, c)) return;
-#pragma unroll
-        for (int jj = 0; jj < 8; ++jj) {
-          const int r = 16 * jj + 2 * cw + rsel;
-          uint4 lo, hi;
-          decode16(c0[jj], sc0[jj], lo, hi);
-          uint8_t* dst = sslot + (u0 >> 2) * kSlotBytes;
-          *reinterpret_cast<uint4*>(dst + swz(r, (u0 & 3) * 2)) = lo;
-          *reinterpret_cast<uint4*>(dst + swz(r, (u0 & 3) * 2 + 1)) = hi;
-        }
-        ptx::fence_proxy_async();
-        for (int s = 0; s < 4; ++s) ptx::mbar_arrive(&c.full[s]);
-        if (tau > 0)
-          for (int s = 4; s < kNumSlots; ++s)
-            if (!wait_or_abort(&c.empty[s], (tau - 1) & 1, c)) return;
-#pragma unroll
-        for (int jj = 0; jj < 8; ++jj) {
-          const int r = 16 * jj + 2 * cw + rsel;
-          uint4 lo, hi;
-          decode16(c1[jj], sc1[jj], lo, hi);
-          uint8_t* dst = sslot + (4 + (u0 >> 2)) * kSlotBytes;
-          *reinterpret_cast<uint4*>(dst + swz(r, (u0 & 3) * 2)) = lo;
-          *reinterpret_cast<uint4*>(dst + swz(r, (u0 & 3) * 2 + 1)) = hi;
-        }
-        // rope: 128 rows x 8 units of bf16, copied as is
-        for (int i = 0; i < 4; ++i) {
-          const int U = i * kConvThreads + ct;
-          const int r = U >> 3, u = U & 7;
-          const uint8_t* row = tile_row<KV>(p, v, list, t, r);
-          ptx::cp_async16(s0 + kRopeSlot * kSlotBytes + swz(r, u), row ? row + 528 + 16 * u : p.kv,
-                          row ? 16u : 0u);
-        }
-      } else {
-        if (tau > 0)
-          for (int s = 0; s < kNumSlots; ++s)
-            if (!wait_or_abort(&c.empty[s], (tau - 1) & 1, c)) return;
-        for (int i = 0; i < 36; ++i) {
-          const int U = i * kConvThreads + ct;
-          const int r = U / 72, u = U % 72;
-          const uint8_t* row = tile_row<KV>(p, v, list, t, r);
-          ptx::cp_async16(s0 + (u >> 3) * kSlotBytes + swz(r, u & 7), row ? row + 16 * u : p.kv,
-                          row ? 16u : 0u);
-        }
-      }
-      // valid-row mask of the tile, published with the rope slot
-      if (ct < 128) {
-        const bool ok = tile_row<KV>(p, v, list, t, ct) != nullptr;
-        const uint32_t m = __ballot_sync(0xffffffffu, ok);
-        if (cl == 0) c.row_mask[cw] = m;
-      }
+  bool range_bad = false;
+  Stage<KV> st;
+  // first tile with work
+  int k = 0;
+  while (k < nseg && seg_view(p, c, k).ntiles == 0) ++k;
+  if (k >= nseg) return;
+  SegView v = seg_view(p, c, k);
+  int t = 0;
+  stage_load(p, v, list, t, ct, st, range_bad);
+  while (true) {
+    if (t == 0) {
+      // new request: its Q replaces the previous one once that one's last
+      // QK has completed
+      if (sigma > 0 && !wait_or_abort(&c.q_empty, (sigma - 1) & 1, c)) return;
+      load_q(p, v.b, sq, ct, range_bad);
       ptx::fence_proxy_async();
-      if constexpr (KV == kKvFp8) {
-        for (int s = 4; s < 8; ++s) ptx::mbar_arrive(&c.full[s]);
-        ptx::cp_async_arrive(&c.full[kRopeSlot]);
-      } else {
-        for (int s = 0; s < kNumSlots; ++s) ptx::cp_async_arrive(&c.full[s]);
-      }
-      if (ct < 128 && cl == 0) ptx::mbar_arrive(&c.full[kRopeSlot]);
+      ptx::mbar_arrive(&c.q_full);
     }
-    ++sigma;
+    if (tau > 0)
+      for (int s = 0; s < 4; ++s)
+        if (!wait_or_abort(&c.empty[s], (tau - 1) & 1, c)) return;
+    stage_store_half0(sslot, ct, st, range_bad);
+    ptx::fence_proxy_async();
+    for (int s = 0; s < 4; ++s) ptx::mbar_arrive(&c.full[s]);
+    stage_load_half1(p, v, list, t, ct, st);
+    if (tau > 0)
+      for (int s = 4; s < kNumSlots; ++s)
+        if (!wait_or_abort(&c.empty[s], (tau - 1) & 1, c)) return;
+    stage_store_half1(sslot, ct, st, range_bad);
+    // valid-row mask of the tile, published with the rope slot
+    if (ct < 128) {
+      const bool ok = tile_row<KV>(p, v, list, t, ct) != nullptr;
+      const uint32_t m = __ballot_sync(0xffffffffu, ok);
+      if (cl == 0) c.row_mask[cw] = m;
+    }
+    ptx::fence_proxy_async();
+    for (int s = 4; s < kNumSlots; ++s) ptx::mbar_arrive(&c.full[s]);
+    ++tau;
+    // next tile (possibly of the next segment): load it now
+    if (++t >= v.ntiles) {
+      ++sigma;
+      t = 0;
+      do {
+        ++k;
+      } while (k < nseg && seg_view(p, c, k).ntiles == 0);
+      if (k >= nseg) break;
+      v = seg_view(p, c, k);
+    }
+    stage_load(p, v, list, t, ct, st, range_bad);
   }
+  if (range_bad && p.flags) atomicOr(p.flags, kFlagRange);
 }
 
 template <int KV>
@@ -508,10 +655,8 @@ __global__ void __launch_bounds__(kThreads, 1) partial_tc_kernel(PartialParams p
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kNumSlots; ++s) {
-      // fp8: 256 converter arrivals on every slot; the rope slot also gets the
-      // 4 row-mask writers.  bf16: the same counts.
-      ptx::mbar_init(&c.full[s], kConvThreads + (s == kRopeSlot ? 4 : 0));
-      ptx::mbar_init(&c.empty[s], 1);
+      ptx::mbar_init(&c.full[s], kConvThreads);   // every converter thread, once per tile
+      ptx::mbar_init(&c.empty[s], 1);             // one tcgen05.commit per tile
     }
     ptx::mbar_init(&c.q_full, kConvThreads);
     ptx::mbar_init(&c.q_empty, 1);

@@ -172,10 +172,9 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t addr, uint32_t lbo, uin
   return d;
 }
 
-// Instruction descriptor, kind::f16 with bf16 inputs and fp32 accumulation.
-__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn_major) {
-  return (1u << 4)                       // D format: f32
-         | (1u << 7) | (1u << 10)        // A, B format: bf16
+// Instruction descriptor, kind::f16 with fp16 inputs and fp32 accumulation.
+__host__ __device__ constexpr uint32_t idesc_f16(int M, int N, bool b_mn_major) {
+  return (1u << 4)                       // D format: f32 (A, B format 0: f16)
          | ((b_mn_major ? 1u : 0u) << 16)
          | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
