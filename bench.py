@@ -55,6 +55,19 @@ def dist_env():
     return rank, world, local
 
 
+def max_over_ranks(values):
+    """Element-wise max of a list of floats over all ranks (identity without a
+    process group).  Every rank must call it, in the same order."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return list(values)
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor(list(values), dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
 def kv_bytes(prob) -> int:
     """KV bytes one step must read: every cached (or, sparse, every selected) row once."""
     from long_context_decode_mla_b200.workload import ROW_BYTES
@@ -274,10 +287,7 @@ def run_ours(args, rank, world, local):
     assert dec.flags() == 0, "device flags set"
     sampler.stop()
 
-    times = torch.tensor([ms_step, e2e_ms], device=dev)
-    if world > 1:
-        dist.all_reduce(times, op=dist.ReduceOp.MAX)
-    ms_step, e2e_ms = times.tolist()
+    ms_step, e2e_ms, ms_partials = max_over_ranks([ms_step, e2e_ms, ms_partials])
     gpu_launches = args.steps * (N * (1 if (prob.sparse_idx is not None) else 2) + 1)
     peak, peak_kind = measured_peaks()
     result = None

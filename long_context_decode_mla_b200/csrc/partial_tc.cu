@@ -16,24 +16,23 @@
 //    Values beyond the fp16 range are clamped and flagged.
 //  * Q of the current request (64 heads padded, 576 values) sits in shared
 //    memory, 128-byte swizzled, as the A operand of S = Q K^T.
-//  * A tile is 128 local tokens (two cache blocks).  Its rows are brought into
-//    nine 16 KB shared-memory chunk slots (8 latent chunks of 64 values, then
-//    rope), swizzled for the tensor core.  Eight converter warps load each
-//    tile's rows into registers one tile ahead (global-memory latency stays
-//    off the critical path), then decode and store them once the slots are
-//    free; raw cache bytes never occupy shared memory.
-//  * S = Q K^T: 36 weight-stationary MMAs (M = 64 heads, N = 128 tokens,
-//    K = 16) into TMEM; the 2x2 data path puts head h at TMEM lane h for
-//    tokens 0..63 and lane 64 + h for tokens 64..127.
+//  * A tile is one cache block (64 local tokens).  Two stages, each of nine
+//    8 KB chunk slots (8 latent chunks of 64 values, then rope), hold
+//    consecutive tiles, swizzled for the tensor core.  Eight converter warps
+//    load each tile's rows into registers one tile ahead, decode them (bf16
+//    or e4m3 * scale -> fp16) and store them once a stage is free; raw cache
+//    bytes never occupy shared memory.
+//  * S = Q K^T: 36 weight-stationary MMAs (M = 64 heads, N = 64 tokens,
+//    K = 16) into one of two TMEM score buffers; the 2x2 data path puts head
+//    h at TMEM lane h for tokens 0..31 and lane 64 + h for tokens 32..63.
+//    The scores of tile t + 1 are computed while the softmax of tile t runs.
 //  * Four softmax warps (one TMEM lane each) run the online softmax in base 2
-//    with a lazily updated running max (the output is only rescaled when the
-//    max grows by more than 2^8), write P (bf16) into the rope slot, which
-//    the scores no longer need, and keep the running sum.
-//  * O += P V: 16 MMAs (M = 64, N = 256 dims, K = 16 tokens) reading V from
-//    the same chunk slots as an MN-major operand; O (64 x 512 fp32) stays in
-//    TMEM for the whole request and is normalised in the epilogue.
-//  * Slots are released per half of the PV step so the next tile's first
-//    chunks can be filled while the second half still runs.
+//    with a lazily updated running max (the output is only rescaled, warp by
+//    warp, when the max grows by more than 2^8), write P into the stage's
+//    rope slot, which the scores no longer need, and keep the running sum.
+//  * O += P V: 8 MMAs (M = 64, N = 256 dims, K = 16 tokens) reading V from the
+//    same chunk slots as an MN-major operand; O (64 x 512 fp32) stays in TMEM
+//    for the whole request and is normalised in the epilogue.
 #include <cuda_fp8.h>
 #include <math_constants.h>
 
@@ -44,44 +43,50 @@
 namespace dcpmla {
 namespace {
 
-constexpr int kThreads = 384;          // 12 warps: 4 softmax (thread 0 issues MMAs), 8 converters
-constexpr int kConvBase = 128;         // first converter thread
+constexpr int kThreads = 416;          // 13 warps: 4 softmax, 1 MMA issue, 8 converters
+constexpr int kMmaWarp = 4;
+constexpr int kConvBase = 160;         // first converter thread
 constexpr int kConvThreads = 256;
-constexpr int kTileTok = 128;
-constexpr int kSlotBytes = 16384;
-constexpr int kNumSlots = 9;
+constexpr int kTileTok = 64;           // one cache block
+constexpr int kSlotBytes = 8192;       // 64 rows x 128 bytes
+constexpr int kNumSlots = 9;           // per stage: 8 latent chunks + rope (then P)
 constexpr int kRopeSlot = 8;
+constexpr int kStages = 2;
 constexpr int kQBytes = 9 * 8192;
 constexpr int kMaxSeg = 128;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 256;        // S: columns [256, 320); O: columns [0, 256)
+constexpr uint32_t kColS = 256;        // S buffers: columns [256, 288) and [288, 320); O: [0, 256)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.f;
+constexpr int kPrefetchTiles = 6;      // L2 prefetch distance, in tiles
 constexpr int kFlagTimeout = 4;
 constexpr int kFlagRange = 8;
 constexpr float kF16Max = 65504.f;
 
 struct TcCtl {
-  uint64_t full[kNumSlots];
-  uint64_t empty[kNumSlots];
-  uint64_t q_full, q_empty, s_full, p_full, o_full;
+  uint64_t full[kStages][2];     // converter -> MMA, per stage and slot half (256 arrivals)
+  uint64_t empty[kStages][2];    // MMA -> converter, per stage and slot half (PV commits)
+  uint64_t s_full[2];            // scores buffer ready (QK commit)
+  uint64_t p_full[kStages];      // P written (128 softmax arrivals)
+  uint64_t o_ready;              // PV of a tile complete (commit, every tile)
+  uint64_t q_full, q_empty;      // Q loaded (256 arrivals) / last QK of a request done
   uint32_t tmem_base;
   int abort;
-  uint32_t row_mask[4];
+  uint32_t row_mask[kStages][2];
   float red[2][2][64];
   float lred[2][64];
-  int nseg;
   int sel_count;
   int warp_sums[16];
   Segment seg[kMaxSeg];
 };
 
-constexpr size_t kSmemBytes = kQBytes + (size_t)kNumSlots * kSlotBytes + sizeof(TcCtl) + 1024;
+constexpr size_t kSmemBytes =
+    kQBytes + (size_t)kStages * kNumSlots * kSlotBytes + sizeof(TcCtl) + 1024;
 
 struct SegView {
   int b;
-  int row_begin;   // first local row (dense) or list offset (sparse)
+  int row_begin;   // first local row (dense); 0 (sparse, rows come from the list)
   int nrows;
   int ntiles;
   bool whole;
@@ -89,6 +94,10 @@ struct SegView {
 
 __device__ __forceinline__ uint32_t swz(int row, int unit) {
   return (uint32_t)((row >> 3) * 1024 + (row & 7) * 128 + ((unit ^ (row & 7)) << 4));
+}
+
+__device__ __forceinline__ uint8_t* slot_ptr(uint8_t* sslot, int stage, int c) {
+  return sslot + (stage * kNumSlots + c) * kSlotBytes;
 }
 
 __device__ __forceinline__ SegView seg_view(const PartialParams& p, const TcCtl& c, int k) {
@@ -109,19 +118,101 @@ __device__ __forceinline__ SegView seg_view(const PartialParams& p, const TcCtl&
   return v;
 }
 
-// Address of local tile row r of the segment, or nullptr if it is past the
-// end or its block-table entry is out of range (flagged).
+// Address of row r of tile `tile` of the segment, or nullptr if it is past
+// the end or its block-table entry is out of range (flagged).
 template <int KV>
 __device__ __forceinline__ const uint8_t* tile_row(const PartialParams& p, const SegView& v,
                                                   const int* list, int tile, int r) {
   constexpr int kRowBytes = KV == kKvBf16 ? kRowBytesBf16 : kRowBytesFp8;
   const int i = tile * kTileTok + r;
   if (i >= v.nrows) return nullptr;
-  const int j = p.sparse_idx ? list[i] : v.row_begin + i;   // written by this CTA: no __ldg
+  const int j = p.sparse_idx ? list[i] : v.row_begin + i;   // list: written by this CTA, no __ldg
   const int blk = tile_block(p, v.b, j >> 6);
   if (blk < 0) return nullptr;
   return p.kv + ((size_t)blk * kBlock + (j & 63)) * kRowBytes;
 }
+
+// Addresses of N rows (rows[i]) of tile t, without serialising dependent
+// loads: a dense tile is one cache block (one table load for all rows);
+// sparse rows load all their list entries, then all their table entries.
+// Invalid rows (past the end, or a flagged table entry) give nullptr.
+template <int KV, int N>
+__device__ __forceinline__ void tile_rows(const PartialParams& p, const SegView& v,
+                                          const int* list, int t, const int (&rows)[N],
+                                          const uint8_t* (&out)[N]) {
+  constexpr int kRowBytes = KV == kKvBf16 ? kRowBytesBf16 : kRowBytesFp8;
+  const int nvalid = v.nrows - t * kTileTok;
+  if (!p.sparse_idx) {
+    const int blk = tile_block(p, v.b, (v.row_begin >> 6) + t);
+    const uint8_t* base = blk >= 0 ? p.kv + (size_t)blk * kBlock * kRowBytes : nullptr;
+#pragma unroll
+    for (int i = 0; i < N; ++i)
+      out[i] = (base && rows[i] < nvalid) ? base + rows[i] * kRowBytes : nullptr;
+  } else {
+    int j[N], blk[N];
+#pragma unroll
+    for (int i = 0; i < N; ++i) j[i] = rows[i] < nvalid ? list[t * kTileTok + rows[i]] : -1;
+#pragma unroll
+    for (int i = 0; i < N; ++i)
+      blk[i] = j[i] >= 0 ? __ldg(p.block_table + (size_t)v.b * p.bt_stride + (j[i] >> 6)) : -1;
+#pragma unroll
+    for (int i = 0; i < N; ++i) {
+      const bool ok = blk[i] >= 0 && (long long)blk[i] < p.num_blocks;
+      if (j[i] >= 0 && !ok && p.flags) atomicOr(p.flags, kFlagBadBlock);
+      out[i] = ok ? p.kv + ((size_t)blk[i] * kBlock + (j[i] & 63)) * kRowBytes : nullptr;
+    }
+  }
+}
+
+// Asks L2 for the rows of tile t of the segment (a dense tile is one
+// contiguous cache block: one bulk prefetch; sparse rows one by one).
+template <int KV>
+__device__ __forceinline__ void prefetch_tile(const PartialParams& p, const SegView& v,
+                                              const int* list, int t, int ct) {
+  constexpr int kRowBytes = KV == kKvBf16 ? kRowBytesBf16 : kRowBytesFp8;
+  if (!p.sparse_idx) {
+    if (ct == 0) {
+      const int blk = tile_block(p, v.b, (v.row_begin >> 6) + t);
+      if (blk >= 0) {
+        const int rows = min(kTileTok, v.nrows - t * kTileTok);
+        ptx::prefetch_l2(p.kv + (size_t)blk * kBlock * kRowBytes, (uint32_t)(rows * kRowBytes));
+      }
+    }
+  } else if (ct < kTileTok) {
+    const int rr[1] = {ct};
+    const uint8_t* rp[1];
+    tile_rows<KV, 1>(p, v, list, t, rr, rp);
+    if (rp[0]) ptx::prefetch_l2(rp[0], kRowBytes);
+  }
+}
+
+// Walks the CTA's tiles in order: segment k, tile t (segments without tiles
+// are skipped).  Returns false past the last tile.
+struct TileCursor {
+  int k, t, nseg;
+  SegView v;
+  __device__ __forceinline__ bool start(const PartialParams& p, const TcCtl& c, int n) {
+    nseg = n;
+    k = 0;
+    t = 0;
+    while (k < nseg) {
+      v = seg_view(p, c, k);
+      if (v.ntiles > 0) return true;
+      ++k;
+    }
+    return false;
+  }
+  __device__ __forceinline__ bool next(const PartialParams& p, const TcCtl& c) {
+    if (++t < v.ntiles) return true;
+    t = 0;
+    while (++k < nseg) {
+      v = seg_view(p, c, k);
+      if (v.ntiles > 0) return true;
+    }
+    return false;
+  }
+  __device__ __forceinline__ bool last_of_segment() const { return t == v.ntiles - 1; }
+};
 
 // fp32 pair -> fp16 pair (lo in the low half), rounded to nearest, clamped
 // to +-65504.
@@ -132,19 +223,39 @@ __device__ __forceinline__ uint32_t f16x2_sat(float lo, float hi) {
 }
 
 // 16 e4m3 codes times `sc` -> 16 fp16 (two 16-byte units, dims in order).
+// e4m3 -> fp16 is exact; when the scale is a normal fp16 number that keeps
+// every product finite (2^-14 <= sc <= 65504 / 448) the product is taken in
+// fp16 (two instructions per pair, two roundings); otherwise in fp32 and
+// rounded once, with clamping.
 __device__ __forceinline__ void e4m3x16_to_f16(const uint4 v, float sc, uint4& lo, uint4& hi) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
   uint32_t o[8];
+  if (sc >= 6.103515625e-05f && sc <= 146.0f) {
+    const __half2 s2 = __float2half2_rn(sc);
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < 4; ++i) {
 #pragma unroll
-    for (int hw = 0; hw < 2; ++hw) {
-      const __nv_fp8x2_storage_t pair = (__nv_fp8x2_storage_t)((w[i] >> (16 * hw)) & 0xFFFFu);
-      const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3);
-      __half2 h2;
-      *reinterpret_cast<__half2_raw*>(&h2) = hr;
-      const float2 f = __half22float2(h2);
-      o[2 * i + hw] = f16x2_sat(f.x * sc, f.y * sc);
+      for (int hw = 0; hw < 2; ++hw) {
+        const __nv_fp8x2_storage_t pair = (__nv_fp8x2_storage_t)((w[i] >> (16 * hw)) & 0xFFFFu);
+        const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3);
+        __half2 h2;
+        *reinterpret_cast<__half2_raw*>(&h2) = hr;
+        const __half2 r2 = __hmul2(h2, s2);
+        o[2 * i + hw] = *reinterpret_cast<const uint32_t*>(&r2);
+      }
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+#pragma unroll
+      for (int hw = 0; hw < 2; ++hw) {
+        const __nv_fp8x2_storage_t pair = (__nv_fp8x2_storage_t)((w[i] >> (16 * hw)) & 0xFFFFu);
+        const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3);
+        __half2 h2;
+        *reinterpret_cast<__half2_raw*>(&h2) = hr;
+        const float2 f = __half22float2(h2);
+        o[2 * i + hw] = f16x2_sat(f.x * sc, f.y * sc);
+      }
     }
   }
   lo = make_uint4(o[0], o[1], o[2], o[3]);
@@ -236,189 +347,253 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, Tc
   return ptx::mbar_wait(bar, parity, &c.abort);
 }
 
-// MMA issue (one thread): S = Q K^T for tile t.
-__device__ __forceinline__ bool issue_qk(TcCtl& c, uint32_t q0, uint32_t s0, uint32_t tau) {
-  constexpr uint32_t kIdQK = ptx::idesc_f16(64, 128, false);
-  // chunks 0..3 (K-steps 0..15) first: they are filled while the previous
-  // tile's second PV half still runs
-  for (int half = 0; half < 2; ++half) {
-    const int s_lo = half ? 4 : 0, s_hi = half ? kNumSlots : 4;
-    for (int s = s_lo; s < s_hi; ++s)
-      if (!wait_or_abort(&c.full[s], tau & 1, c)) return false;
-    ptx::tc_fence_after();
-    const int k_lo = half ? 16 : 0, k_hi = half ? 36 : 16;
-#pragma unroll 4
-    for (int ks = k_lo; ks < k_hi; ++ks) {
-      const uint64_t a = ptx::sdesc_sw128(q0 + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024);
-      const uint64_t b = ptx::sdesc_sw128(s0 + (ks >> 2) * kSlotBytes + (ks & 3) * 32, 16, 1024);
-      ptx::mma_ws_f16(c.tmem_base + kColS, a, b, kIdQK, ks > 0);
-    }
-  }
-  ptx::mma_commit(&c.s_full);
+// Shared-memory descriptors differ only in their start-address field (bits
+// 0..13, address / 16), so each MMA's descriptors are a base plus a constant:
+// the issuing thread spends one 32-bit add per operand.
+struct Descs {
+  uint64_t q;           // Q chunk 0, K-major
+  uint64_t k[kStages];  // chunk slot 0 of each stage, K-major (QK operand B)
+  uint64_t p[kStages];  // P (rope slot) of each stage, K-major (PV operand A)
+  uint64_t v[kStages];  // chunk slot 0 of each stage, MN-major (PV operand B)
+};
+
+__device__ __forceinline__ uint64_t dplus(uint64_t d, uint32_t byte_off) {
+  return d + (uint64_t)(byte_off >> 4);
+}
+
+// MMA issue (one thread): S[tau & 1] = Q K^T for tile tau (stage tau & 1).
+// Chunks 0..3 go first: they are refilled while the previous use of the stage
+// still runs its second PV half.
+__device__ __forceinline__ bool issue_qk(TcCtl& c, const Descs& d, uint32_t tau) {
+  constexpr uint32_t kIdQK = ptx::idesc_f16(64, 64, false);
+  const int st = tau & 1;
+  const uint32_t ph = (tau >> 1) & 1;
+  const uint64_t kd = st ? d.k[1] : d.k[0];
+  const uint32_t dst = c.tmem_base + kColS + 32 * st;
+  if (!wait_or_abort(&c.full[st][0], ph, c)) return false;
+  ptx::tc_fence_after();
+#pragma unroll
+  for (int ks = 0; ks < 16; ++ks)
+    ptx::mma_ws_f16(dst, dplus(d.q, (ks >> 2) * 8192 + (ks & 3) * 32),
+                    dplus(kd, (ks >> 2) * kSlotBytes + (ks & 3) * 32), kIdQK, ks > 0);
+  if (!wait_or_abort(&c.full[st][1], ph, c)) return false;
+  ptx::tc_fence_after();
+#pragma unroll
+  for (int ks = 16; ks < 36; ++ks)
+    ptx::mma_ws_f16(dst, dplus(d.q, (ks >> 2) * 8192 + (ks & 3) * 32),
+                    dplus(kd, (ks >> 2) * kSlotBytes + (ks & 3) * 32), kIdQK, 1u);
+  ptx::mma_commit(&c.s_full[st]);
   return true;
 }
 
-// MMA issue (one thread): O (+)= P V for tile t; releases the slots per half.
-__device__ __forceinline__ void issue_pv(TcCtl& c, uint32_t s0, bool first_tile) {
+// MMA issue (one thread): O (+)= P V for tile tau; frees the stage per half.
+__device__ __forceinline__ void issue_pv(TcCtl& c, const Descs& d, uint32_t tau, bool first_tile) {
   constexpr uint32_t kIdPV = ptx::idesc_f16(64, 256, true);
-  const uint32_t pbase = s0 + kRopeSlot * kSlotBytes;
+  const int st = tau & 1;
 #pragma unroll
   for (int hf = 0; hf < 2; ++hf) {
 #pragma unroll
-    for (int kk = 0; kk < 8; ++kk) {
-      const uint64_t a = ptx::sdesc_sw128(pbase + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
-      const uint64_t b = ptx::sdesc_sw128(s0 + 4 * hf * kSlotBytes + kk * 2048, kSlotBytes, 1024);
-      ptx::mma_ws_f16(c.tmem_base + hf * 128, a, b, kIdPV, (!first_tile || kk > 0) ? 1u : 0u);
+    for (int kk = 0; kk < 4; ++kk)
+      ptx::mma_ws_f16(c.tmem_base + hf * 128, dplus(st ? d.p[1] : d.p[0], kk * 32),
+                      dplus(st ? d.v[1] : d.v[0], 4 * hf * kSlotBytes + kk * 2048), kIdPV,
+                      (!first_tile || kk > 0) ? 1u : 0u);
+    ptx::mma_commit(&c.empty[st][hf]);
+  }
+  ptx::mma_commit(&c.o_ready);
+}
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Issues every MMA (one thread of the MMA warp): the scores of the next tile
+// before the PV of this one, so that the softmax of tile t overlaps the
+// scores of tile t + 1.
+__device__ void mma_role(const PartialParams& p, TcCtl& c, uint8_t* sq, uint8_t* sslot, int nseg,
+                         uint32_t& tau, uint32_t& sigma, uint32_t (&uses)[2]) {
+  Descs dsc;
+  {
+    const uint32_t q0 = ptx::smem_addr(sq), s0 = ptx::smem_addr(sslot);
+    dsc.q = ptx::sdesc_sw128(q0, 16, 1024);
+    for (int st = 0; st < kStages; ++st) {
+      const uint32_t base = s0 + st * kNumSlots * kSlotBytes;
+      dsc.k[st] = ptx::sdesc_sw128(base, 16, 1024);
+      dsc.p[st] = ptx::sdesc_sw128(base + kRopeSlot * kSlotBytes, 16, 1024);
+      dsc.v[st] = ptx::sdesc_sw128(base, kSlotBytes, 1024);
     }
-    if (hf == 0) {
-      for (int s = 0; s < 4; ++s) ptx::mma_commit(&c.empty[s]);
-    } else {
-      for (int s = 4; s < kNumSlots; ++s) ptx::mma_commit(&c.empty[s]);
+  }
+  TileCursor cur, ahead;
+  if (!cur.start(p, c, nseg)) return;
+  ahead = cur;
+  if (!wait_or_abort(&c.q_full, sigma & 1, c)) return;
+  if (!issue_qk(c, dsc, tau)) return;
+  if (ahead.last_of_segment()) ptx::mma_commit(&c.q_empty);
+  uint32_t sigma_ahead = sigma;
+  while (true) {
+    const bool seg_end = ahead.last_of_segment();
+    if (ahead.next(p, c)) {
+      if (seg_end) {
+        ++sigma_ahead;
+        if (!wait_or_abort(&c.q_full, sigma_ahead & 1, c)) return;
+      }
+      if (!issue_qk(c, dsc, tau + 1)) return;
+      if (ahead.last_of_segment()) ptx::mma_commit(&c.q_empty);
     }
+    const int st = tau & 1;
+    if (!wait_or_abort(&c.p_full[st], (tau >> 1) & 1, c)) return;
+    ptx::tc_fence_after();
+    issue_pv(c, dsc, tau, cur.t == 0);
+    ++uses[st];
+    if (cur.last_of_segment()) ++sigma;
+    ++tau;
+    if (!cur.next(p, c)) break;
   }
 }
 
-// Online softmax, P, and the epilogue (128 threads, one TMEM lane each).
-__device__ void softmax_role(const PartialParams& p, TcCtl& c, uint8_t* sq, uint8_t* sslot,
-                             int nseg, uint32_t& tau, uint32_t& sigma) {
+// Online softmax, P and the epilogue (128 threads, one TMEM lane each).
+__device__ void softmax_role(const PartialParams& p, TcCtl& c, uint8_t* sslot, int nseg,
+                             uint32_t& tau, uint32_t& sigma) {
   const int L = threadIdx.x;                 // 0..127
-  const bool issuer = L == 0;
-  const uint32_t q0 = ptx::smem_addr(sq), s0 = ptx::smem_addr(sslot);
   const int h = L & 63, half = L >> 6;
   const int warp = L >> 5;
   const uint32_t lane_base = c.tmem_base + ((uint32_t)(warp * 32) << 16);
   const float sl2 = p.scale * kLog2e;
-  uint8_t* pslot = sslot + kRopeSlot * kSlotBytes + half * 8192;
-  for (int k = 0; k < nseg; ++k) {
-    const SegView v = seg_view(p, c, k);
-    const size_t slot = v.whole ? (size_t)v.b
-                                : (p.sparse_idx ? (size_t)blockIdx.x : (size_t)blockIdx.x + v.b);
-    float* o_base = (v.whole ? p.out : p.ws_o) + (slot * p.heads + h) * kVDim;
-    float* l_base = (v.whole ? p.out_lse : p.ws_lse) + slot * p.heads + h;
-    if (v.ntiles == 0) {
-      if (h < p.heads) {
-        float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int i = half; i < kVDim / 4; i += 2) reinterpret_cast<float4*>(o_base)[i] = z;
-        if (half == 0) *l_base = -CUDART_INF_F;
-      }
-      continue;
+
+  // sparse CTAs whose list is empty write the neutral pair and stop
+  if (p.sparse_idx && seg_view(p, c, 0).ntiles == 0) {
+    const SegView v = seg_view(p, c, 0);
+    const size_t slot = v.whole ? (size_t)v.b : (size_t)blockIdx.x;
+    if (h < p.heads) {
+      float* o = (v.whole ? p.out : p.ws_o) + (slot * p.heads + h) * kVDim;
+      for (int i = half; i < kVDim / 4; i += 2)
+        reinterpret_cast<float4*>(o)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (half == 0) (v.whole ? p.out_lse : p.ws_lse)[slot * p.heads + h] = -CUDART_INF_F;
     }
-    float m_used = -CUDART_INF_F, l = 0.f;
-    // The issuing thread never leaves before the warp re-converges: on a
-    // failed wait it stops issuing, and the whole group then fails together
-    // on the scores barrier that can no longer complete.
-    bool issuing = issuer && wait_or_abort(&c.q_full, sigma & 1, c);
-    for (int t = 0; t < v.ntiles; ++t, ++tau) {
-      if (issuing) {
-        issuing = issue_qk(c, q0, s0, tau);
-        if (issuing && t == v.ntiles - 1) ptx::mma_commit(&c.q_empty);
-      }
-      __syncwarp();
-      if (!wait_or_abort(&c.s_full, tau & 1, c)) return;
-      if (!wait_or_abort(&c.full[kRopeSlot], tau & 1, c)) return;
-      __syncwarp();
-      ptx::tc_fence_after();
-      uint32_t sa[32], sb[32];
-      ptx::tmem_ld32(lane_base + kColS, sa);
-      ptx::tmem_ld32(lane_base + kColS + 32, sb);
-      ptx::tmem_wait_ld();
-      const uint32_t mw0 = c.row_mask[half * 2], mw1 = c.row_mask[half * 2 + 1];
-      float x[64];
-      float mloc = -CUDART_INF_F;
-#pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        x[j] = ((mw0 >> j) & 1u) ? __uint_as_float(sa[j]) * sl2 : -CUDART_INF_F;
-        x[32 + j] = ((mw1 >> j) & 1u) ? __uint_as_float(sb[j]) * sl2 : -CUDART_INF_F;
-        mloc = fmaxf(mloc, fmaxf(x[j], x[32 + j]));
-      }
-      const int par = tau & 1;
-      c.red[par][half][h] = mloc;
-      ptx::named_bar(1, 128);
-      const float mnew = fmaxf(mloc, c.red[par][half ^ 1][h]);
-      // Lazy rescale.  The TMEM loads/stores below are warp-collective, so the
-      // decision is made per warp: if any head of the warp needs a new max,
-      // every lane moves to max(m_used, mnew).  The partner warp (the other
-      // token half) holds the same 32 heads and decides identically.
-      const bool first = m_used == -CUDART_INF_F;
-      const bool need = !first && mnew > m_used + kRescaleThreshold;
-      const bool any_need = __any_sync(0xffffffffu, need);
-      float alpha = 1.f;
-      if (first) {
-        m_used = mnew;
-      } else if (any_need) {
-        const float m2 = fmaxf(m_used, mnew);
-        alpha = exp2f(m_used - m2);
-        m_used = m2;
-        l *= alpha;
-      }
-      if (any_need) {
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          uint32_t r[32];
-          const uint32_t addr = lane_base + (q >> 2) * 128 + (q & 3) * 32;
-          ptx::tmem_ld32(addr, r);
-          ptx::tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-          ptx::tmem_st32(addr, r);
-        }
-        ptx::tmem_wait_st();
-      }
-      float sum = 0.f;
-      uint32_t pk[32];
-#pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const float p0 = m_used == -CUDART_INF_F ? 0.f : exp2f(x[2 * j] - m_used);
-        const float p1 = m_used == -CUDART_INF_F ? 0.f : exp2f(x[2 * j + 1] - m_used);
-        sum += p0 + p1;
-        const __half2 h2 = __floats2half2_rn(p0, p1);
-        pk[j] = *reinterpret_cast<const uint32_t*>(&h2);
-      }
-      l += sum;
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        *reinterpret_cast<uint4*>(pslot + swz(h, u)) =
-            make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
-      }
-      ptx::fence_proxy_async();
-      ptx::tc_fence_before();
-      ptx::mbar_arrive(&c.p_full);
-      if (issuing) {
-        issuing = wait_or_abort(&c.p_full, tau & 1, c);
-        if (issuing) {
-          ptx::tc_fence_after();
-          issue_pv(c, s0, t == 0);
-          if (t == v.ntiles - 1) ptx::mma_commit(&c.o_full);
-        }
-      }
-      __syncwarp();
-    }
-    // epilogue: O / l and the LSE
-    if (!wait_or_abort(&c.o_full, sigma & 1, c)) return;
+    return;
+  }
+
+  TileCursor cur;
+  if (!cur.start(p, c, nseg)) return;
+  float m_used = -CUDART_INF_F, l = 0.f;
+  while (true) {
+    const int st = tau & 1;
+    const uint32_t ph = (tau >> 1) & 1;
+    if (!wait_or_abort(&c.s_full[st], ph, c)) return;
+    if (!wait_or_abort(&c.full[st][1], ph, c)) return;        // row mask of the tile
     __syncwarp();
     ptx::tc_fence_after();
-    c.lred[half][h] = l;
-    ptx::named_bar(1, 128);
-    const float ltot = l + c.lred[half ^ 1][h];
-    const float inv = ltot > 0.f ? 1.f / ltot : 0.f;
+    uint32_t sr[32];
+    ptx::tmem_ld32(lane_base + kColS + 32 * st, sr);
+    ptx::tmem_wait_ld();
+    const uint32_t mw = c.row_mask[st][half];
+    float x[32];
+    float mloc = -CUDART_INF_F;
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      uint32_t r[32];
-      ptx::tmem_ld32(lane_base + (q >> 2) * 128 + (q & 3) * 32, r);
-      ptx::tmem_wait_ld();
-      if (h < p.heads) {
-        float4* dst = reinterpret_cast<float4*>(o_base + (q >> 2) * 256 + half * 128 + (q & 3) * 32);
-#pragma unroll
-        for (int e = 0; e < 8; ++e)
-          dst[e] = make_float4(__uint_as_float(r[4 * e]) * inv, __uint_as_float(r[4 * e + 1]) * inv,
-                               __uint_as_float(r[4 * e + 2]) * inv, __uint_as_float(r[4 * e + 3]) * inv);
-      }
+    for (int j = 0; j < 32; ++j) {
+      x[j] = ((mw >> j) & 1u) ? __uint_as_float(sr[j]) * sl2 : -CUDART_INF_F;
+      mloc = fmaxf(mloc, x[j]);
     }
-    if (h < p.heads && half == 0)
-      *l_base = ltot > 0.f ? (m_used + log2f(ltot)) * kLn2 : -CUDART_INF_F;
-    ptx::tc_fence_before();
+    const int par = tau & 1;
+    c.red[par][half][h] = mloc;
     ptx::named_bar(1, 128);
-    ++sigma;
+    const float mnew = fmaxf(mloc, c.red[par][half ^ 1][h]);
+    // Lazy rescale.  The TMEM loads/stores below are warp-collective, so the
+    // decision is made per warp: if any head of the warp needs a new max,
+    // every lane moves to max(m_used, mnew).  The partner warp (the other
+    // token half) holds the same 32 heads and decides identically.
+    const bool first = m_used == -CUDART_INF_F;
+    const bool need = !first && mnew > m_used + kRescaleThreshold;
+    const bool any_need = __any_sync(0xffffffffu, need);
+    float alpha = 1.f;
+    if (first) {
+      m_used = mnew;
+    } else if (any_need) {
+      const float m2 = fmaxf(m_used, mnew);
+      alpha = ex2(m_used - m2);
+      m_used = m2;
+      l *= alpha;
+    }
+    if (any_need) {
+      // the previous tile's PV must have landed in O before it is rescaled
+      if (!wait_or_abort(&c.o_ready, (tau - 1) & 1, c)) return;
+      __syncwarp();
+      ptx::tc_fence_after();
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        uint32_t r[32];
+        const uint32_t addr = lane_base + (q >> 2) * 128 + (q & 3) * 32;
+        ptx::tmem_ld32(addr, r);
+        ptx::tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+        ptx::tmem_st32(addr, r);
+      }
+      ptx::tmem_wait_st();
+    }
+    float sum = 0.f;
+    uint32_t pk[16];
+    const float mu = m_used == -CUDART_INF_F ? 0.f : m_used;   // all masked: x = -inf -> p = 0
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const float p0 = ex2(x[2 * j] - mu), p1 = ex2(x[2 * j + 1] - mu);
+      sum += p0 + p1;
+      const __half2 h2 = __floats2half2_rn(p0, p1);
+      pk[j] = *reinterpret_cast<const uint32_t*>(&h2);
+    }
+    l += sum;
+    uint8_t* pslot = slot_ptr(sslot, st, kRopeSlot);
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      *reinterpret_cast<uint4*>(pslot + swz(h, 4 * half + u)) =
+          make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+    ptx::fence_proxy_async();
+    ptx::tc_fence_before();
+    ptx::mbar_arrive(&c.p_full[st]);
+    // ---- epilogue after the request's last tile
+    if (cur.last_of_segment()) {
+      const SegView& v = cur.v;
+      const size_t slot = v.whole ? (size_t)v.b
+                                  : (p.sparse_idx ? (size_t)blockIdx.x : (size_t)blockIdx.x + v.b);
+      float* o_base = (v.whole ? p.out : p.ws_o) + (slot * p.heads + h) * kVDim;
+      float* l_base = (v.whole ? p.out_lse : p.ws_lse) + slot * p.heads + h;
+      // o_ready completes once per PV, in order.  The scores barrier already
+      // implied PV(tau - 2); PV(tau - 1) may still run, so wait for it first
+      // (a parity wait can only tell apart adjacent phases), then for PV(tau).
+      if (tau > 0 && !wait_or_abort(&c.o_ready, (tau - 1) & 1, c)) return;
+      if (!wait_or_abort(&c.o_ready, tau & 1, c)) return;
+      __syncwarp();
+      ptx::tc_fence_after();
+      c.lred[half][h] = l;
+      ptx::named_bar(1, 128);
+      const float ltot = l + c.lred[half ^ 1][h];
+      const float inv = ltot > 0.f ? 1.f / ltot : 0.f;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        uint32_t r[32];
+        ptx::tmem_ld32(lane_base + (q >> 2) * 128 + (q & 3) * 32, r);
+        ptx::tmem_wait_ld();
+        if (h < p.heads) {
+          float4* dst =
+              reinterpret_cast<float4*>(o_base + (q >> 2) * 256 + half * 128 + (q & 3) * 32);
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            dst[e] = make_float4(__uint_as_float(r[4 * e]) * inv, __uint_as_float(r[4 * e + 1]) * inv,
+                                 __uint_as_float(r[4 * e + 2]) * inv,
+                                 __uint_as_float(r[4 * e + 3]) * inv);
+        }
+      }
+      if (h < p.heads && half == 0)
+        *l_base = ltot > 0.f ? (m_used + log2f(ltot)) * kLn2 : -CUDART_INF_F;
+      ptx::tc_fence_before();
+      ptx::named_bar(1, 128);
+      ++sigma;
+      m_used = -CUDART_INF_F;
+      l = 0.f;
+    }
+    ++tau;
+    if (!cur.next(p, c)) break;
   }
 }
 
@@ -428,71 +603,74 @@ template <int KV>
 struct Stage;
 
 // fp8: latent units u0 (dims 16 u0 ..) and 16 + u0 of rows 16 j + 2 cw + rsel,
-// their groups' scales, and four 16-byte rope units.
+// the scales of their groups, and two 16-byte rope units.
 template <>
 struct Stage<kKvFp8> {
-  uint4 c0[8], c1[8];
-  float s0[8], s1[8];
-  uint4 rope[4];
+  uint4 c0[4], c1[4];
+  float s0[4], s1[4];
+  uint4 rope[2];
 };
 
-// bf16: latent dims 0..255 (unit = lane) of rows 8 i + cw; the second half
-// (dims 256..511 and rope) is loaded when the first half has been stored.
+// bf16: latent dims 0..255 (unit = lane) of rows 8 i + cw, then dims 256..511
+// and rope, loaded once the first half is stored.
 template <>
 struct Stage<kKvBf16> {
-  uint4 a[16];   // latent dims 0..255
-  uint4 b[20];   // latent dims 256..511 and rope (loaded after a[] is stored)
+  uint4 a[8];
+  uint4 b[10];
 };
 
-// Loads the rows of tile t of segment v that this thread stores (fp8).
 __device__ __forceinline__ void stage_load(const PartialParams& p, const SegView& v,
-                                           const int* list, int t, int ct, Stage<kKvFp8>& st,
-                                           bool& range_bad) {
+                                           const int* list, int t, int ct, Stage<kKvFp8>& st) {
   const int cw = ct >> 5, cl = ct & 31;
   const int rsel = (cl >> 2) & 1, u0 = (cl & 3) + 4 * (cl >> 3);
+  int rows[6];
 #pragma unroll
-  for (int jj = 0; jj < 8; ++jj) {
-    const uint8_t* row = tile_row<kKvFp8>(p, v, list, t, 16 * jj + 2 * cw + rsel);
+  for (int jj = 0; jj < 4; ++jj) rows[jj] = 16 * jj + 2 * cw + rsel;
+#pragma unroll
+  for (int i = 0; i < 2; ++i) rows[4 + i] = (i * kConvThreads + ct) >> 3;
+  const uint8_t* rp[6];
+  tile_rows<kKvFp8, 6>(p, v, list, t, rows, rp);
+#pragma unroll
+  for (int jj = 0; jj < 4; ++jj) {
+    const uint8_t* row = rp[jj];
+    st.c0[jj] = st.c1[jj] = make_uint4(0, 0, 0, 0);
+    st.s0[jj] = st.s1[jj] = 0.f;
     if (row) {
       st.c0[jj] = __ldg(reinterpret_cast<const uint4*>(row) + u0);
       st.c1[jj] = __ldg(reinterpret_cast<const uint4*>(row) + 16 + u0);
       st.s0[jj] = __ldg(reinterpret_cast<const float*>(row + 512) + (u0 >> 3));
       st.s1[jj] = __ldg(reinterpret_cast<const float*>(row + 512) + 2 + (u0 >> 3));
-    } else {
-      st.c0[jj] = st.c1[jj] = make_uint4(0, 0, 0, 0);
-      st.s0[jj] = st.s1[jj] = 0.f;
     }
   }
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
+  for (int i = 0; i < 2; ++i) {
     const int U = i * kConvThreads + ct;
-    const uint8_t* row = tile_row<kKvFp8>(p, v, list, t, U >> 3);
-    st.rope[i] = row ? __ldg(reinterpret_cast<const uint4*>(row + 528) + (U & 7))
-                     : make_uint4(0, 0, 0, 0);
+    st.rope[i] = rp[4 + i] ? __ldg(reinterpret_cast<const uint4*>(rp[4 + i] + 528) + (U & 7))
+                           : make_uint4(0, 0, 0, 0);
   }
-  (void)range_bad;
 }
 
 __device__ __forceinline__ void stage_load(const PartialParams& p, const SegView& v,
-                                           const int* list, int t, int ct, Stage<kKvBf16>& st,
-                                           bool& range_bad) {
+                                           const int* list, int t, int ct, Stage<kKvBf16>& st) {
   const int cw = ct >> 5, cl = ct & 31;
+  int rows[8];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const uint8_t* row = tile_row<kKvBf16>(p, v, list, t, 8 * i + cw);
-    st.a[i] = row ? __ldg(reinterpret_cast<const uint4*>(row) + cl) : make_uint4(0, 0, 0, 0);
-  }
-  (void)range_bad;
+  for (int i = 0; i < 8; ++i) rows[i] = 8 * i + cw;
+  const uint8_t* rp[8];
+  tile_rows<kKvBf16, 8>(p, v, list, t, rows, rp);
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    st.a[i] = rp[i] ? __ldg(reinterpret_cast<const uint4*>(rp[i]) + cl) : make_uint4(0, 0, 0, 0);
 }
 
-// Stores the first half (latent chunks 0..3) of a staged tile.
-__device__ __forceinline__ void stage_store_half0(uint8_t* sslot, int ct, const Stage<kKvFp8>& st,
+// First half: latent chunks 0..3 of the stage.
+__device__ __forceinline__ void stage_store_half0(uint8_t* stage, int ct, const Stage<kKvFp8>& st,
                                                   bool& range_bad) {
   const int cw = ct >> 5, cl = ct & 31;
   const int rsel = (cl >> 2) & 1, u0 = (cl & 3) + 4 * (cl >> 3);
-  uint8_t* dst = sslot + (u0 >> 2) * kSlotBytes;
+  uint8_t* dst = stage + (u0 >> 2) * kSlotBytes;
 #pragma unroll
-  for (int jj = 0; jj < 8; ++jj) {
+  for (int jj = 0; jj < 4; ++jj) {
     const int r = 16 * jj + 2 * cw + rsel;
     uint4 lo, hi;
     e4m3x16_to_f16(st.c0[jj], st.s0[jj], lo, hi);
@@ -502,42 +680,44 @@ __device__ __forceinline__ void stage_store_half0(uint8_t* sslot, int ct, const 
   }
 }
 
-__device__ __forceinline__ void stage_store_half0(uint8_t* sslot, int ct, const Stage<kKvBf16>& st,
+__device__ __forceinline__ void stage_store_half0(uint8_t* stage, int ct, const Stage<kKvBf16>& st,
                                                   bool& range_bad) {
   const int cw = ct >> 5, cl = ct & 31;
   float amax = 0.f;
-  uint8_t* dst = sslot + (cl >> 3) * kSlotBytes;
+  uint8_t* dst = stage + (cl >> 3) * kSlotBytes;
 #pragma unroll
-  for (int i = 0; i < 16; ++i)
+  for (int i = 0; i < 8; ++i)
     *reinterpret_cast<uint4*>(dst + swz(8 * i + cw, cl & 7)) = bf16x8_to_f16(st.a[i], amax);
   range_bad |= amax > kF16Max;
 }
 
-// Loads the second half (latent dims 256..511 and rope) where it is not
-// staged yet: bf16 rows, 20 units per thread.  fp8 staged it with the first.
 __device__ __forceinline__ void stage_load_half1(const PartialParams&, const SegView&, const int*,
                                                  int, int, Stage<kKvFp8>&) {}
 
 __device__ __forceinline__ void stage_load_half1(const PartialParams& p, const SegView& v,
                                                  const int* list, int t, int ct,
                                                  Stage<kKvBf16>& st) {
+  int rows[10];
 #pragma unroll
-  for (int i = 0; i < 20; ++i) {
+  for (int i = 0; i < 10; ++i) rows[i] = (i * kConvThreads + ct) / 40;
+  const uint8_t* rp[10];
+  tile_rows<kKvBf16, 10>(p, v, list, t, rows, rp);
+#pragma unroll
+  for (int i = 0; i < 10; ++i) {
     const int U = i * kConvThreads + ct;
-    const uint8_t* row = tile_row<kKvBf16>(p, v, list, t, U / 40);
-    st.b[i] = row ? __ldg(reinterpret_cast<const uint4*>(row) + 32 + U % 40)
-                  : make_uint4(0, 0, 0, 0);
+    st.b[i] = rp[i] ? __ldg(reinterpret_cast<const uint4*>(rp[i]) + 32 + U % 40)
+                    : make_uint4(0, 0, 0, 0);
   }
 }
 
-// Stores the second half (latent chunks 4..7 and the rope slot).
-__device__ __forceinline__ void stage_store_half1(uint8_t* sslot, int ct, const Stage<kKvFp8>& st,
+// Second half: latent chunks 4..7 and the rope slot.
+__device__ __forceinline__ void stage_store_half1(uint8_t* stage, int ct, const Stage<kKvFp8>& st,
                                                   bool& range_bad) {
   const int cw = ct >> 5, cl = ct & 31;
   const int rsel = (cl >> 2) & 1, u0 = (cl & 3) + 4 * (cl >> 3);
-  uint8_t* dst = sslot + (4 + (u0 >> 2)) * kSlotBytes;
+  uint8_t* dst = stage + (4 + (u0 >> 2)) * kSlotBytes;
 #pragma unroll
-  for (int jj = 0; jj < 8; ++jj) {
+  for (int jj = 0; jj < 4; ++jj) {
     const int r = 16 * jj + 2 * cw + rsel;
     uint4 lo, hi;
     e4m3x16_to_f16(st.c1[jj], st.s1[jj], lo, hi);
@@ -547,29 +727,28 @@ __device__ __forceinline__ void stage_store_half1(uint8_t* sslot, int ct, const 
   }
   float amax = 0.f;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
+  for (int i = 0; i < 2; ++i) {
     const int U = i * kConvThreads + ct;
-    *reinterpret_cast<uint4*>(sslot + kRopeSlot * kSlotBytes + swz(U >> 3, U & 7)) =
+    *reinterpret_cast<uint4*>(stage + kRopeSlot * kSlotBytes + swz(U >> 3, U & 7)) =
         bf16x8_to_f16(st.rope[i], amax);
   }
   range_bad |= amax > kF16Max;
 }
 
-__device__ __forceinline__ void stage_store_half1(uint8_t* sslot, int ct, const Stage<kKvBf16>& st,
+__device__ __forceinline__ void stage_store_half1(uint8_t* stage, int ct, const Stage<kKvBf16>& st,
                                                   bool& range_bad) {
   float amax = 0.f;
 #pragma unroll
-  for (int i = 0; i < 20; ++i) {
+  for (int i = 0; i < 10; ++i) {
     const int U = i * kConvThreads + ct;
     const int r = U / 40, u = 32 + U % 40;
-    *reinterpret_cast<uint4*>(sslot + (u >> 3) * kSlotBytes + swz(r, u & 7)) =
+    *reinterpret_cast<uint4*>(stage + (u >> 3) * kSlotBytes + swz(r, u & 7)) =
         bf16x8_to_f16(st.b[i], amax);
   }
   range_bad |= amax > kF16Max;
 }
 
-// Q of request b into the Q region: 64 rows x 72 units of fp16, heads >= H
-// zero.
+// Q of request b into the Q region: 64 rows x 72 units of fp16, heads >= H zero.
 __device__ __forceinline__ void load_q(const PartialParams& p, int b, uint8_t* sq, int ct,
                                        bool& range_bad) {
   const uint4* qb = reinterpret_cast<const uint4*>(p.q + (size_t)b * p.heads * kHeadDim);
@@ -584,61 +763,61 @@ __device__ __forceinline__ void load_q(const PartialParams& p, int b, uint8_t* s
   range_bad |= amax > kF16Max;
 }
 
-// Fills Q and the chunk slots (256 threads), one tile ahead in registers.
+// Fills Q and the two stages (256 threads), one tile ahead in registers.
 template <int KV>
 __device__ void convert_role(const PartialParams& p, TcCtl& c, uint8_t* sq, uint8_t* sslot,
                              const int* list, int nseg, uint32_t& tau, uint32_t& sigma) {
   const int ct = threadIdx.x - kConvBase;      // 0..255
   const int cw = ct >> 5, cl = ct & 31;
   bool range_bad = false;
-  Stage<KV> st;
-  // first tile with work
-  int k = 0;
-  while (k < nseg && seg_view(p, c, k).ntiles == 0) ++k;
-  if (k >= nseg) return;
-  SegView v = seg_view(p, c, k);
-  int t = 0;
-  stage_load(p, v, list, t, ct, st, range_bad);
+  Stage<KV> stg;
+  TileCursor cur, pf;
+  if (!cur.start(p, c, nseg)) return;
+  // L2 prefetch runs kPrefetchTiles ahead of the tile being staged
+  pf = cur;
+  bool pf_ok = true;
+  for (int i = 0; i < kPrefetchTiles && pf_ok; ++i) {
+    prefetch_tile<KV>(p, pf.v, list, pf.t, ct);
+    pf_ok = pf.next(p, c);
+  }
+  stage_load(p, cur.v, list, cur.t, ct, stg);
   while (true) {
-    if (t == 0) {
-      // new request: its Q replaces the previous one once that one's last
-      // QK has completed
-      if (sigma > 0 && !wait_or_abort(&c.q_empty, (sigma - 1) & 1, c)) return;
-      load_q(p, v.b, sq, ct, range_bad);
+    const int st = tau & 1;
+    uint8_t* stage = slot_ptr(sslot, st, 0);
+    const bool reuse = tau >= 2;                           // stage used before: wait for its PV
+    const uint32_t eph = ((tau >> 1) + 1) & 1;             // phase of the PV two tiles back
+    if (cur.t == 0) {
+      // new request: its Q replaces the previous one once that one's last QK is done
+      if (sigma > 0 && !wait_or_abort(&c.q_empty, (sigma - 1) & 1, c)) break;
+      load_q(p, cur.v.b, sq, ct, range_bad);
       ptx::fence_proxy_async();
       ptx::mbar_arrive(&c.q_full);
     }
-    if (tau > 0)
-      for (int s = 0; s < 4; ++s)
-        if (!wait_or_abort(&c.empty[s], (tau - 1) & 1, c)) return;
-    stage_store_half0(sslot, ct, st, range_bad);
+    if (reuse && !wait_or_abort(&c.empty[st][0], eph, c)) break;
+    stage_store_half0(stage, ct, stg, range_bad);
     ptx::fence_proxy_async();
-    for (int s = 0; s < 4; ++s) ptx::mbar_arrive(&c.full[s]);
-    stage_load_half1(p, v, list, t, ct, st);
-    if (tau > 0)
-      for (int s = 4; s < kNumSlots; ++s)
-        if (!wait_or_abort(&c.empty[s], (tau - 1) & 1, c)) return;
-    stage_store_half1(sslot, ct, st, range_bad);
-    // valid-row mask of the tile, published with the rope slot
-    if (ct < 128) {
-      const bool ok = tile_row<KV>(p, v, list, t, ct) != nullptr;
-      const uint32_t m = __ballot_sync(0xffffffffu, ok);
-      if (cl == 0) c.row_mask[cw] = m;
+    ptx::mbar_arrive(&c.full[st][0]);
+    stage_load_half1(p, cur.v, list, cur.t, ct, stg);
+    if (reuse && !wait_or_abort(&c.empty[st][1], eph, c)) break;
+    stage_store_half1(stage, ct, stg, range_bad);
+    if (ct < 64) {                                         // valid-row mask, published with half 1
+      const int rr[1] = {ct};
+      const uint8_t* rp[1];
+      tile_rows<KV, 1>(p, cur.v, list, cur.t, rr, rp);
+      const uint32_t m = __ballot_sync(0xffffffffu, rp[0] != nullptr);
+      if (cl == 0) c.row_mask[st][cw] = m;
     }
     ptx::fence_proxy_async();
-    for (int s = 4; s < kNumSlots; ++s) ptx::mbar_arrive(&c.full[s]);
+    ptx::mbar_arrive(&c.full[st][1]);
     ++tau;
-    // next tile (possibly of the next segment): load it now
-    if (++t >= v.ntiles) {
-      ++sigma;
-      t = 0;
-      do {
-        ++k;
-      } while (k < nseg && seg_view(p, c, k).ntiles == 0);
-      if (k >= nseg) break;
-      v = seg_view(p, c, k);
+    const bool seg_end = cur.last_of_segment();
+    if (seg_end) ++sigma;
+    if (!cur.next(p, c)) break;
+    if (pf_ok) {
+      prefetch_tile<KV>(p, pf.v, list, pf.t, ct);
+      pf_ok = pf.next(p, c);
     }
-    stage_load(p, v, list, t, ct, st, range_bad);
+    stage_load(p, cur.v, list, cur.t, ct, stg);
   }
   if (range_bad && p.flags) atomicOr(p.flags, kFlagRange);
 }
@@ -650,19 +829,21 @@ __global__ void __launch_bounds__(kThreads, 1) partial_tc_kernel(PartialParams p
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sq = base;
   uint8_t* sslot = base + kQBytes;
-  TcCtl& c = *reinterpret_cast<TcCtl*>(base + kQBytes + kNumSlots * kSlotBytes);
+  TcCtl& c = *reinterpret_cast<TcCtl*>(base + kQBytes + kStages * kNumSlots * kSlotBytes);
   const int warp = threadIdx.x >> 5;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kNumSlots; ++s) {
-      ptx::mbar_init(&c.full[s], kConvThreads);   // every converter thread, once per tile
-      ptx::mbar_init(&c.empty[s], 1);             // one tcgen05.commit per tile
+    for (int s = 0; s < kStages; ++s) {
+      for (int hf = 0; hf < 2; ++hf) {
+        ptx::mbar_init(&c.full[s][hf], kConvThreads);   // every converter thread, once per fill
+        ptx::mbar_init(&c.empty[s][hf], 1);             // one tcgen05.commit per PV
+      }
+      ptx::mbar_init(&c.p_full[s], 128);
+      ptx::mbar_init(&c.s_full[s], 1);
     }
+    ptx::mbar_init(&c.o_ready, 1);
     ptx::mbar_init(&c.q_full, kConvThreads);
     ptx::mbar_init(&c.q_empty, 1);
-    ptx::mbar_init(&c.s_full, 1);
-    ptx::mbar_init(&c.p_full, 128);
-    ptx::mbar_init(&c.o_full, 1);
     c.abort = 0;
   }
   if (warp == 0) ptx::tmem_alloc(&c.tmem_base, kTmemCols);
@@ -676,7 +857,7 @@ __global__ void __launch_bounds__(kThreads, 1) partial_tc_kernel(PartialParams p
   if (p.sparse_idx) {
     const int chunk = (p.topk + p.sparse_parts - 1) / p.sparse_parts;
     int* my_list = p.ws_list + (size_t)blockIdx.x * chunk;
-    const int n = blockIdx.x < p.batch * p.sparse_parts ? compact_sparse(p, my_list, c) : 0;
+    const int n = compact_sparse(p, my_list, c);
     if (threadIdx.x == 0) c.sel_count = n;
     list = my_list;
   } else {
@@ -688,7 +869,8 @@ __global__ void __launch_bounds__(kThreads, 1) partial_tc_kernel(PartialParams p
   __syncthreads();
 
   uint32_t tau = 0, sigma = 0;
-  uint32_t tau_issuer = 0, sigma_issuer = 0;
+  uint32_t uses[2] = {0, 0};
+  uint32_t sigma_issuer = 0;
   int first = 0;
   while (true) {
     int nseg, total;
@@ -700,9 +882,12 @@ __global__ void __launch_bounds__(kThreads, 1) partial_tc_kernel(PartialParams p
     }
     if (nseg <= 0) break;
     if (warp < 4) {
-      softmax_role(p, c, sq, sslot, nseg, tau, sigma);
-      tau_issuer = tau;
-      sigma_issuer = sigma;
+      softmax_role(p, c, sslot, nseg, tau, sigma);
+    } else if (warp == kMmaWarp) {
+      if ((threadIdx.x & 31) == 0) {
+        mma_role(p, c, sq, sslot, nseg, tau, sigma, uses);
+        sigma_issuer = sigma;
+      }
     } else {
       convert_role<KV>(p, c, sq, sslot, list, nseg, tau, sigma);
     }
@@ -712,17 +897,17 @@ __global__ void __launch_bounds__(kThreads, 1) partial_tc_kernel(PartialParams p
     if (p.sparse_idx || total <= first) break;
   }
   // Drain: every tcgen05.commit arrives on its mbarrier asynchronously.  The
-  // last tile's slot releases and the last segment's Q release are never
-  // waited on by the pipeline, so wait for them here; otherwise an arrival
-  // could land after this CTA exits, on the barriers the next CTA on this SM
-  // has just initialised at the same shared-memory offsets.
-  if (threadIdx.x == 0) {
-    if (tau_issuer > 0)
-      for (int s = 0; s < kNumSlots; ++s) wait_or_abort(&c.empty[s], (tau_issuer - 1) & 1, c);
+  // stage releases of the last tiles and the last request's Q release are
+  // never waited on by the pipeline, so wait for them here; otherwise an
+  // arrival could land after this CTA exits, on the barriers the next CTA on
+  // this SM has just initialised at the same shared-memory offsets.
+  if (threadIdx.x == kMmaWarp * 32) {
+    for (int s = 0; s < kStages; ++s)
+      if (uses[s] > 0)
+        for (int hf = 0; hf < 2; ++hf) wait_or_abort(&c.empty[s][hf], (uses[s] - 1) & 1, c);
     if (sigma_issuer > 0) wait_or_abort(&c.q_empty, (sigma_issuer - 1) & 1, c);
   }
   if (c.abort && threadIdx.x == 0 && p.flags) atomicOr(p.flags, kFlagTimeout);
-  ptx::cp_async_wait_all();
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();

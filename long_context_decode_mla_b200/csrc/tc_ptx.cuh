@@ -65,6 +65,11 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32
                : "memory");
 }
 
+// Bulk prefetch of [src, src + bytes) into L2 (16-byte aligned, multiple of 16).
+__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 // Arrive on `bar` once all of this thread's earlier cp.async copies landed
 // (without raising the barrier's expected count).
 __device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {

@@ -1,10 +1,15 @@
 """GPU-vs-oracle parity of the whole emulated DCP step, through the C ABI.
 
-Tolerances (stated by the target, applied to every shard's partials and to the
-merged result): bf16 cache max|dO| <= 2e-3 * max|O| and |dLSE| <= 1e-4; fp8
-cache max|dO| <= 2e-2 * max|O| and |dLSE| <= 1e-3 (the LSE bound for fp8 is a
-reading: the target states none).  Empty shards must return exactly (0, -inf).
-Addressing and sparse selection are checked bit-exactly with id-coded rows.
+Tolerances, applied to every shard's partials and to the merged result: bf16
+cache max|dO| <= 2e-3 * max|O| and |dLSE| <= 1e-4, fp8 cache max|dO| <=
+2e-2 * max|O| (all stated by the target).  The target states no LSE bound for
+fp8 rows; it is derived from the arithmetic: the tensor cores read e4m3 *
+scale rounded to fp16 (relative error <= 2^-10 after the two roundings of the
+fp16 product), so a score moves by about 0.072 * 2^-10 * sqrt(sum_d q_d^2
+k_d^2) ~ 1.7e-3 (rms, N(0,1) data, 512 latent values); the LSE, a softmax-
+weighted mean of score errors, stays within 5e-3 over all heads and requests.
+Empty shards must return exactly (0, -inf).  Addressing and sparse selection
+are checked bit-exactly with id-coded rows.
 """
 import math
 
@@ -18,7 +23,7 @@ from long_context_decode_mla_b200 import workload as wl
 
 pytestmark = pytest.mark.gpu
 
-TOL = {"bf16": (2e-3, 1e-4), "fp8": (2e-2, 1e-2)}
+TOL = {"bf16": (2e-3, 1e-4), "fp8": (2e-2, 5e-3)}
 IMPLS = ["simt", "auto"]
 
 
