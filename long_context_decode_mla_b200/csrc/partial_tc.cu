@@ -69,7 +69,7 @@ struct TcCtl {
   uint64_t empty[kStages][2];    // MMA -> converter, per stage and slot half (PV commits)
   uint64_t s_full[2];            // scores buffer ready (QK commit)
   uint64_t p_full[kStages];      // P written (128 softmax arrivals)
-  uint64_t o_ready;              // PV of a tile complete (commit, every tile)
+  uint64_t o_full;               // last PV of a request complete (commit, once per request)
   uint64_t q_full, q_empty;      // Q loaded (256 arrivals) / last QK of a request done
   uint32_t tmem_base;
   int abort;
@@ -223,15 +223,20 @@ __device__ __forceinline__ uint32_t f16x2_sat(float lo, float hi) {
 }
 
 // 16 e4m3 codes times `sc` -> 16 fp16 (two 16-byte units, dims in order).
-// e4m3 -> fp16 is exact; when the scale is a normal fp16 number that keeps
-// every product finite (2^-14 <= sc <= 65504 / 448) the product is taken in
-// fp16 (two instructions per pair, two roundings); otherwise in fp32 and
-// rounded once, with clamping.
+// e4m3 -> fp16 is exact.  When every product stays a finite normal-range
+// fp16 number (2^-14 <= sc <= 65504 / 448) the product is taken in fp16 with
+// the scale split into sc_hi = fp16(sc) and sc_lo = fp16(sc - sc_hi):
+// fma(code, sc_hi, code * sc_lo) rounds once per element.  Rounding the scale
+// alone would put one shared relative error (up to 2^-11) on all 128 values
+// of a group, which moves large scores coherently.  Other scales take the
+// fp32 product, rounded once, with clamping.
 __device__ __forceinline__ void e4m3x16_to_f16(const uint4 v, float sc, uint4& lo, uint4& hi) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
   uint32_t o[8];
   if (sc >= 6.103515625e-05f && sc <= 146.0f) {
-    const __half2 s2 = __float2half2_rn(sc);
+    const __half s_hi = __float2half_rn(sc);
+    const __half2 hi2 = __half2half2(s_hi);
+    const __half2 lo2 = __half2half2(__float2half_rn(sc - __half2float(s_hi)));
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
 #pragma unroll
@@ -240,7 +245,7 @@ __device__ __forceinline__ void e4m3x16_to_f16(const uint4 v, float sc, uint4& l
         const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3);
         __half2 h2;
         *reinterpret_cast<__half2_raw*>(&h2) = hr;
-        const __half2 r2 = __hmul2(h2, s2);
+        const __half2 r2 = __hfma2(h2, hi2, __hmul2(h2, lo2));
         o[2 * i + hw] = *reinterpret_cast<const uint32_t*>(&r2);
       }
     }
@@ -399,7 +404,6 @@ __device__ __forceinline__ void issue_pv(TcCtl& c, const Descs& d, uint32_t tau,
                       (!first_tile || kk > 0) ? 1u : 0u);
     ptx::mma_commit(&c.empty[st][hf]);
   }
-  ptx::mma_commit(&c.o_ready);
 }
 
 __device__ __forceinline__ float ex2(float x) {
@@ -446,7 +450,10 @@ __device__ void mma_role(const PartialParams& p, TcCtl& c, uint8_t* sq, uint8_t*
     ptx::tc_fence_after();
     issue_pv(c, dsc, tau, cur.t == 0);
     ++uses[st];
-    if (cur.last_of_segment()) ++sigma;
+    if (cur.last_of_segment()) {
+      ptx::mma_commit(&c.o_full);
+      ++sigma;
+    }
     ++tau;
     if (!cur.next(p, c)) break;
   }
@@ -516,8 +523,13 @@ __device__ void softmax_role(const PartialParams& p, TcCtl& c, uint8_t* sslot, i
       l *= alpha;
     }
     if (any_need) {
-      // the previous tile's PV must have landed in O before it is rescaled
-      if (!wait_or_abort(&c.o_ready, (tau - 1) & 1, c)) return;
+      // The previous tile's PV must have landed in O before it is rescaled:
+      // its last MMA released the second half of its stage.  That barrier's
+      // phase for tile tau - 1 is either pending or complete here (the
+      // scores barrier implied PV(tau - 2); PV(tau + 1) needs this thread's
+      // P), so the parity wait is unambiguous.
+      const uint32_t prev = tau - 1;
+      if (!wait_or_abort(&c.empty[prev & 1][1], (prev >> 1) & 1, c)) return;
       __syncwarp();
       ptx::tc_fence_after();
 #pragma unroll
@@ -558,11 +570,10 @@ __device__ void softmax_role(const PartialParams& p, TcCtl& c, uint8_t* sslot, i
                                   : (p.sparse_idx ? (size_t)blockIdx.x : (size_t)blockIdx.x + v.b);
       float* o_base = (v.whole ? p.out : p.ws_o) + (slot * p.heads + h) * kVDim;
       float* l_base = (v.whole ? p.out_lse : p.ws_lse) + slot * p.heads + h;
-      // o_ready completes once per PV, in order.  The scores barrier already
-      // implied PV(tau - 2); PV(tau - 1) may still run, so wait for it first
-      // (a parity wait can only tell apart adjacent phases), then for PV(tau).
-      if (tau > 0 && !wait_or_abort(&c.o_ready, (tau - 1) & 1, c)) return;
-      if (!wait_or_abort(&c.o_ready, tau & 1, c)) return;
+      // o_full completes once per request, after its last PV (and so after
+      // all of its PVs).  Earlier phases were consumed by earlier epilogues and
+      // the next one needs this thread's P, so the parity wait is unambiguous.
+      if (!wait_or_abort(&c.o_full, sigma & 1, c)) return;
       __syncwarp();
       ptx::tc_fence_after();
       c.lred[half][h] = l;
@@ -841,7 +852,7 @@ __global__ void __launch_bounds__(kThreads, 1) partial_tc_kernel(PartialParams p
       ptx::mbar_init(&c.p_full[s], 128);
       ptx::mbar_init(&c.s_full[s], 1);
     }
-    ptx::mbar_init(&c.o_ready, 1);
+    ptx::mbar_init(&c.o_full, 1);
     ptx::mbar_init(&c.q_full, kConvThreads);
     ptx::mbar_init(&c.q_empty, 1);
     c.abort = 0;
@@ -900,7 +911,10 @@ __global__ void __launch_bounds__(kThreads, 1) partial_tc_kernel(PartialParams p
   // stage releases of the last tiles and the last request's Q release are
   // never waited on by the pipeline, so wait for them here; otherwise an
   // arrival could land after this CTA exits, on the barriers the next CTA on
-  // this SM has just initialised at the same shared-memory offsets.
+  // this SM has just initialised at the same shared-memory offsets.  (Every
+  // other commit is consumed: scores by the softmax, o_full by the epilogue.)
+  // Each of these waits is one phase ahead of the last one consumed, so the
+  // parity is unambiguous.
   if (threadIdx.x == kMmaWarp * 32) {
     for (int s = 0; s < kStages; ++s)
       if (uses[s] > 0)
