@@ -138,6 +138,53 @@ int mla_decode_partial(const void* q, const void* kv_cache, int kv_dtype, int64_
                        void* stream);
 
 /*
+ * Bytes of the scratch array built into the library for
+ * mla_decode_partial_noalloc (32 MiB per device that calls it; enough for
+ * batch 64 x 64 heads x 148 splits, about 27.8 MB).
+ */
+#define DCPMLA_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+/*
+ * mla_decode_partial without a caller-supplied workspace.  The method's
+ * description has no counterpart to this call: it is a library convenience
+ * for callers that cannot hand the library device memory (a C host program
+ * with no device allocator of its own, or a serving loop that must not call
+ * cudaMalloc / cudaFree between steps because they synchronise the device).
+ *
+ * Arguments, layouts and results are those of mla_decode_partial, minus
+ * workspace / workspace_bytes, plus:
+ *   out_flags  NULL, or a DEVICE int32 that receives (in stream order) this
+ *              call's DCPMLA_FLAG_* bits.
+ *
+ * The workspace is a fixed DCPMLA_NOALLOC_SCRATCH_BYTES array in device
+ * memory of the library (one per device); nothing is allocated, by this call
+ * or on its behalf.  Its flag word is cleared at setup and again after every
+ * call, so each call's flags stand alone.
+ *
+ * Limits:
+ *  - A request whose mla_decode_workspace_size(batch, num_heads, num_splits,
+ *    sparse_idx ? topk : 0) exceeds DCPMLA_NOALLOC_SCRATCH_BYTES returns
+ *    DCPMLA_ERR_WORKSPACE before any work is enqueued.
+ *  - Every call on a device uses the same scratch: calls whose work overlaps
+ *    on the device (different streams, different host threads) race and
+ *    corrupt each other's results.  Serialise them, e.g. on one stream.
+ *  - The first call on each device (with that device current) performs the
+ *    setup: it looks the scratch array up with cudaGetSymbolAddress, which
+ *    may load the library's module, and enqueues the first clear of the flag
+ *    word.  Make that first call before any stream capture begins.
+ *
+ * Returns DCPMLA_OK or a negative DCPMLA_ERR_* code (DCPMLA_ERR_CUDA if the
+ * setup fails).
+ */
+int mla_decode_partial_noalloc(const void* q, const void* kv_cache, int kv_dtype,
+                               int64_t num_blocks, int block_size, const int32_t* block_table,
+                               int block_table_stride, const int32_t* seq_lens, int batch,
+                               int num_heads, int shard_id, int num_shards,
+                               const int32_t* sparse_idx, int topk, float softmax_scale,
+                               float* out_partial, float* out_lse, int32_t* out_flags,
+                               int num_splits, int impl, void* stream);
+
+/*
  * LSE-weighted merge of N shard partials into the full-context result.
  *
  *   partials  [num_shards][batch][num_heads][512] fp32 (16-byte aligned).

@@ -125,6 +125,48 @@ def mla_decode_partial(q, kv_cache, kv_dtype, block_table, seq_lens, shard_id, n
     _check(rc, "mla_decode_partial")
 
 
+NOALLOC_SCRATCH_BYTES = 32 << 20          # DCPMLA_NOALLOC_SCRATCH_BYTES
+_noalloc_fn = None
+
+
+def _noalloc():
+    global _noalloc_fn
+    if _noalloc_fn is None:
+        f = lib().mla_decode_partial_noalloc
+        vp, i32, i64, f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float
+        f.argtypes = [vp, vp, i32, i64, i32, vp, i32, vp, i32, i32, i32, i32, vp, i32, f32,
+                      vp, vp, vp, i32, i32, vp]
+        f.restype = i32
+        _noalloc_fn = f
+    return _noalloc_fn
+
+
+def mla_decode_partial_noalloc(q, kv_cache, kv_dtype, block_table, seq_lens, shard_id,
+                               num_shards, sparse_idx, softmax_scale, out_partial, out_lse,
+                               out_flags=None, num_splits: int = 0, impl: str | int = "auto",
+                               stream=None, block_size: int = BLOCK_SIZE,
+                               num_blocks: int | None = None):
+    """mla_decode_partial on the library's built-in scratch (see include/dcpmla.h).
+
+    For callers that cannot pass device memory for a workspace.  ``out_flags``
+    is an optional one-element int32 device tensor that receives this call's
+    flag bits.  Calls whose work overlaps on one device race on the shared
+    scratch; the first call on a device does the setup and should come before
+    any stream capture.
+    """
+    B, H = q.shape[0], q.shape[1]
+    kvd = KV_DTYPES[kv_dtype] if isinstance(kv_dtype, str) else int(kv_dtype)
+    nb = kv_cache.shape[0] if num_blocks is None else num_blocks
+    topk = 0 if sparse_idx is None else sparse_idx.shape[1]
+    impl_code = IMPLS[impl] if isinstance(impl, str) else int(impl)
+    rc = _noalloc()(
+        _ptr(q), _ptr(kv_cache), kvd, nb, block_size, _ptr(block_table), block_table.shape[-1],
+        _ptr(seq_lens), B, H, shard_id, num_shards, _ptr(sparse_idx), topk,
+        float(softmax_scale), _ptr(out_partial), _ptr(out_lse), _ptr(out_flags),
+        num_splits, impl_code, _stream(stream))
+    _check(rc, "mla_decode_partial_noalloc")
+
+
 def dcp_merge(partials, lses, out, out_lse=None, stream=None):
     """LSE-weighted merge of [N, B, H, 512] partials (see include/dcpmla.h)."""
     N, B, H = partials.shape[0], partials.shape[1], partials.shape[2]

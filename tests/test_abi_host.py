@@ -116,3 +116,30 @@ def test_head_envelope_matches_the_page_table():
         assert row["gathered"] == row["local"] * row["dcp"]
         assert dcpmla.padded_heads(row["local"]) == row["local_pad"]
         assert dcpmla.padded_heads(row["gathered"]) == row["gathered_pad"]
+
+
+def test_noalloc_refuses_before_touching_the_device():
+    """Refusals of mla_decode_partial_noalloc come from host checks alone."""
+    L = dcpmla.lib()
+    f = L.mla_decode_partial_noalloc
+    vp, i32, i64, f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float
+    f.argtypes = [vp, vp, i32, i64, i32, vp, i32, vp, i32, i32, i32, i32, vp, i32, f32,
+                  vp, vp, vp, i32, i32, vp]
+    f.restype = i32
+
+    def call(batch, heads, splits, topk=0, sparse=None):
+        return f(None, None, 0, 1, 64, None, 1, None, batch, heads, 0, 1, sparse, topk, 1.0,
+                 None, None, None, splits, 0, None)
+
+    need = dcpmla.mla_decode_workspace_size(600, 64, 148)
+    assert need > dcpmla.NOALLOC_SCRATCH_BYTES
+    assert call(600, 64, 148) == EWS                 # beyond the built-in scratch
+    assert call(4, 0, 148) == EINVAL                 # bad sizes fail before the size check
+    assert call(-1, 64, 148) == EINVAL
+    assert call(4, 65, 148) == EUNSUP
+
+
+def test_noalloc_scratch_size_matches_header():
+    text = open(HEADER).read()
+    m = re.search(r"#define DCPMLA_NOALLOC_SCRATCH_BYTES \((\d+)u << (\d+)\)", text)
+    assert m and int(m.group(1)) << int(m.group(2)) == dcpmla.NOALLOC_SCRATCH_BYTES
