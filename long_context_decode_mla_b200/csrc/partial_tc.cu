@@ -522,6 +522,25 @@ __device__ void softmax_role(const PartialParams& p, TcCtl& c, uint8_t* sslot, i
       m_used = m2;
       l *= alpha;
     }
+    float sum = 0.f;
+    uint32_t pk[16];
+    const float mu = m_used == -CUDART_INF_F ? 0.f : m_used;   // all masked: x = -inf -> p = 0
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const float p0 = ex2(x[2 * j] - mu), p1 = ex2(x[2 * j + 1] - mu);
+      sum += p0 + p1;
+      const __half2 h2 = __floats2half2_rn(p0, p1);
+      pk[j] = *reinterpret_cast<const uint32_t*>(&h2);
+    }
+    l += sum;
+    uint8_t* pslot = slot_ptr(sslot, st, kRopeSlot);
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      *reinterpret_cast<uint4*>(pslot + swz(h, 4 * half + u)) =
+          make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+    // O is rescaled after P is written, so that the scores are no longer held
+    // in registers while O passes through them (P does not depend on O; it
+    // only has to be in place before p_full, like the rescaled O).
     if (any_need) {
       // The previous tile's PV must have landed in O before it is rescaled:
       // its last MMA released the second half of its stage.  That barrier's
@@ -544,22 +563,6 @@ __device__ void softmax_role(const PartialParams& p, TcCtl& c, uint8_t* sslot, i
       }
       ptx::tmem_wait_st();
     }
-    float sum = 0.f;
-    uint32_t pk[16];
-    const float mu = m_used == -CUDART_INF_F ? 0.f : m_used;   // all masked: x = -inf -> p = 0
-#pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      const float p0 = ex2(x[2 * j] - mu), p1 = ex2(x[2 * j + 1] - mu);
-      sum += p0 + p1;
-      const __half2 h2 = __floats2half2_rn(p0, p1);
-      pk[j] = *reinterpret_cast<const uint32_t*>(&h2);
-    }
-    l += sum;
-    uint8_t* pslot = slot_ptr(sslot, st, kRopeSlot);
-#pragma unroll
-    for (int u = 0; u < 4; ++u)
-      *reinterpret_cast<uint4*>(pslot + swz(h, 4 * half + u)) =
-          make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
     ptx::fence_proxy_async();
     ptx::tc_fence_before();
     ptx::mbar_arrive(&c.p_full[st]);
