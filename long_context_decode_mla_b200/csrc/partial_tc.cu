@@ -222,6 +222,36 @@ __device__ __forceinline__ uint32_t f16x2_sat(float lo, float hi) {
   return r;
 }
 
+// e4m3 pair (16 bits) -> fp16 pair, exact.
+__device__ __forceinline__ __half2 e4m3x2_to_f16x2(uint32_t pair) {
+  const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(pair & 0xFFFFu), __NV_E4M3);
+  __half2 h2;
+  *reinterpret_cast<__half2_raw*>(&h2) = hr;
+  return h2;
+}
+
+// Scales outside the fp16 fast path (rare): fp32 products rounded once,
+// with clamping; returns true if a product was clamped.  Kept out of line
+// so the hot conversion code stays small.
+__device__ __noinline__ bool e4m3x16_to_f16_slow(const uint4 v, float sc, uint4& lo, uint4& hi) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t o[8];
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+#pragma unroll
+    for (int hw = 0; hw < 2; ++hw) {
+      const float2 f = __half22float2(e4m3x2_to_f16x2(w[i] >> (16 * hw)));
+      const float a = f.x * sc, b = f.y * sc;
+      amax = fmaxf(amax, fmaxf(fabsf(a), fabsf(b)));
+      o[2 * i + hw] = f16x2_sat(a, b);
+    }
+  }
+  lo = make_uint4(o[0], o[1], o[2], o[3]);
+  hi = make_uint4(o[4], o[5], o[6], o[7]);
+  return amax > kF16Max;
+}
+
 // 16 e4m3 codes times `sc` -> 16 fp16 (two 16-byte units, dims in order).
 // e4m3 -> fp16 is exact.  When every product stays a finite normal-range
 // fp16 number (2^-14 <= sc <= 65504 / 448) the product is taken in fp16 with
@@ -229,42 +259,27 @@ __device__ __forceinline__ uint32_t f16x2_sat(float lo, float hi) {
 // fma(code, sc_hi, code * sc_lo) rounds once per element.  Rounding the scale
 // alone would put one shared relative error (up to 2^-11) on all 128 values
 // of a group, which moves large scores coherently.  Other scales take the
-// fp32 product, rounded once, with clamping.
-__device__ __forceinline__ void e4m3x16_to_f16(const uint4 v, float sc, uint4& lo, uint4& hi) {
+// fp32 product, rounded once, with clamping.  Returns true if a product was
+// clamped (only possible off the fast path).
+__device__ __forceinline__ bool e4m3x16_to_f16(const uint4 v, float sc, uint4& lo, uint4& hi) {
+  if (!(sc >= 6.103515625e-05f && sc <= 146.0f)) return e4m3x16_to_f16_slow(v, sc, lo, hi);
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
   uint32_t o[8];
-  if (sc >= 6.103515625e-05f && sc <= 146.0f) {
-    const __half s_hi = __float2half_rn(sc);
-    const __half2 hi2 = __half2half2(s_hi);
-    const __half2 lo2 = __half2half2(__float2half_rn(sc - __half2float(s_hi)));
+  const __half s_hi = __float2half_rn(sc);
+  const __half2 hi2 = __half2half2(s_hi);
+  const __half2 lo2 = __half2half2(__float2half_rn(sc - __half2float(s_hi)));
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
+  for (int i = 0; i < 4; ++i) {
 #pragma unroll
-      for (int hw = 0; hw < 2; ++hw) {
-        const __nv_fp8x2_storage_t pair = (__nv_fp8x2_storage_t)((w[i] >> (16 * hw)) & 0xFFFFu);
-        const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3);
-        __half2 h2;
-        *reinterpret_cast<__half2_raw*>(&h2) = hr;
-        const __half2 r2 = __hfma2(h2, hi2, __hmul2(h2, lo2));
-        o[2 * i + hw] = *reinterpret_cast<const uint32_t*>(&r2);
-      }
-    }
-  } else {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-#pragma unroll
-      for (int hw = 0; hw < 2; ++hw) {
-        const __nv_fp8x2_storage_t pair = (__nv_fp8x2_storage_t)((w[i] >> (16 * hw)) & 0xFFFFu);
-        const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3);
-        __half2 h2;
-        *reinterpret_cast<__half2_raw*>(&h2) = hr;
-        const float2 f = __half22float2(h2);
-        o[2 * i + hw] = f16x2_sat(f.x * sc, f.y * sc);
-      }
+    for (int hw = 0; hw < 2; ++hw) {
+      const __half2 h2 = e4m3x2_to_f16x2(w[i] >> (16 * hw));
+      const __half2 r2 = __hfma2(h2, hi2, __hmul2(h2, lo2));
+      o[2 * i + hw] = *reinterpret_cast<const uint32_t*>(&r2);
     }
   }
   lo = make_uint4(o[0], o[1], o[2], o[3]);
   hi = make_uint4(o[4], o[5], o[6], o[7]);
+  return false;
 }
 
 // 8 bf16 -> 8 fp16; `amax` collects the largest magnitude seen.
@@ -415,7 +430,7 @@ __device__ __forceinline__ float ex2(float x) {
 // Issues every MMA (one thread of the MMA warp): the scores of the next tile
 // before the PV of this one, so that the softmax of tile t overlaps the
 // scores of tile t + 1.
-__device__ void mma_role(const PartialParams& p, TcCtl& c, uint8_t* sq, uint8_t* sslot, int nseg,
+__device__ __forceinline__ void mma_role(const PartialParams& p, TcCtl& c, uint8_t* sq, uint8_t* sslot, int nseg,
                          uint32_t& tau, uint32_t& sigma, uint32_t (&uses)[2]) {
   Descs dsc;
   {
@@ -460,7 +475,7 @@ __device__ void mma_role(const PartialParams& p, TcCtl& c, uint8_t* sq, uint8_t*
 }
 
 // Online softmax, P and the epilogue (128 threads, one TMEM lane each).
-__device__ void softmax_role(const PartialParams& p, TcCtl& c, uint8_t* sslot, int nseg,
+__device__ __forceinline__ void softmax_role(const PartialParams& p, TcCtl& c, uint8_t* sslot, int nseg,
                              uint32_t& tau, uint32_t& sigma) {
   const int L = threadIdx.x;                 // 0..127
   const int h = L & 63, half = L >> 6;
@@ -687,8 +702,7 @@ __device__ __forceinline__ void stage_store_half0(uint8_t* stage, int ct, const 
   for (int jj = 0; jj < 4; ++jj) {
     const int r = 16 * jj + 2 * cw + rsel;
     uint4 lo, hi;
-    e4m3x16_to_f16(st.c0[jj], st.s0[jj], lo, hi);
-    range_bad |= st.s0[jj] * 448.f > kF16Max;
+    range_bad |= e4m3x16_to_f16(st.c0[jj], st.s0[jj], lo, hi);
     *reinterpret_cast<uint4*>(dst + swz(r, (u0 & 3) * 2)) = lo;
     *reinterpret_cast<uint4*>(dst + swz(r, (u0 & 3) * 2 + 1)) = hi;
   }
@@ -734,8 +748,7 @@ __device__ __forceinline__ void stage_store_half1(uint8_t* stage, int ct, const 
   for (int jj = 0; jj < 4; ++jj) {
     const int r = 16 * jj + 2 * cw + rsel;
     uint4 lo, hi;
-    e4m3x16_to_f16(st.c1[jj], st.s1[jj], lo, hi);
-    range_bad |= st.s1[jj] * 448.f > kF16Max;
+    range_bad |= e4m3x16_to_f16(st.c1[jj], st.s1[jj], lo, hi);
     *reinterpret_cast<uint4*>(dst + swz(r, (u0 & 3) * 2)) = lo;
     *reinterpret_cast<uint4*>(dst + swz(r, (u0 & 3) * 2 + 1)) = hi;
   }
@@ -779,7 +792,7 @@ __device__ __forceinline__ void load_q(const PartialParams& p, int b, uint8_t* s
 
 // Fills Q and the two stages (256 threads), one tile ahead in registers.
 template <int KV>
-__device__ void convert_role(const PartialParams& p, TcCtl& c, uint8_t* sq, uint8_t* sslot,
+__device__ __forceinline__ void convert_role(const PartialParams& p, TcCtl& c, uint8_t* sq, uint8_t* sslot,
                              const int* list, int nseg, uint32_t& tau, uint32_t& sigma) {
   const int ct = threadIdx.x - kConvBase;      // 0..255
   const int cw = ct >> 5, cl = ct & 31;
@@ -836,8 +849,13 @@ __device__ void convert_role(const PartialParams& p, TcCtl& c, uint8_t* sq, uint
   if (range_bad && p.flags) atomicOr(p.flags, kFlagRange);
 }
 
-template <int KV>
-__global__ void __launch_bounds__(kThreads, 1) partial_tc_kernel(PartialParams p) {
+// kSparse is fixed per instantiation: the dense kernel sees a null index
+// list at compile time, so none of the sparse paths are compiled into it
+// (a smaller kernel keeps its four concurrent roles in the instruction cache).
+template <int KV, bool kSparse>
+__global__ void __launch_bounds__(kThreads, 1) partial_tc_kernel(const PartialParams pin) {
+  PartialParams p = pin;
+  if constexpr (!kSparse) p.sparse_idx = nullptr;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -941,14 +959,17 @@ bool tc_supports(const PartialParams& p, int kv_dtype) {
 cudaError_t launch_partial_tc(const PartialParams& p, int kv_dtype, cudaStream_t st) {
   const int grid = p.sparse_idx ? p.batch * p.sparse_parts : p.num_ctas;
   const int smem = (int)kSmemBytes;
-  auto kernel = kv_dtype == kKvBf16 ? partial_tc_kernel<kKvBf16> : partial_tc_kernel<kKvFp8>;
+  const bool sparse = p.sparse_idx != nullptr;
+  auto kernel = kv_dtype == kKvBf16
+                    ? (sparse ? partial_tc_kernel<kKvBf16, true> : partial_tc_kernel<kKvBf16, false>)
+                    : (sparse ? partial_tc_kernel<kKvFp8, true> : partial_tc_kernel<kKvFp8, false>);
   // Raise the shared-memory limit once per kernel and device, so that later
   // launches (including ones captured into a CUDA graph) are plain launches.
-  static int configured[2][64] = {};
+  static int configured[4][64] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  int& done = configured[kv_dtype == kKvBf16 ? 0 : 1][dev & 63];
+  int& done = configured[(kv_dtype == kKvBf16 ? 0 : 2) + (sparse ? 1 : 0)][dev & 63];
   if (!done) {
     e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;

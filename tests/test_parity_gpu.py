@@ -277,3 +277,39 @@ def test_growing_scores_force_mixed_rescales(impl, kv_dtype):
     q[:, ::3] = 0                                     # every third head never rescales
     prob = wl.DecodeProblem(q, cache, kv_dtype, tables, lens, 2)
     _check_problem(prob, impl, num_splits=1)
+
+
+@pytest.mark.parametrize("impl", IMPLS)
+def test_fp8_scales_outside_the_fp16_fast_path(impl):
+    """Group scales above 65504 / 448 (codes capped at +-384 so every product
+    stays finite) and below 2^-14 take the fp32 conversion path of the
+    tensor-core kernel; they must match the oracle like any other scale.
+    Request 0 has every scale at 160, request 1 every scale at 3e-5, request
+    2 a random mix of 160, 3e-5 and ordinary scales.  The queries of requests
+    0 and 2 are scaled down so that scores stay O(1)."""
+    g = torch.Generator().manual_seed(31)
+    L = 2500
+    rows = []
+    for b in range(3):
+        x = torch.randn(L, 576, generator=g)
+        r = wl.pack_fp8_rows(x[:, :512], x[:, 512:])
+        codes = r[:, :512]
+        big = codes & 0x7F > 0x7C                      # |value| > 384 -> 384, sign kept
+        r[:, :512] = torch.where(big, (codes & 0x80) | 0x7C, codes)
+        scales = r[:, 512:528].contiguous().view(torch.float32).view(L, 4)
+        if b == 0:
+            scales = torch.full_like(scales, 160.0)
+        elif b == 1:
+            scales = torch.full_like(scales, 3e-5)
+        else:
+            choice = torch.randint(0, 3, (L, 4), generator=g)
+            scales = torch.where(choice == 0, torch.full_like(scales, 160.0),
+                                 torch.where(choice == 1, torch.full_like(scales, 3e-5), scales))
+        r[:, 512:528] = scales.contiguous().view(torch.uint8).view(L, 16)
+        rows.append(r)
+    cache, tables, lens = wl.place_rows(rows, 2, "fp8", seed=5)
+    q = wl.random_q(3, 64, 31).float()
+    q[0] *= 1e-4
+    q[2] *= 1e-4
+    prob = wl.DecodeProblem(q.to(torch.bfloat16), cache, "fp8", tables, lens, 2)
+    _check_problem(prob, impl, num_splits=3)
