@@ -54,6 +54,12 @@ constexpr int kRopeSlot = 8;
 constexpr int kStages = 2;
 constexpr int kQBytes = 9 * 8192;
 constexpr int kMaxSeg = 128;
+// A stage is filled, and its scores issued, in five parts: the four 128-value
+// scale groups of the latent row (two 64-value chunk slots each, 8 K-steps)
+// and the rope slot (4 K-steps).  The MMA starts on a part as soon as it
+// lands, so little of QK is left once the last part is stored.
+constexpr int kParts = 5;
+constexpr int kRopePart = 4;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 256;        // S buffers: columns [256, 288) and [288, 320); O: [0, 256)
 constexpr float kLog2e = 1.4426950408889634f;
@@ -65,7 +71,7 @@ constexpr int kFlagRange = 8;
 constexpr float kF16Max = 65504.f;
 
 struct TcCtl {
-  uint64_t full[kStages][2];     // converter -> MMA, per stage and slot half (256 arrivals)
+  uint64_t full[kStages][kParts]; // converter -> MMA, per stage and part (256 arrivals)
   uint64_t empty[kStages][2];    // MMA -> converter, per stage and slot half (PV commits)
   uint64_t s_full[2];            // scores buffer ready (QK commit)
   uint64_t p_full[kStages];      // P written (128 softmax arrivals)
@@ -381,27 +387,40 @@ __device__ __forceinline__ uint64_t dplus(uint64_t d, uint32_t byte_off) {
   return d + (uint64_t)(byte_off >> 4);
 }
 
-// MMA issue (one thread): S[tau & 1] = Q K^T for tile tau (stage tau & 1).
-// Chunks 0..3 go first: they are refilled while the previous use of the stage
-// still runs its second PV half.
-__device__ __forceinline__ bool issue_qk(TcCtl& c, const Descs& d, uint32_t tau) {
+// MMA issue (one thread): S[tau & 1] = Q K^T for tile tau (stage tau & 1),
+// part by part as the converters publish them (K-steps 8k .. 8k+7 for scale
+// group k, 32 .. 35 for the rope).
+template <int kPart>
+__device__ __forceinline__ void issue_qk_part(const TcCtl& c, const Descs& d, uint64_t kd,
+                                              uint32_t dst) {
   constexpr uint32_t kIdQK = ptx::idesc_f16(64, 64, false);
+  constexpr int k0 = 8 * kPart, k1 = kPart == kRopePart ? 36 : 8 * kPart + 8;
+#pragma unroll
+  for (int ks = k0; ks < k1; ++ks)
+    ptx::mma_ws_f16(dst, dplus(d.q, (ks >> 2) * 8192 + (ks & 3) * 32),
+                    dplus(kd, (ks >> 2) * kSlotBytes + (ks & 3) * 32), kIdQK, ks > 0);
+}
+
+__device__ __forceinline__ bool issue_qk(TcCtl& c, const Descs& d, uint32_t tau) {
   const int st = tau & 1;
   const uint32_t ph = (tau >> 1) & 1;
   const uint64_t kd = st ? d.k[1] : d.k[0];
   const uint32_t dst = c.tmem_base + kColS + 32 * st;
   if (!wait_or_abort(&c.full[st][0], ph, c)) return false;
   ptx::tc_fence_after();
-#pragma unroll
-  for (int ks = 0; ks < 16; ++ks)
-    ptx::mma_ws_f16(dst, dplus(d.q, (ks >> 2) * 8192 + (ks & 3) * 32),
-                    dplus(kd, (ks >> 2) * kSlotBytes + (ks & 3) * 32), kIdQK, ks > 0);
+  issue_qk_part<0>(c, d, kd, dst);
   if (!wait_or_abort(&c.full[st][1], ph, c)) return false;
   ptx::tc_fence_after();
-#pragma unroll
-  for (int ks = 16; ks < 36; ++ks)
-    ptx::mma_ws_f16(dst, dplus(d.q, (ks >> 2) * 8192 + (ks & 3) * 32),
-                    dplus(kd, (ks >> 2) * kSlotBytes + (ks & 3) * 32), kIdQK, 1u);
+  issue_qk_part<1>(c, d, kd, dst);
+  if (!wait_or_abort(&c.full[st][2], ph, c)) return false;
+  ptx::tc_fence_after();
+  issue_qk_part<2>(c, d, kd, dst);
+  if (!wait_or_abort(&c.full[st][3], ph, c)) return false;
+  ptx::tc_fence_after();
+  issue_qk_part<3>(c, d, kd, dst);
+  if (!wait_or_abort(&c.full[st][kRopePart], ph, c)) return false;
+  ptx::tc_fence_after();
+  issue_qk_part<kRopePart>(c, d, kd, dst);
   ptx::mma_commit(&c.s_full[st]);
   return true;
 }
@@ -503,7 +522,7 @@ __device__ __forceinline__ void softmax_role(const PartialParams& p, TcCtl& c, u
     const int st = tau & 1;
     const uint32_t ph = (tau >> 1) & 1;
     if (!wait_or_abort(&c.s_full[st], ph, c)) return;
-    if (!wait_or_abort(&c.full[st][1], ph, c)) return;        // row mask of the tile
+    if (!wait_or_abort(&c.full[st][kRopePart], ph, c)) return;   // row mask of the tile
     __syncwarp();
     ptx::tc_fence_after();
     uint32_t sr[32];
@@ -631,12 +650,14 @@ __device__ __forceinline__ void softmax_role(const PartialParams& p, TcCtl& c, u
 template <int KV>
 struct Stage;
 
-// fp8: latent units u0 (dims 16 u0 ..) and 16 + u0 of rows 16 j + 2 cw + rsel,
-// the scales of their groups, and two 16-byte rope units.
+// fp8: thread ct stages rows 32 i + (ct >> 3) (i = 0, 1) of the tile: of each
+// 128-value scale group g, the 16-value unit u = ct & 7 of both rows with
+// the group's scale, and rope unit u.  Eight threads cover a row, so each
+// load is part of a contiguous 128-byte run of the row.
 template <>
 struct Stage<kKvFp8> {
-  uint4 c0[4], c1[4];
-  float s0[4], s1[4];
+  uint4 c[4][2];
+  float s[4][2];
   uint4 rope[2];
 };
 
@@ -650,32 +671,19 @@ struct Stage<kKvBf16> {
 
 __device__ __forceinline__ void stage_load(const PartialParams& p, const SegView& v,
                                            const int* list, int t, int ct, Stage<kKvFp8>& st) {
-  const int cw = ct >> 5, cl = ct & 31;
-  const int rsel = (cl >> 2) & 1, u0 = (cl & 3) + 4 * (cl >> 3);
-  int rows[6];
-#pragma unroll
-  for (int jj = 0; jj < 4; ++jj) rows[jj] = 16 * jj + 2 * cw + rsel;
-#pragma unroll
-  for (int i = 0; i < 2; ++i) rows[4 + i] = (i * kConvThreads + ct) >> 3;
-  const uint8_t* rp[6];
-  tile_rows<kKvFp8, 6>(p, v, list, t, rows, rp);
-#pragma unroll
-  for (int jj = 0; jj < 4; ++jj) {
-    const uint8_t* row = rp[jj];
-    st.c0[jj] = st.c1[jj] = make_uint4(0, 0, 0, 0);
-    st.s0[jj] = st.s1[jj] = 0.f;
-    if (row) {
-      st.c0[jj] = __ldg(reinterpret_cast<const uint4*>(row) + u0);
-      st.c1[jj] = __ldg(reinterpret_cast<const uint4*>(row) + 16 + u0);
-      st.s0[jj] = __ldg(reinterpret_cast<const float*>(row + 512) + (u0 >> 3));
-      st.s1[jj] = __ldg(reinterpret_cast<const float*>(row + 512) + 2 + (u0 >> 3));
-    }
-  }
+  const int u = ct & 7;
+  const int rows[2] = {ct >> 3, 32 + (ct >> 3)};
+  const uint8_t* rp[2];
+  tile_rows<kKvFp8, 2>(p, v, list, t, rows, rp);
 #pragma unroll
   for (int i = 0; i < 2; ++i) {
-    const int U = i * kConvThreads + ct;
-    st.rope[i] = rp[4 + i] ? __ldg(reinterpret_cast<const uint4*>(rp[4 + i] + 528) + (U & 7))
-                           : make_uint4(0, 0, 0, 0);
+    const uint8_t* row = rp[i];
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      st.c[g][i] = row ? __ldg(reinterpret_cast<const uint4*>(row) + 8 * g + u) : make_uint4(0, 0, 0, 0);
+      st.s[g][i] = row ? __ldg(reinterpret_cast<const float*>(row + 512) + g) : 0.f;
+    }
+    st.rope[i] = row ? __ldg(reinterpret_cast<const uint4*>(row + 528) + u) : make_uint4(0, 0, 0, 0);
   }
 }
 
@@ -692,22 +700,35 @@ __device__ __forceinline__ void stage_load(const PartialParams& p, const SegView
     st.a[i] = rp[i] ? __ldg(reinterpret_cast<const uint4*>(rp[i]) + cl) : make_uint4(0, 0, 0, 0);
 }
 
-// First half: latent chunks 0..3 of the stage.
-__device__ __forceinline__ void stage_store_half0(uint8_t* stage, int ct, const Stage<kKvFp8>& st,
+// fp8 scale group g: latent dims 128 g .. 128 g + 127, chunk slots 2 g and
+// 2 g + 1 of the stage.
+template <int g>
+__device__ __forceinline__ void stage_store_group(uint8_t* stage, int ct, const Stage<kKvFp8>& st,
                                                   bool& range_bad) {
-  const int cw = ct >> 5, cl = ct & 31;
-  const int rsel = (cl >> 2) & 1, u0 = (cl & 3) + 4 * (cl >> 3);
-  uint8_t* dst = stage + (u0 >> 2) * kSlotBytes;
+  const int u = ct & 7;
+  uint8_t* dst = stage + (2 * g + (u >> 2)) * kSlotBytes;
 #pragma unroll
-  for (int jj = 0; jj < 4; ++jj) {
-    const int r = 16 * jj + 2 * cw + rsel;
+  for (int i = 0; i < 2; ++i) {
+    const int r = 32 * i + (ct >> 3);
     uint4 lo, hi;
-    range_bad |= e4m3x16_to_f16(st.c0[jj], st.s0[jj], lo, hi);
-    *reinterpret_cast<uint4*>(dst + swz(r, (u0 & 3) * 2)) = lo;
-    *reinterpret_cast<uint4*>(dst + swz(r, (u0 & 3) * 2 + 1)) = hi;
+    range_bad |= e4m3x16_to_f16(st.c[g][i], st.s[g][i], lo, hi);
+    *reinterpret_cast<uint4*>(dst + swz(r, (u & 3) * 2)) = lo;
+    *reinterpret_cast<uint4*>(dst + swz(r, (u & 3) * 2 + 1)) = hi;
   }
 }
 
+// fp8 rope units (bf16 -> fp16) into the rope slot.
+__device__ __forceinline__ void stage_store_rope(uint8_t* stage, int ct, const Stage<kKvFp8>& st,
+                                                 bool& range_bad) {
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 2; ++i)
+    *reinterpret_cast<uint4*>(stage + kRopeSlot * kSlotBytes + swz(32 * i + (ct >> 3), ct & 7)) =
+        bf16x8_to_f16(st.rope[i], amax);
+  range_bad |= amax > kF16Max;
+}
+
+// bf16, first half: latent chunks 0..3 of the stage.
 __device__ __forceinline__ void stage_store_half0(uint8_t* stage, int ct, const Stage<kKvBf16>& st,
                                                   bool& range_bad) {
   const int cw = ct >> 5, cl = ct & 31;
@@ -718,9 +739,6 @@ __device__ __forceinline__ void stage_store_half0(uint8_t* stage, int ct, const 
     *reinterpret_cast<uint4*>(dst + swz(8 * i + cw, cl & 7)) = bf16x8_to_f16(st.a[i], amax);
   range_bad |= amax > kF16Max;
 }
-
-__device__ __forceinline__ void stage_load_half1(const PartialParams&, const SegView&, const int*,
-                                                 int, int, Stage<kKvFp8>&) {}
 
 __device__ __forceinline__ void stage_load_half1(const PartialParams& p, const SegView& v,
                                                  const int* list, int t, int ct,
@@ -738,30 +756,7 @@ __device__ __forceinline__ void stage_load_half1(const PartialParams& p, const S
   }
 }
 
-// Second half: latent chunks 4..7 and the rope slot.
-__device__ __forceinline__ void stage_store_half1(uint8_t* stage, int ct, const Stage<kKvFp8>& st,
-                                                  bool& range_bad) {
-  const int cw = ct >> 5, cl = ct & 31;
-  const int rsel = (cl >> 2) & 1, u0 = (cl & 3) + 4 * (cl >> 3);
-  uint8_t* dst = stage + (4 + (u0 >> 2)) * kSlotBytes;
-#pragma unroll
-  for (int jj = 0; jj < 4; ++jj) {
-    const int r = 16 * jj + 2 * cw + rsel;
-    uint4 lo, hi;
-    range_bad |= e4m3x16_to_f16(st.c1[jj], st.s1[jj], lo, hi);
-    *reinterpret_cast<uint4*>(dst + swz(r, (u0 & 3) * 2)) = lo;
-    *reinterpret_cast<uint4*>(dst + swz(r, (u0 & 3) * 2 + 1)) = hi;
-  }
-  float amax = 0.f;
-#pragma unroll
-  for (int i = 0; i < 2; ++i) {
-    const int U = i * kConvThreads + ct;
-    *reinterpret_cast<uint4*>(stage + kRopeSlot * kSlotBytes + swz(U >> 3, U & 7)) =
-        bf16x8_to_f16(st.rope[i], amax);
-  }
-  range_bad |= amax > kF16Max;
-}
-
+// bf16, second half: latent chunks 4..7 and the rope slot.
 __device__ __forceinline__ void stage_store_half1(uint8_t* stage, int ct, const Stage<kKvBf16>& st,
                                                   bool& range_bad) {
   float amax = 0.f;
@@ -790,7 +785,8 @@ __device__ __forceinline__ void load_q(const PartialParams& p, int b, uint8_t* s
   range_bad |= amax > kF16Max;
 }
 
-// Fills Q and the two stages (256 threads), one tile ahead in registers.
+// Fills Q and the two stages (256 threads), one tile ahead in registers, and
+// publishes each stage in kParts parts (fp8: per scale group, then rope).
 template <int KV>
 __device__ __forceinline__ void convert_role(const PartialParams& p, TcCtl& c, uint8_t* sq, uint8_t* sslot,
                              const int* list, int nseg, uint32_t& tau, uint32_t& sigma) {
@@ -820,14 +816,39 @@ __device__ __forceinline__ void convert_role(const PartialParams& p, TcCtl& c, u
       ptx::fence_proxy_async();
       ptx::mbar_arrive(&c.q_full);
     }
+    // chunks 0..3 (scale groups 0, 1) are free once the first PV half of the
+    // tile two back is done, chunks 4..7 and the rope slot after the second
     if (reuse && !wait_or_abort(&c.empty[st][0], eph, c)) break;
-    stage_store_half0(stage, ct, stg, range_bad);
-    ptx::fence_proxy_async();
-    ptx::mbar_arrive(&c.full[st][0]);
-    stage_load_half1(p, cur.v, list, cur.t, ct, stg);
+    if constexpr (KV == kKvFp8) {
+      stage_store_group<0>(stage, ct, stg, range_bad);
+      ptx::fence_proxy_async();
+      ptx::mbar_arrive(&c.full[st][0]);
+      stage_store_group<1>(stage, ct, stg, range_bad);
+      ptx::fence_proxy_async();
+      ptx::mbar_arrive(&c.full[st][1]);
+    } else {
+      stage_store_half0(stage, ct, stg, range_bad);
+      ptx::fence_proxy_async();
+      ptx::mbar_arrive(&c.full[st][0]);
+      ptx::mbar_arrive(&c.full[st][1]);
+      stage_load_half1(p, cur.v, list, cur.t, ct, stg);
+    }
     if (reuse && !wait_or_abort(&c.empty[st][1], eph, c)) break;
-    stage_store_half1(stage, ct, stg, range_bad);
-    if (ct < 64) {                                         // valid-row mask, published with half 1
+    if constexpr (KV == kKvFp8) {
+      stage_store_group<2>(stage, ct, stg, range_bad);
+      ptx::fence_proxy_async();
+      ptx::mbar_arrive(&c.full[st][2]);
+      stage_store_group<3>(stage, ct, stg, range_bad);
+      ptx::fence_proxy_async();
+      ptx::mbar_arrive(&c.full[st][3]);
+      stage_store_rope(stage, ct, stg, range_bad);
+    } else {
+      stage_store_half1(stage, ct, stg, range_bad);
+      ptx::fence_proxy_async();
+      ptx::mbar_arrive(&c.full[st][2]);
+      ptx::mbar_arrive(&c.full[st][3]);
+    }
+    if (ct < 64) {                                         // valid-row mask, published with the rope
       const int rr[1] = {ct};
       const uint8_t* rp[1];
       tile_rows<KV, 1>(p, cur.v, list, cur.t, rr, rp);
@@ -835,7 +856,7 @@ __device__ __forceinline__ void convert_role(const PartialParams& p, TcCtl& c, u
       if (cl == 0) c.row_mask[st][cw] = m;
     }
     ptx::fence_proxy_async();
-    ptx::mbar_arrive(&c.full[st][1]);
+    ptx::mbar_arrive(&c.full[st][kRopePart]);
     ++tau;
     const bool seg_end = cur.last_of_segment();
     if (seg_end) ++sigma;
@@ -866,10 +887,9 @@ __global__ void __launch_bounds__(kThreads, 1) partial_tc_kernel(const PartialPa
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      for (int hf = 0; hf < 2; ++hf) {
-        ptx::mbar_init(&c.full[s][hf], kConvThreads);   // every converter thread, once per fill
-        ptx::mbar_init(&c.empty[s][hf], 1);             // one tcgen05.commit per PV
-      }
+      for (int k = 0; k < kParts; ++k)
+        ptx::mbar_init(&c.full[s][k], kConvThreads);    // every converter thread, once per fill
+      for (int hf = 0; hf < 2; ++hf) ptx::mbar_init(&c.empty[s][hf], 1);   // one commit per PV half
       ptx::mbar_init(&c.p_full[s], 128);
       ptx::mbar_init(&c.s_full[s], 1);
     }
