@@ -8,3 +8,6 @@ from .mla_decode import (  # noqa: F401
     attention_with_lse, dcp_decode, dcp_merge, decode_bf16, decode_e4m3,
     decode_rows, e4m3_value, fetch_rows, local_positions, mla_decode_partial,
 )
+from .cache_write import (  # noqa: F401
+    bf16_row, encode_e4m3, kv_append, quantize_fp8_row,
+)
