@@ -201,6 +201,47 @@ int mla_decode_partial_noalloc(const void* q, const void* kv_cache, int kv_dtype
 int dcp_merge(const float* partials, const float* lses, int num_shards, int batch,
               int num_heads, float* out, float* out_lse, void* stream);
 
+/*
+ * DCP cache write of new decode tokens: this shard writes the tokens it owns.
+ *
+ * "GLM-5.2 vLLM Decode Context Parallelism", section "Keep the current-main
+ * correctness blocker visible": under DCP a token whose cache slot another
+ * rank owns gets no cache write here (its query is still processed); the
+ * write is guarded, not the query.  Ownership is round-robin ("How vLLM Serves
+ * GLM-5.3 with Million-Token Contexts on 16 H200s", "The core design"): token
+ * t belongs to shard t mod N and lands at local row j = t div N, i.e. row
+ * j % 64 of physical block block_table[b][j / 64] -- the rows
+ * mla_decode_partial reads.
+ *
+ *   latent       [num_tokens][512] bf16 (the absorbed latent, already normed),
+ *                16-byte aligned.
+ *   rope         [num_tokens][64] bf16 (rope part of the key), 16-byte aligned.
+ *   positions    [num_tokens] int32 global position t of each token (< 0:
+ *                no token, skipped).
+ *   req_idx      [num_tokens] int32 request b of each token.
+ *   block_table  [batch][block_table_stride] int32: this shard's table.
+ *   shard_id, num_shards: 0 <= shard_id < num_shards.
+ *   kv_cache     [num_blocks][64][row bytes], 16-byte aligned; rows of owned
+ *                tokens are overwritten, nothing else is touched.
+ *   kv_dtype     DCPMLA_KV_BF16: the 576 values are copied.  DCPMLA_KV_FP8:
+ *                per 128-value group g, scale_g = amax_g / 448 (1 if amax_g
+ *                is 0, fp32 division), codes = E4M3 of fp32(x / scale_g),
+ *                round to nearest even, saturated at +-448; the row holds the
+ *                512 codes, the 4 scales (fp32) and the 64 rope values (bf16).
+ *   flags        NULL, or a DEVICE int32 the kernel ORs DCPMLA_FLAG_BAD_BLOCK
+ *                (table entry outside [0, num_blocks)) and
+ *                DCPMLA_FLAG_BAD_LENGTH (request index outside [0, batch), or
+ *                a local block index beyond the table row) into; such tokens
+ *                are not written.
+ *
+ * Returns DCPMLA_OK or a negative DCPMLA_ERR_* code (checked on the host
+ * before any launch).
+ */
+int mla_kv_append(const void* latent, const void* rope, int num_tokens, const int32_t* positions,
+                  const int32_t* req_idx, const int32_t* block_table, int block_table_stride,
+                  int batch, int shard_id, int num_shards, void* kv_cache, int kv_dtype,
+                  int64_t num_blocks, int block_size, int32_t* flags, void* stream);
+
 /* Static description of a return code (never NULL). */
 const char* dcpmla_error_string(int code);
 

@@ -125,6 +125,38 @@ def mla_decode_partial(q, kv_cache, kv_dtype, block_table, seq_lens, shard_id, n
     _check(rc, "mla_decode_partial")
 
 
+_append_fn = None
+
+
+def _append():
+    global _append_fn
+    if _append_fn is None:
+        f = lib().mla_kv_append
+        vp, i32, i64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
+        f.argtypes = [vp, vp, i32, vp, vp, vp, i32, i32, i32, i32, vp, i32, i64, i32, vp, vp]
+        f.restype = i32
+        _append_fn = f
+    return _append_fn
+
+
+def mla_kv_append(latent, rope, positions, req_idx, block_table, shard_id, num_shards, kv_cache,
+                  kv_dtype, flags=None, stream=None, block_size: int = BLOCK_SIZE,
+                  num_blocks: int | None = None):
+    """This shard's cache write of new tokens (see include/dcpmla.h).
+
+    latent [T, 512] bf16, rope [T, 64] bf16, positions / req_idx [T] int32,
+    block_table [B, stride] int32 (this shard's), kv_cache the raw pool;
+    ``flags`` an optional one-element int32 device tensor.
+    """
+    T = latent.shape[0]
+    kvd = KV_DTYPES[kv_dtype] if isinstance(kv_dtype, str) else int(kv_dtype)
+    nb = kv_cache.shape[0] if num_blocks is None else num_blocks
+    rc = _append()(_ptr(latent), _ptr(rope), T, _ptr(positions), _ptr(req_idx), _ptr(block_table),
+                   block_table.shape[-1], block_table.shape[0], shard_id, num_shards,
+                   _ptr(kv_cache), kvd, nb, block_size, _ptr(flags), _stream(stream))
+    _check(rc, "mla_kv_append")
+
+
 NOALLOC_SCRATCH_BYTES = 32 << 20          # DCPMLA_NOALLOC_SCRATCH_BYTES
 _noalloc_fn = None
 

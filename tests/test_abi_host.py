@@ -143,3 +143,33 @@ def test_noalloc_scratch_size_matches_header():
     text = open(HEADER).read()
     m = re.search(r"#define DCPMLA_NOALLOC_SCRATCH_BYTES \((\d+)u << (\d+)\)", text)
     assert m and int(m.group(1)) << int(m.group(2)) == dcpmla.NOALLOC_SCRATCH_BYTES
+
+
+def _append_fn():
+    L = dcpmla.lib()
+    f = L.mla_kv_append
+    vp, i32, i64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
+    f.argtypes = [vp, vp, i32, vp, vp, vp, i32, i32, i32, i32, vp, i32, i64, i32, vp, vp]
+    f.restype = i32
+    return f
+
+
+def test_kv_append_fails_closed_before_any_launch():
+    f = _append_fn()
+    A = 0x10000                       # 16-byte aligned fake pointers: never dereferenced
+    base = dict(lat=A, rope=A, T=4, pos=A, req=A, bt=A, stride=2, B=1, s=0, N=2, cache=A,
+                kvd=1, nb=8, bs=64)
+
+    def call(**kw):
+        a = dict(base, **kw)
+        return f(a["lat"], a["rope"], a["T"], a["pos"], a["req"], a["bt"], a["stride"], a["B"],
+                 a["s"], a["N"], a["cache"], a["kvd"], a["nb"], a["bs"], None, None)
+
+    assert call(T=-1) == EINVAL
+    assert call(s=2) == EINVAL and call(s=-1) == EINVAL and call(N=0) == EINVAL
+    assert call(kvd=5) == EINVAL
+    assert call(nb=0) == EINVAL and call(B=0) == EINVAL and call(stride=0) == EINVAL
+    assert call(bs=32) == EUNSUP
+    assert call(T=0) == OK                                   # nothing to write
+    assert call(lat=None) == EINVAL and call(cache=None) == EINVAL and call(bt=None) == EINVAL
+    assert call(lat=A + 8) == EALIGN and call(cache=A + 4) == EALIGN and call(rope=A + 2) == EALIGN
