@@ -43,6 +43,8 @@ def parse():
     ap.add_argument("--kernel", default="auto", choices=["auto", "simt", "tc"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the secondary at-64K measurement")
     ap.add_argument("--shard-streams", type=int, default=None,
                     help="CUDA streams the N shard launches are spread over (default N; 1 = serial)")
     ap.add_argument("--batch", type=int, default=None,
@@ -103,10 +105,15 @@ def measured_peaks():
     return 6650.0, "fallback"
 
 
+# the sources the partial kernel (whose DRAM traffic profiles/traffic.json
+# records) is built from; other entry points do not invalidate the figure
+PARTIAL_KERNEL_SOURCES = ("common.cuh", "kernels.h", "merge.cu", "partial_tc.cu", "tc_ptx.cuh")
+
+
 def kernel_source_hash() -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "long_context_decode_mla_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in PARTIAL_KERNEL_SOURCES:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
@@ -334,10 +341,96 @@ def run_ours(args, rank, world, local):
             "gpu_launches": gpu_launches,
             "clocks": clocks,
         }
+    # secondary measurements (same rank layout; every rank runs them, rank 0 reports)
+    extras = {}
+    if args.workload == "agentic" and not args.no_extras:
+        extras["at_64k"] = time_other_workload("agentic64k", dev, rank, world, args, streams_for=N)
+    extras["kv_append"] = time_append(prob, dev, max(20, args.steps // 4))
+    if result is not None:
+        result.update(extras)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
     return result, prob
+
+
+def time_other_workload(name, dev, rank, world, args, streams_for):
+    """Graph-replayed steps of another workload (for "steps/s at 64K context")."""
+    import torch
+    from long_context_decode_mla_b200 import dcpmla, workload
+    cfg = dict(workload.CONFIGS[name])
+    prob = workload.make_problem(name, device=dev, kv_device=dev, seed=cfg["seed"] + 1000 * rank)
+    N = prob.num_shards
+    streams = [torch.cuda.Stream(device=dev) for _ in range(N)]
+    dec = dcpmla.DcpDecoder(prob.batch, prob.heads, N, device=dev, impl=args.kernel,
+                            streams=streams)
+    graph = dec.capture(prob)
+    for _ in range(max(3, args.warmup)):
+        graph.replay()
+    torch.cuda.synchronize(dev)
+    steps = max(20, args.steps // 4)
+    stream = torch.cuda.current_stream(dev)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(steps):
+        graph.replay()
+    t1.record(stream)
+    t1.synchronize()
+    assert dec.flags() == 0, "device flags set"
+    ms = max_over_ranks([t0.elapsed_time(t1) / steps])[0]
+    kvb = kv_bytes(prob)
+    desc = describe(name, prob)
+    del graph, dec, prob
+    torch.cuda.empty_cache()
+    return {"workload": desc, "steps_per_s": round(world * 1e3 / ms, 2),
+            "ms_per_step": round(ms, 4), "value": round(world * kvb / (ms * 1e-3) / 1e9, 1),
+            "unit": UNIT, "steps": steps}
+
+
+def time_append(prob, dev, steps):
+    """The DCP cache write of one new token per request on every shard
+    (mla_kv_append x N, graph-replayed).  It rewrites each request's last
+    existing token, so every write lands inside the block tables."""
+    import torch
+    from long_context_decode_mla_b200 import dcpmla
+    B, N = prob.batch, prob.num_shards
+    g = torch.Generator(device=dev).manual_seed(5)
+    lat = torch.randn(B, 512, generator=g, device=dev).to(torch.bfloat16)
+    rope = torch.randn(B, 64, generator=g, device=dev).to(torch.bfloat16)
+    pos = (prob.seq_lens - 1).to(torch.int32).contiguous()
+    req = torch.arange(B, dtype=torch.int32, device=dev)
+    flags = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def step(stream):
+        for s in range(N):
+            dcpmla.mla_kv_append(lat, rope, pos, req, prob.block_tables[s], s, N, prob.kv_cache,
+                                 prob.kv_dtype, flags, stream)
+
+    side = torch.cuda.Stream(device=dev)
+    side.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(side):
+        step(side)
+    torch.cuda.current_stream(dev).wait_stream(side)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=side):
+        step(side)
+    for _ in range(3):
+        graph.replay()
+    torch.cuda.synchronize(dev)
+    stream = torch.cuda.current_stream(dev)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(steps):
+        graph.replay()
+    t1.record(stream)
+    t1.synchronize()
+    assert int(flags.item()) == 0, "append flags set"
+    us = t0.elapsed_time(t1) / steps * 1e3
+    from long_context_decode_mla_b200.workload import ROW_BYTES
+    written = B * ROW_BYTES[prob.kv_dtype]
+    return {"us_per_step": round(us, 2), "tokens_per_s": round(B / (us * 1e-6), 1),
+            "launches_per_step": N, "bytes_written_per_step": written,
+            "note": "one new token per request, written on its owner shard (N shard calls)"}
 
 
 def describe(name, prob):

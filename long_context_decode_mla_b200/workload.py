@@ -56,6 +56,9 @@ CONFIGS = {
     "million": dict(batch=1, heads=64, seq_len=1 << 20, kv_dtype="fp8", num_shards=8, seed=1004),
     "sparse": dict(batch=128, heads=64, seq_len=131072, kv_dtype="fp8", num_shards=8,
                    topk=2048, seed=1005),
+    # the agentic shape with every request at exactly 64K tokens ("steps/s at 64K")
+    "agentic64k": dict(batch=64, heads=64, seq_len=65536, kv_dtype="fp8", num_shards=8,
+                       seed=1006),
 }
 
 LOGNORMAL_MEDIAN = 67000
