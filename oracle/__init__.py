@@ -11,3 +11,4 @@ from .mla_decode import (  # noqa: F401
 from .cache_write import (  # noqa: F401
     bf16_row, encode_e4m3, kv_append, quantize_fp8_row,
 )
+from .multi_query import dcp_decode_multi, mla_decode_partial_multi  # noqa: F401
