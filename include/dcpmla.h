@@ -138,6 +138,36 @@ int mla_decode_partial(const void* q, const void* kv_cache, int kv_dtype, int64_
                        void* stream);
 
 /*
+ * Multi-query decode (speculative / multi-token-prediction verification):
+ * q_len query tokens per request, all N shards as in mla_decode_partial.
+ *
+ * "GLM-5.2 vLLM Decode Context Parallelism", section "Add MTP only after
+ * plain decode passes": multi-token prediction adds draft-token query shapes
+ * to the same decode attention.  Reading (the pages give no formula): the
+ * cache already holds the q_len new tokens, L_b in total; query i sits at
+ * position L_b - q_len + i and attends to every cached t <= that position.
+ *
+ *   q            [batch][q_len][num_heads][576] bf16 (16-byte aligned).
+ *   num_heads    query heads per token; num_heads * q_len <= 64 (the rows of
+ *                the tensor-core tile), else DCPMLA_ERR_UNSUPPORTED.
+ *   out_partial  [batch][q_len][num_heads][512] fp32; out_lse
+ *                [batch][q_len][num_heads] fp32; queries that see no token of
+ *                this shard give (0, -inf).
+ *   workspace    mla_decode_workspace_size(batch, num_heads * q_len, ...).
+ *   impl         DCPMLA_IMPL_AUTO or DCPMLA_IMPL_TC (the CUDA-core kernel has
+ *                no causal rows: DCPMLA_ERR_UNSUPPORTED when q_len > 1).
+ * Other arguments as in mla_decode_partial (no sparse variant).  The merge is
+ * dcp_merge with num_heads * q_len rows.
+ */
+int mla_decode_partial_multi(const void* q, const void* kv_cache, int kv_dtype,
+                             int64_t num_blocks, int block_size, const int32_t* block_table,
+                             int block_table_stride, const int32_t* seq_lens, int batch,
+                             int num_heads, int q_len, int shard_id, int num_shards,
+                             float softmax_scale, float* out_partial, float* out_lse,
+                             void* workspace, size_t workspace_bytes, int num_splits, int impl,
+                             void* stream);
+
+/*
  * Bytes of the scratch array built into the library for
  * mla_decode_partial_noalloc (32 MiB per device that calls it; enough for
  * batch 64 x 64 heads x 148 splits, about 27.8 MB).

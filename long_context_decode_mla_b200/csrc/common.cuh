@@ -24,14 +24,16 @@ enum : int { kFlagBadBlock = 1, kFlagBadLength = 2 };
 
 // Everything one shard's partial-attention launch needs.
 struct PartialParams {
-  const __nv_bfloat16* q;     // [B][H][576]
+  const __nv_bfloat16* q;     // [B][H][576]; multi-query: [B][q_len][H / q_len][576]
   const uint8_t* kv;          // [num_blocks][64][row_bytes]
   long long num_blocks;
   const int* block_table;     // [B][bt_stride] this shard's table
   int bt_stride;
   const int* seq_lens;        // [B] global lengths
   int batch;
-  int heads;
+  int heads;                  // rows per request: query heads x q_len (<= 64)
+  int q_len;                  // query tokens per request (1 = plain decode); row r is
+                              // query r / (heads / q_len), causal at L_b - q_len + that
   int shard;
   int nshards;
   const int* sparse_idx;      // [B][topk] or nullptr

@@ -99,13 +99,18 @@ int mla_decode_workspace_size(int batch, int num_heads, int num_splits, int topk
   return DCPMLA_OK;
 }
 
-int mla_decode_partial(const void* q, const void* kv_cache, int kv_dtype, int64_t num_blocks,
-                       int block_size, const int32_t* block_table, int block_table_stride,
-                       const int32_t* seq_lens, int batch, int num_heads, int shard_id,
-                       int num_shards, const int32_t* sparse_idx, int topk,
-                       float softmax_scale, float* out_partial, float* out_lse,
-                       void* workspace, size_t workspace_bytes, int num_splits, int impl,
-                       void* stream) {
+}  // extern "C"
+
+namespace {
+
+// Shared body of mla_decode_partial (q_len = 1) and mla_decode_partial_multi:
+// num_heads here counts rows (query heads x q_len).
+int decode_partial(const void* q, const void* kv_cache, int kv_dtype, int64_t num_blocks,
+                   int block_size, const int32_t* block_table, int block_table_stride,
+                   const int32_t* seq_lens, int batch, int num_heads, int q_len, int shard_id,
+                   int num_shards, const int32_t* sparse_idx, int topk, float softmax_scale,
+                   float* out_partial, float* out_lse, void* workspace, size_t workspace_bytes,
+                   int num_splits, int impl, void* stream) {
   // ---- scalar checks (fail closed, nothing launched on error) ----
   if (batch < 0 || num_heads < 1 || num_shards < 1 || shard_id < 0 || shard_id >= num_shards ||
       block_size < 1 || block_table_stride < 1 || num_blocks < 1 || num_splits < 0 ||
@@ -139,6 +144,7 @@ int mla_decode_partial(const void* q, const void* kv_cache, int kv_dtype, int64_
   p.seq_lens = seq_lens;
   p.batch = batch;
   p.heads = num_heads;
+  p.q_len = q_len;
   p.shard = shard_id;
   p.nshards = num_shards;
   p.sparse_idx = sparse_idx;
@@ -157,12 +163,45 @@ int mla_decode_partial(const void* q, const void* kv_cache, int kv_dtype, int64_
   const bool tc_ok = tc_supports(p, kv_dtype);
   if (impl == DCPMLA_IMPL_TC && !tc_ok) return DCPMLA_ERR_UNSUPPORTED;
   const bool use_tc = impl == DCPMLA_IMPL_TC || (impl == DCPMLA_IMPL_AUTO && tc_ok);
+  if (q_len > 1 && !use_tc) return DCPMLA_ERR_UNSUPPORTED;   // causal rows: tensor-core kernel only
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e = use_tc ? launch_partial_tc(p, kv_dtype, st) : launch_partial_simt(p, kv_dtype, st);
   if (e != cudaSuccess) return DCPMLA_ERR_CUDA;
   e = launch_split_combine(p, st);
   return e == cudaSuccess ? DCPMLA_OK : DCPMLA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int mla_decode_partial(const void* q, const void* kv_cache, int kv_dtype, int64_t num_blocks,
+                       int block_size, const int32_t* block_table, int block_table_stride,
+                       const int32_t* seq_lens, int batch, int num_heads, int shard_id,
+                       int num_shards, const int32_t* sparse_idx, int topk,
+                       float softmax_scale, float* out_partial, float* out_lse,
+                       void* workspace, size_t workspace_bytes, int num_splits, int impl,
+                       void* stream) {
+  return decode_partial(q, kv_cache, kv_dtype, num_blocks, block_size, block_table,
+                        block_table_stride, seq_lens, batch, num_heads, 1, shard_id, num_shards,
+                        sparse_idx, topk, softmax_scale, out_partial, out_lse, workspace,
+                        workspace_bytes, num_splits, impl, stream);
+}
+
+int mla_decode_partial_multi(const void* q, const void* kv_cache, int kv_dtype,
+                             int64_t num_blocks, int block_size, const int32_t* block_table,
+                             int block_table_stride, const int32_t* seq_lens, int batch,
+                             int num_heads, int q_len, int shard_id, int num_shards,
+                             float softmax_scale, float* out_partial, float* out_lse,
+                             void* workspace, size_t workspace_bytes, int num_splits, int impl,
+                             void* stream) {
+  if (q_len < 1 || num_heads < 1) return DCPMLA_ERR_INVALID_ARGUMENT;
+  if ((long long)num_heads * q_len > kMaxHeads) return DCPMLA_ERR_UNSUPPORTED;
+  return decode_partial(q, kv_cache, kv_dtype, num_blocks, block_size, block_table,
+                        block_table_stride, seq_lens, batch, num_heads * q_len, q_len, shard_id,
+                        num_shards, nullptr, 0, softmax_scale, out_partial, out_lse, workspace,
+                        workspace_bytes, num_splits, impl, stream);
 }
 
 int dcp_merge(const float* partials, const float* lses, int num_shards, int batch,

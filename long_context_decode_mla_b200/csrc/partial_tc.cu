@@ -518,6 +518,7 @@ __device__ __forceinline__ void softmax_role(const PartialParams& p, TcCtl& c, u
   TileCursor cur;
   if (!cur.start(p, c, nseg)) return;
   float m_used = -CUDART_INF_F, l = 0.f;
+  int jmax = 0;                              // multi-query: last local row this row may see
   while (true) {
     const int st = tau & 1;
     const uint32_t ph = (tau >> 1) & 1;
@@ -528,7 +529,17 @@ __device__ __forceinline__ void softmax_role(const PartialParams& p, TcCtl& c, u
     uint32_t sr[32];
     ptx::tmem_ld32(lane_base + kColS + 32 * st, sr);
     ptx::tmem_wait_ld();
-    const uint32_t mw = c.row_mask[st][half];
+    uint32_t mw = c.row_mask[st][half];
+    if (p.q_len > 1) {
+      // Causal rows: row h is query i = h / (heads / q_len) at global position
+      // L_b - q_len + i; it sees local rows j with j * N + shard <= that.
+      if (cur.t == 0) {
+        const int lim = max(__ldg(p.seq_lens + cur.v.b), 0) - p.q_len + h / (p.heads / p.q_len);
+        jmax = lim >= p.shard ? (lim - p.shard) / p.nshards : -1;
+      }
+      const int cmax = jmax - (cur.v.row_begin + cur.t * kTileTok + half * 32);
+      mw &= cmax >= 31 ? 0xffffffffu : (cmax < 0 ? 0u : ((2u << cmax) - 1u));
+    }
     float x[32];
     float mloc = -CUDART_INF_F;
 #pragma unroll

@@ -199,6 +199,38 @@ def mla_decode_partial_noalloc(q, kv_cache, kv_dtype, block_table, seq_lens, sha
     _check(rc, "mla_decode_partial_noalloc")
 
 
+_multi_fn = None
+
+
+def _multi():
+    global _multi_fn
+    if _multi_fn is None:
+        f = lib().mla_decode_partial_multi
+        vp, i32, i64, f32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+        f.argtypes = [vp, vp, i32, i64, i32, vp, i32, vp, i32, i32, i32, i32, i32, f32, vp, vp,
+                      vp, sz, i32, i32, vp]
+        f.restype = i32
+        _multi_fn = f
+    return _multi_fn
+
+
+def mla_decode_partial_multi(q, kv_cache, kv_dtype, block_table, seq_lens, shard_id, num_shards,
+                             softmax_scale, out_partial, out_lse, workspace, num_splits: int = 0,
+                             impl: str | int = "auto", stream=None, block_size: int = BLOCK_SIZE,
+                             num_blocks: int | None = None):
+    """One shard's multi-query partials (see include/dcpmla.h): q [B, q_len, H, 576]."""
+    B, q_len, H = q.shape[0], q.shape[1], q.shape[2]
+    kvd = KV_DTYPES[kv_dtype] if isinstance(kv_dtype, str) else int(kv_dtype)
+    nb = kv_cache.shape[0] if num_blocks is None else num_blocks
+    impl_code = IMPLS[impl] if isinstance(impl, str) else int(impl)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = _multi()(_ptr(q), _ptr(kv_cache), kvd, nb, block_size, _ptr(block_table),
+                  block_table.shape[-1], _ptr(seq_lens), B, H, q_len, shard_id, num_shards,
+                  float(softmax_scale), _ptr(out_partial), _ptr(out_lse), _ptr(workspace),
+                  ws_bytes, num_splits, impl_code, _stream(stream))
+    _check(rc, "mla_decode_partial_multi")
+
+
 def dcp_merge(partials, lses, out, out_lse=None, stream=None):
     """LSE-weighted merge of [N, B, H, 512] partials (see include/dcpmla.h)."""
     N, B, H = partials.shape[0], partials.shape[1], partials.shape[2]
@@ -216,15 +248,16 @@ class DcpDecoder:
     """
 
     def __init__(self, batch, heads, num_shards, topk=0, num_splits=0, device="cuda",
-                 impl="auto", streams=None):
+                 impl="auto", streams=None, q_len=1):
         self.batch, self.heads, self.num_shards = batch, heads, num_shards
-        self.num_splits, self.impl, self.topk = num_splits, impl, topk
+        self.num_splits, self.impl, self.topk, self.q_len = num_splits, impl, topk, q_len
+        rows = heads * q_len                 # multi-query: rows [q_len][heads]
         dev = torch.device(device)
-        self.partials = torch.empty(num_shards, batch, heads, V_DIM, device=dev)
-        self.lses = torch.empty(num_shards, batch, heads, device=dev)
-        self.out = torch.empty(batch, heads, V_DIM, device=dev)
-        self.out_lse = torch.empty(batch, heads, device=dev)
-        nbytes = mla_decode_workspace_size(batch, heads, num_splits, topk)
+        self.partials = torch.empty(num_shards, batch, rows, V_DIM, device=dev)
+        self.lses = torch.empty(num_shards, batch, rows, device=dev)
+        self.out = torch.empty(batch, rows, V_DIM, device=dev)
+        self.out_lse = torch.empty(batch, rows, device=dev)
+        nbytes = mla_decode_workspace_size(batch, rows, num_splits, topk)
         self.workspaces = [torch.zeros(nbytes, dtype=torch.uint8, device=dev)
                            for _ in range(num_shards)]
         self.streams = streams
@@ -247,11 +280,18 @@ class DcpDecoder:
             st = streams[s % len(streams)] if streams else base
             if streams:
                 st.wait_event(ev)
-            mla_decode_partial(prob.q, prob.kv_cache, prob.kv_dtype, prob.block_tables[s],
-                               prob.seq_lens, s, self.num_shards, prob.sparse_idx,
-                               prob.softmax_scale, self.partials[s], self.lses[s],
-                               self.workspaces[s], self.num_splits, self.impl, st,
-                               prob.block_size)
+            if self.q_len > 1:
+                qv = prob.q.view(self.batch, self.q_len, self.heads, HEAD_DIM)
+                mla_decode_partial_multi(qv, prob.kv_cache, prob.kv_dtype, prob.block_tables[s],
+                                         prob.seq_lens, s, self.num_shards, prob.softmax_scale,
+                                         self.partials[s], self.lses[s], self.workspaces[s],
+                                         self.num_splits, self.impl, st, prob.block_size)
+            else:
+                mla_decode_partial(prob.q, prob.kv_cache, prob.kv_dtype, prob.block_tables[s],
+                                   prob.seq_lens, s, self.num_shards, prob.sparse_idx,
+                                   prob.softmax_scale, self.partials[s], self.lses[s],
+                                   self.workspaces[s], self.num_splits, self.impl, st,
+                                   prob.block_size)
         if streams:
             for st in streams:
                 e2 = torch.cuda.Event()

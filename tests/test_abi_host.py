@@ -173,3 +173,23 @@ def test_kv_append_fails_closed_before_any_launch():
     assert call(T=0) == OK                                   # nothing to write
     assert call(lat=None) == EINVAL and call(cache=None) == EINVAL and call(bt=None) == EINVAL
     assert call(lat=A + 8) == EALIGN and call(cache=A + 4) == EALIGN and call(rope=A + 2) == EALIGN
+
+
+def test_multi_query_fails_closed_before_any_launch():
+    L = dcpmla.lib()
+    f = L.mla_decode_partial_multi
+    vp, i32, i64, f32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+    f.argtypes = [vp, vp, i32, i64, i32, vp, i32, vp, i32, i32, i32, i32, i32, f32, vp, vp, vp, sz,
+                  i32, i32, vp]
+    f.restype = i32
+
+    def call(heads=16, q_len=4, batch=2, shard=0, nshards=2, kvd=1, bs=64, impl=0, q=FAKE):
+        return f(q, FAKE, kvd, 16, bs, FAKE, 4, FAKE, batch, heads, q_len, shard, nshards, 0.07,
+                 FAKE, FAKE, FAKE, 0, 4, impl, None)
+
+    assert call(q_len=0) == EINVAL and call(heads=0) == EINVAL
+    assert call(heads=16, q_len=5) == EUNSUP                 # 80 rows > 64
+    assert call(heads=64, q_len=2) == EUNSUP
+    assert call(shard=2) == EINVAL and call(kvd=3) == EINVAL and call(bs=16) == EUNSUP
+    assert call(q=FAKE + 2) == EALIGN
+    assert call(batch=0) == OK                               # nothing to do
