@@ -345,6 +345,8 @@ def run_ours(args, rank, world, local):
     extras = {}
     if args.workload == "agentic" and not args.no_extras:
         extras["at_64k"] = time_other_workload("agentic64k", dev, rank, world, args, streams_for=N)
+    if prob.sparse_idx is None and prob.heads % 4 == 0:
+        extras["multi_query"] = time_multi_query(prob, dev, args, q_len=4)
     extras["kv_append"] = time_append(prob, dev, max(20, args.steps // 4))
     if result is not None:
         result.update(extras)
@@ -385,6 +387,36 @@ def time_other_workload(name, dev, rank, world, args, streams_for):
     return {"workload": desc, "steps_per_s": round(world * 1e3 / ms, 2),
             "ms_per_step": round(ms, 4), "value": round(world * kvb / (ms * 1e-3) / 1e9, 1),
             "unit": UNIT, "steps": steps}
+
+
+def time_multi_query(prob, dev, args, q_len):
+    """The same cache and rows as the headline step, read as heads / q_len
+    heads x q_len query tokens with causal limits (speculative verification):
+    KV bytes per step are unchanged, query tokens per step are q_len x."""
+    import torch
+    from long_context_decode_mla_b200 import dcpmla
+    B, N, H = prob.batch, prob.num_shards, prob.heads // q_len
+    streams = [torch.cuda.Stream(device=dev) for _ in range(N)]
+    dec = dcpmla.DcpDecoder(B, H, N, device=dev, impl=args.kernel, streams=streams, q_len=q_len)
+    graph = dec.capture(prob)
+    for _ in range(3):
+        graph.replay()
+    torch.cuda.synchronize(dev)
+    steps = max(20, args.steps // 4)
+    stream = torch.cuda.current_stream(dev)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(steps):
+        graph.replay()
+    t1.record(stream)
+    t1.synchronize()
+    assert dec.flags() == 0, "device flags set"
+    ms = t0.elapsed_time(t1) / steps
+    kvb = kv_bytes(prob)
+    del graph, dec
+    return {"heads": H, "q_len": q_len, "ms_per_step": round(ms, 4),
+            "value": round(kvb / (ms * 1e-3) / 1e9, 1), "unit": UNIT,
+            "query_tokens_per_s": round(B * q_len * 1e3 / ms, 1)}
 
 
 def time_append(prob, dev, steps):
