@@ -244,7 +244,9 @@ class DcpDecoder:
 
     Holds the outputs ([N, B, H, 512] partials, [N, B, H] LSEs, merged
     [B, H, 512] and [B, H]) and one workspace per shard, so shards issued on
-    different streams never share scratch memory.
+    different streams never share scratch memory.  With ``q_len`` > 1 the
+    step is multi-query decode: ``prob.q`` holds [B, q_len * H, 576] rows
+    ordered [q_len][H], and the outputs have q_len * H rows in that order.
     """
 
     def __init__(self, batch, heads, num_shards, topk=0, num_splits=0, device="cuda",
