@@ -65,6 +65,12 @@ extern "C" {
 #define DCPMLA_IMPL_AUTO 0   /* fastest available for the arguments */
 #define DCPMLA_IMPL_SIMT 1   /* plain CUDA-core kernel (any H <= 64) */
 #define DCPMLA_IMPL_TC 2     /* tcgen05 / TMEM tensor-core kernel */
+/* Test only, OR-ed into DCPMLA_IMPL_TC: the converter warps withhold their
+ * first arrival, so every pipeline wait of every CTA runs out (about 2 s);
+ * the kernel then drains, frees its tensor memory, sets
+ * DCPMLA_FLAG_TIMEOUT and returns with invalid outputs.  Exercises the
+ * timeout path; the context stays usable. */
+#define DCPMLA_TEST_WITHHOLD_ARRIVAL 0x100
 
 /* Return codes. */
 #define DCPMLA_OK 0

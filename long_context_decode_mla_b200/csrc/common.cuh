@@ -47,6 +47,7 @@ struct PartialParams {
   float* ws_lse;              // [slots][H]
   int* ws_list;               // sparse mode: per-CTA lists of selected local rows
   int num_ctas;               // G: CTAs sharing the dense tile space
+  int test_withhold;          // test only: converters skip their first arrival (timeout path)
 };
 
 // Number of tokens t in [0, L) with t mod N == s (round-robin ownership).

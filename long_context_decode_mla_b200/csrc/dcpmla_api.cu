@@ -112,6 +112,9 @@ int decode_partial(const void* q, const void* kv_cache, int kv_dtype, int64_t nu
                    float* out_partial, float* out_lse, void* workspace, size_t workspace_bytes,
                    int num_splits, int impl, void* stream) {
   // ---- scalar checks (fail closed, nothing launched on error) ----
+  const bool withhold = (impl & DCPMLA_TEST_WITHHOLD_ARRIVAL) != 0;
+  impl &= ~DCPMLA_TEST_WITHHOLD_ARRIVAL;
+  if (withhold && impl != DCPMLA_IMPL_TC) return DCPMLA_ERR_INVALID_ARGUMENT;
   if (batch < 0 || num_heads < 1 || num_shards < 1 || shard_id < 0 || shard_id >= num_shards ||
       block_size < 1 || block_table_stride < 1 || num_blocks < 1 || num_splits < 0 ||
       topk < 0 || (sparse_idx && topk < 1) || !std::isfinite(softmax_scale))
@@ -159,6 +162,7 @@ int decode_partial(const void* q, const void* kv_cache, int kv_dtype, int64_t nu
   p.ws_lse = reinterpret_cast<float*>(ws + ws_lse_offset(slots, num_heads));
   p.ws_list = list_ints ? reinterpret_cast<int*>(ws + ws_list_offset(slots, num_heads)) : nullptr;
   p.num_ctas = ctas;
+  p.test_withhold = withhold ? 1 : 0;
 
   const bool tc_ok = tc_supports(p, kv_dtype);
   if (impl == DCPMLA_IMPL_TC && !tc_ok) return DCPMLA_ERR_UNSUPPORTED;

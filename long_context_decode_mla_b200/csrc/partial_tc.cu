@@ -830,17 +830,20 @@ __device__ __forceinline__ void convert_role(const PartialParams& p, TcCtl& c, u
     // chunks 0..3 (scale groups 0, 1) are free once the first PV half of the
     // tile two back is done, chunks 4..7 and the rope slot after the second
     if (reuse && !wait_or_abort(&c.empty[st][0], eph, c)) break;
+    // test only: withholding the very first arrival makes every pipeline wait
+    // of the CTA run out, which exercises the timeout path
+    const bool withhold = p.test_withhold && tau == 0;
     if constexpr (KV == kKvFp8) {
       stage_store_group<0>(stage, ct, stg, range_bad);
       ptx::fence_proxy_async();
-      ptx::mbar_arrive(&c.full[st][0]);
+      if (!withhold) ptx::mbar_arrive(&c.full[st][0]);
       stage_store_group<1>(stage, ct, stg, range_bad);
       ptx::fence_proxy_async();
       ptx::mbar_arrive(&c.full[st][1]);
     } else {
       stage_store_half0(stage, ct, stg, range_bad);
       ptx::fence_proxy_async();
-      ptx::mbar_arrive(&c.full[st][0]);
+      if (!withhold) ptx::mbar_arrive(&c.full[st][0]);
       ptx::mbar_arrive(&c.full[st][1]);
       stage_load_half1(p, cur.v, list, cur.t, ct, stg);
     }

@@ -1,0 +1,66 @@
+"""The bounded-wait (timeout) path of the tensor-core kernel, on the GPU.
+
+With DCPMLA_TEST_WITHHOLD_ARRIVAL the converter warps withhold their first
+arrival, so nothing ever completes the first stage: every waiting role of
+every CTA gives up after its clock budget (about 2 s), the CTA drains, frees
+its tensor memory and sets DCPMLA_FLAG_TIMEOUT.  No trap, fault or unbounded
+wait is involved, and the context must stay usable: a normal call right after
+must succeed and match the oracle.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from long_context_decode_mla_b200 import dcpmla
+from long_context_decode_mla_b200 import workload as wl
+
+pytestmark = pytest.mark.gpu
+
+WITHHOLD = 0x100          # DCPMLA_TEST_WITHHOLD_ARRIVAL
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    dcpmla.lib()
+    torch.cuda.set_device(0)
+
+
+def test_withheld_arrival_times_out_and_the_context_survives():
+    prob = wl.make_problem("tiny", num_shards=2).to("cuda")        # 8 tiles per shard
+    B, H = prob.batch, prob.heads
+    o = torch.empty(B, H, 512, device="cuda")
+    l = torch.empty(B, H, device="cuda")
+    ws = torch.zeros(dcpmla.mla_decode_workspace_size(B, H, 8), dtype=torch.uint8, device="cuda")
+    # one tile per CTA: only the MMA and softmax waits run out, once each
+    dcpmla.mla_decode_partial(prob.q, prob.kv_cache, "bf16", prob.block_tables[0], prob.seq_lens,
+                              0, 2, None, prob.softmax_scale, o, l, ws, 8,
+                              dcpmla.IMPLS["tc"] | WITHHOLD)
+    torch.cuda.synchronize()
+    flags = int(ws[:4].view(torch.int32).item())
+    assert flags & dcpmla.FLAG_TIMEOUT
+
+    # the context is intact: a normal step gives the oracle's result
+    dec = dcpmla.DcpDecoder(B, H, 2, impl="tc")
+    dec.step(prob)
+    torch.cuda.synchronize()
+    assert dec.flags() == 0
+    ni = wl.make_problem("tiny", num_shards=2).numpy_inputs()
+    _, _, ref, ref_lse = oracle.dcp_decode(ni["q"], ni["kv_cache"], "bf16", ni["block_tables"],
+                                           ni["seq_lens"], 2, ni["softmax_scale"])
+    out = dec.out.double().cpu().numpy()
+    assert np.abs(out - ref).max() <= 2e-3 * np.abs(ref).max()
+
+
+def test_withhold_needs_the_tensor_core_kernel():
+    prob = wl.make_problem("tiny", num_shards=2).to("cuda")
+    o = torch.empty(1, 8, 512, device="cuda")
+    l = torch.empty(1, 8, device="cuda")
+    ws = torch.zeros(dcpmla.mla_decode_workspace_size(1, 8, 8), dtype=torch.uint8, device="cuda")
+    for impl in (dcpmla.IMPLS["simt"] | WITHHOLD, dcpmla.IMPLS["auto"] | WITHHOLD):
+        with pytest.raises(dcpmla.DcpMlaError) as e:
+            dcpmla.mla_decode_partial(prob.q, prob.kv_cache, "bf16", prob.block_tables[0],
+                                      prob.seq_lens, 0, 2, None, prob.softmax_scale, o, l, ws, 8,
+                                      impl)
+        assert e.value.code == -1
