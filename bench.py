@@ -114,12 +114,25 @@ def measured_peaks():
 PARTIAL_KERNEL_SOURCES = ("common.cuh", "kernels.h", "merge.cu", "partial_tc.cu", "tc_ptx.cuh")
 
 
-def kernel_source_hash() -> str:
+def _code_only(text: str) -> str:
+    """C/C++ source without comments and with whitespace collapsed, so that
+    edits to comments do not count as kernel changes."""
+    import re
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
+
+
+def kernel_source_hash(read=None) -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "long_context_decode_mla_b200", "csrc")
     for name in PARTIAL_KERNEL_SOURCES:
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(name.encode() + f.read())
+        if read is None:
+            with open(os.path.join(csrc, name), encoding="utf-8") as f:
+                text = f.read()
+        else:
+            text = read(name)
+        h.update(name.encode() + _code_only(text).encode())
     return h.hexdigest()[:16]
 
 

@@ -21,7 +21,9 @@
 //    consecutive tiles, swizzled for the tensor core.  Eight converter warps
 //    load each tile's rows into registers one tile ahead, decode them (bf16
 //    or e4m3 * scale -> fp16) and store them once a stage is free; raw cache
-//    bytes never occupy shared memory.
+//    bytes never occupy shared memory.  A stage is published in five parts
+//    (the four 128-value scale groups, then the rope), and the scores of each
+//    part are issued as soon as it lands.
 //  * S = Q K^T: 36 weight-stationary MMAs (M = 64 heads, N = 64 tokens,
 //    K = 16) into one of two TMEM score buffers; the 2x2 data path puts head
 //    h at TMEM lane h for tokens 0..31 and lane 64 + h for tokens 32..63.
@@ -30,9 +32,13 @@
 //    with a lazily updated running max (the output is only rescaled, warp by
 //    warp, when the max grows by more than 2^8), write P into the stage's
 //    rope slot, which the scores no longer need, and keep the running sum.
+//    With several query tokens per request (rows = q_len x heads) each row
+//    also masks the tokens beyond its query's causal limit.
 //  * O += P V: 8 MMAs (M = 64, N = 256 dims, K = 16 tokens) reading V from the
 //    same chunk slots as an MN-major operand; O (64 x 512 fp32) stays in TMEM
 //    for the whole request and is normalised in the epilogue.
+//  * The kernel is instantiated per row format and per dense / sparse mode,
+//    so the dense kernels carry no sparse addressing code.
 #include <cuda_fp8.h>
 #include <math_constants.h>
 
