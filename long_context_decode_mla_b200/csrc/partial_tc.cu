@@ -813,6 +813,18 @@ __device__ __forceinline__ void convert_role(const PartialParams& p, TcCtl& c, u
   Stage<KV> stg;
   TileCursor cur, pf;
   if (!cur.start(p, c, nseg)) return;
+  // The first tile's rows and, at the very start, the first request's Q are
+  // requested before the L2 prefetch burst of the next tiles: at kernel start
+  // every CTA prefetches at once, and loads issued after that burst would
+  // queue behind it.
+  stage_load(p, cur.v, list, cur.t, ct, stg);
+  bool q_loaded = false;
+  if (sigma == 0) {                          // no earlier request's Q to wait for
+    load_q(p, cur.v.b, sq, ct, range_bad);
+    ptx::fence_proxy_async();
+    ptx::mbar_arrive(&c.q_full);
+    q_loaded = true;
+  }
   // L2 prefetch runs kPrefetchTiles ahead of the tile being staged
   pf = cur;
   bool pf_ok = true;
@@ -820,19 +832,19 @@ __device__ __forceinline__ void convert_role(const PartialParams& p, TcCtl& c, u
     prefetch_tile<KV>(p, pf.v, list, pf.t, ct);
     pf_ok = pf.next(p, c);
   }
-  stage_load(p, cur.v, list, cur.t, ct, stg);
   while (true) {
     const int st = tau & 1;
     uint8_t* stage = slot_ptr(sslot, st, 0);
     const bool reuse = tau >= 2;                           // stage used before: wait for its PV
     const uint32_t eph = ((tau >> 1) + 1) & 1;             // phase of the PV two tiles back
-    if (cur.t == 0) {
+    if (cur.t == 0 && !q_loaded) {
       // new request: its Q replaces the previous one once that one's last QK is done
       if (sigma > 0 && !wait_or_abort(&c.q_empty, (sigma - 1) & 1, c)) break;
       load_q(p, cur.v.b, sq, ct, range_bad);
       ptx::fence_proxy_async();
       ptx::mbar_arrive(&c.q_full);
     }
+    q_loaded = false;
     // chunks 0..3 (scale groups 0, 1) are free once the first PV half of the
     // tile two back is done, chunks 4..7 and the rope slot after the second
     if (reuse && !wait_or_abort(&c.empty[st][0], eph, c)) break;
