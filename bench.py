@@ -109,9 +109,10 @@ def measured_peaks():
     return 6650.0, "fallback"
 
 
-# the sources the partial kernel (whose DRAM traffic profiles/traffic.json
-# records) is built from; other entry points do not invalidate the figure
-PARTIAL_KERNEL_SOURCES = ("common.cuh", "kernels.h", "merge.cu", "partial_tc.cu", "tc_ptx.cuh")
+# the translation unit of the partial kernel (whose DRAM traffic
+# profiles/traffic.json records) and the headers it includes; other files are
+# compiled separately and cannot change that kernel
+PARTIAL_KERNEL_SOURCES = ("common.cuh", "kernels.h", "partial_tc.cu", "tc_ptx.cuh")
 
 
 def _code_only(text: str) -> str:
