@@ -239,6 +239,51 @@ def dcp_merge(partials, lses, out, out_lse=None, stream=None):
     _check(rc, "dcp_merge")
 
 
+def check_inputs(block_tables, seq_lens, num_blocks: int, num_shards: int,
+                 sparse_idx=None, block_size: int = BLOCK_SIZE) -> None:
+    """Debug-mode validation of device contents on the host side.
+
+    The kernels never read outside the cache: an out-of-range table entry or
+    length is skipped and reported through a flag bit.  This check finds such
+    inputs before a call, with a precise message: block tables [N, B, stride]
+    must map every block a shard's local rows use into [0, num_blocks);
+    lengths must be >= 0 and fit the table rows; sparse indices must be -1
+    (padding) or inside [0, L_b).  Raises ValueError on the first problem.
+    """
+    import torch
+    bt = torch.as_tensor(block_tables)
+    lens = torch.as_tensor(seq_lens).to(torch.int64)
+    if bt.dim() != 3 or bt.shape[0] != num_shards:
+        raise ValueError(f"block_tables must be [num_shards, batch, stride], got {tuple(bt.shape)}")
+    N, B, stride = bt.shape
+    if lens.shape != (B,):
+        raise ValueError(f"seq_lens must be [{B}], got {tuple(lens.shape)}")
+    if bool((lens < 0).any()):
+        b = int(torch.nonzero(lens < 0)[0, 0])
+        raise ValueError(f"seq_lens[{b}] = {int(lens[b])} is negative")
+    for s in range(N):
+        local = torch.where(lens > s, (lens - s - 1) // N + 1, torch.zeros_like(lens))
+        need = (local + block_size - 1) // block_size
+        if bool((need > stride).any()):
+            b = int(torch.nonzero(need > stride)[0, 0])
+            raise ValueError(f"shard {s}, request {b}: {int(local[b])} local rows need "
+                             f"{int(need[b])} blocks, the table row has {stride}")
+        used = torch.arange(stride, device=bt.device)[None, :] < need.to(bt.device)[:, None]
+        bad = used & ((bt[s] < 0) | (bt[s] >= num_blocks))
+        if bool(bad.any()):
+            b, k = (int(v) for v in torch.nonzero(bad)[0])
+            raise ValueError(f"shard {s}, request {b}: block_tables[{s}][{b}][{k}] = "
+                             f"{int(bt[s, b, k])} is outside [0, {num_blocks})")
+    if sparse_idx is not None:
+        idx = torch.as_tensor(sparse_idx).to(torch.int64)
+        lim = lens.to(idx.device)[:, None]
+        bad = (idx != -1) & ((idx < 0) | (idx >= lim))
+        if bool(bad.any()):
+            b, i = (int(v) for v in torch.nonzero(bad)[0])
+            raise ValueError(f"sparse_idx[{b}][{i}] = {int(idx[b, i])} is neither -1 nor in "
+                             f"[0, {int(lens[b])})")
+
+
 class DcpDecoder:
     """Buffers and calls for whole emulated DCP decode steps on one GPU.
 
