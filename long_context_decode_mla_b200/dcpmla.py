@@ -53,6 +53,15 @@ def lib() -> ctypes.CDLL:
     L.dcpmla_error_string.restype = ctypes.c_char_p
     L.dcpmla_device_sm_count.argtypes = [ctypes.POINTER(i32)]
     L.dcpmla_device_sm_count.restype = i32
+    L.mla_decode_partial_multi.argtypes = [vp, vp, i32, i64, i32, vp, i32, vp, i32, i32, i32, i32,
+                                           i32, f32, vp, vp, vp, sz, i32, i32, vp]
+    L.mla_decode_partial_multi.restype = i32
+    L.mla_decode_partial_noalloc.argtypes = [vp, vp, i32, i64, i32, vp, i32, vp, i32, i32, i32,
+                                             i32, vp, i32, f32, vp, vp, vp, i32, i32, vp]
+    L.mla_decode_partial_noalloc.restype = i32
+    L.mla_kv_append.argtypes = [vp, vp, i32, vp, vp, vp, i32, i32, i32, i32, vp, i32, i64, i32,
+                                vp, vp]
+    L.mla_kv_append.restype = i32
     _lib = L
     return L
 
@@ -125,20 +134,6 @@ def mla_decode_partial(q, kv_cache, kv_dtype, block_table, seq_lens, shard_id, n
     _check(rc, "mla_decode_partial")
 
 
-_append_fn = None
-
-
-def _append():
-    global _append_fn
-    if _append_fn is None:
-        f = lib().mla_kv_append
-        vp, i32, i64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
-        f.argtypes = [vp, vp, i32, vp, vp, vp, i32, i32, i32, i32, vp, i32, i64, i32, vp, vp]
-        f.restype = i32
-        _append_fn = f
-    return _append_fn
-
-
 def mla_kv_append(latent, rope, positions, req_idx, block_table, shard_id, num_shards, kv_cache,
                   kv_dtype, flags=None, stream=None, block_size: int = BLOCK_SIZE,
                   num_blocks: int | None = None):
@@ -151,26 +146,14 @@ def mla_kv_append(latent, rope, positions, req_idx, block_table, shard_id, num_s
     T = latent.shape[0]
     kvd = KV_DTYPES[kv_dtype] if isinstance(kv_dtype, str) else int(kv_dtype)
     nb = kv_cache.shape[0] if num_blocks is None else num_blocks
-    rc = _append()(_ptr(latent), _ptr(rope), T, _ptr(positions), _ptr(req_idx), _ptr(block_table),
-                   block_table.shape[-1], block_table.shape[0], shard_id, num_shards,
-                   _ptr(kv_cache), kvd, nb, block_size, _ptr(flags), _stream(stream))
+    rc = lib().mla_kv_append(
+        _ptr(latent), _ptr(rope), T, _ptr(positions), _ptr(req_idx), _ptr(block_table),
+        block_table.shape[-1], block_table.shape[0], shard_id, num_shards, _ptr(kv_cache), kvd, nb,
+        block_size, _ptr(flags), _stream(stream))
     _check(rc, "mla_kv_append")
 
 
 NOALLOC_SCRATCH_BYTES = 32 << 20          # DCPMLA_NOALLOC_SCRATCH_BYTES
-_noalloc_fn = None
-
-
-def _noalloc():
-    global _noalloc_fn
-    if _noalloc_fn is None:
-        f = lib().mla_decode_partial_noalloc
-        vp, i32, i64, f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float
-        f.argtypes = [vp, vp, i32, i64, i32, vp, i32, vp, i32, i32, i32, i32, vp, i32, f32,
-                      vp, vp, vp, i32, i32, vp]
-        f.restype = i32
-        _noalloc_fn = f
-    return _noalloc_fn
 
 
 def mla_decode_partial_noalloc(q, kv_cache, kv_dtype, block_table, seq_lens, shard_id,
@@ -191,27 +174,12 @@ def mla_decode_partial_noalloc(q, kv_cache, kv_dtype, block_table, seq_lens, sha
     nb = kv_cache.shape[0] if num_blocks is None else num_blocks
     topk = 0 if sparse_idx is None else sparse_idx.shape[1]
     impl_code = IMPLS[impl] if isinstance(impl, str) else int(impl)
-    rc = _noalloc()(
+    rc = lib().mla_decode_partial_noalloc(
         _ptr(q), _ptr(kv_cache), kvd, nb, block_size, _ptr(block_table), block_table.shape[-1],
         _ptr(seq_lens), B, H, shard_id, num_shards, _ptr(sparse_idx), topk,
         float(softmax_scale), _ptr(out_partial), _ptr(out_lse), _ptr(out_flags),
         num_splits, impl_code, _stream(stream))
     _check(rc, "mla_decode_partial_noalloc")
-
-
-_multi_fn = None
-
-
-def _multi():
-    global _multi_fn
-    if _multi_fn is None:
-        f = lib().mla_decode_partial_multi
-        vp, i32, i64, f32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
-        f.argtypes = [vp, vp, i32, i64, i32, vp, i32, vp, i32, i32, i32, i32, i32, f32, vp, vp,
-                      vp, sz, i32, i32, vp]
-        f.restype = i32
-        _multi_fn = f
-    return _multi_fn
 
 
 def mla_decode_partial_multi(q, kv_cache, kv_dtype, block_table, seq_lens, shard_id, num_shards,
@@ -224,10 +192,10 @@ def mla_decode_partial_multi(q, kv_cache, kv_dtype, block_table, seq_lens, shard
     nb = kv_cache.shape[0] if num_blocks is None else num_blocks
     impl_code = IMPLS[impl] if isinstance(impl, str) else int(impl)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    rc = _multi()(_ptr(q), _ptr(kv_cache), kvd, nb, block_size, _ptr(block_table),
-                  block_table.shape[-1], _ptr(seq_lens), B, H, q_len, shard_id, num_shards,
-                  float(softmax_scale), _ptr(out_partial), _ptr(out_lse), _ptr(workspace),
-                  ws_bytes, num_splits, impl_code, _stream(stream))
+    rc = lib().mla_decode_partial_multi(
+        _ptr(q), _ptr(kv_cache), kvd, nb, block_size, _ptr(block_table), block_table.shape[-1],
+        _ptr(seq_lens), B, H, q_len, shard_id, num_shards, float(softmax_scale), _ptr(out_partial),
+        _ptr(out_lse), _ptr(workspace), ws_bytes, num_splits, impl_code, _stream(stream))
     _check(rc, "mla_decode_partial_multi")
 
 
