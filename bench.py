@@ -360,6 +360,8 @@ def run_ours(args, rank, world, local):
     if prob.sparse_idx is None and prob.heads % 4 == 0:
         extras["multi_query"] = time_multi_query(prob, dev, args, q_len=4)
     extras["kv_append"] = time_append(prob, dev, max(20, args.steps // 4))
+    if H % N == 0:
+        extras["merge_heads"] = time_merge_heads(dec, dev, max(20, args.steps // 4))
     if result is not None:
         result.update(extras)
     if world > 1:
@@ -456,6 +458,64 @@ def time_multi_query(prob, dev, args, q_len):
     return {"heads": H, "q_len": q_len, "ms_per_step": round(ms, 4),
             "value": round(kvb / (ms * 1e-3) / 1e9, 1), "unit": UNIT,
             "query_tokens_per_s": round(B * q_len * 1e3 / ms, 1)}
+
+
+def time_merge_heads(dec, dev, steps):
+    """The cross-rank exchange of real multi-GPU DCP, emulated on one GPU: the
+    step's N shard partials sit in N exchange buffers (one per rank), and each
+    of the N ranks' dcp_merge_heads launches merges its H/N heads from all N
+    buffers (graph-replayed, back to back on one stream).  On N GPUs each
+    launch reads (N - 1) / N of its bytes over NVLink; here all are local."""
+    import torch
+    from long_context_decode_mla_b200 import dcp_group, dcpmla
+    N, B, H = dec.partials.shape[0], dec.partials.shape[1], dec.partials.shape[2]
+    lse_off, slot = dcp_group.slot_layout(B, H)
+    bufs = [dcpmla.dcp_exchange_alloc(slot)[0] for _ in range(N)]
+    try:
+        for s, a in enumerate(bufs):
+            dcp_group.device_view(a, (B, H, 512)).copy_(dec.partials[s])
+            dcp_group.device_view(a + lse_off, (B, H)).copy_(dec.lses[s])
+        lse_ptrs = [a + lse_off for a in bufs]
+        slices = [dcp_group.head_slice(r, N, H) for r in range(N)]
+        outs = [(torch.empty(B, hn, 512, device=dev), torch.empty(B, hn, device=dev))
+                for _, hn in slices]
+
+        def step(stream):
+            for (h0, hn), (o, l) in zip(slices, outs):
+                dcpmla.dcp_merge_heads(bufs, lse_ptrs, B, H, h0, hn, o, l, stream)
+
+        side = torch.cuda.Stream(device=dev)
+        side.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(side):
+            step(side)
+        torch.cuda.current_stream(dev).wait_stream(side)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=side):
+            step(side)
+        for _ in range(3):
+            graph.replay()
+        torch.cuda.synchronize(dev)
+        merged = torch.cat([o for o, _ in outs], dim=1)
+        assert torch.equal(merged, dec.out), "head-sliced merge differs from dcp_merge"
+        stream = torch.cuda.current_stream(dev)
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(steps):
+            graph.replay()
+        t1.record(stream)
+        t1.synchronize()
+        us = t0.elapsed_time(t1) * 1e3 / steps / N
+        del graph
+    finally:
+        torch.cuda.synchronize(dev)
+        for a in bufs:
+            dcpmla.dcp_exchange_free(a)
+    per_rank = B * H * 513 * 4                  # its H/N heads from all N shards
+    nvlink_gbs = 770.0                          # measured peer copy, GB/s per direction
+    return {"ranks": N, "us_per_rank": round(us, 2), "bytes_per_rank": per_rank,
+            "GBps_local": round(per_rank / (us * 1e-6) / 1e9, 1),
+            "nvlink_bound_us_per_rank": round((N - 1) / N * per_rank / (nvlink_gbs * 1e9) * 1e6,
+                                              2)}
 
 
 def time_append(prob, dev, steps):

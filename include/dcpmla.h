@@ -238,6 +238,76 @@ int dcp_merge(const float* partials, const float* lses, int num_shards, int batc
               int num_heads, float* out, float* out_lse, void* stream);
 
 /*
+ * Real multi-GPU DCP: one rank per GPU, rank r holding shard r of the cache.
+ *
+ * "GLM-5.2 vLLM Decode Context Parallelism", section "Keep the current-main
+ * correctness blocker visible": pure DCP gathers the query heads before
+ * attention and combines the partial output/LSE across ranks after it; section
+ * "Separate the backend merge from stable": the cross-rank combine takes the
+ * ag_rs path (all-gather of LSEs, reduce-scatter of the rescaled partials),
+ * after which each rank holds the merged result of its own query heads
+ * (section "Calculate the GLM-5.2 head envelope": gathered heads = local
+ * heads x DCP size).
+ *
+ * dcp_merge_heads is that exchange as one kernel: this rank reads its slice
+ * of heads from every shard's partial and LSE buffers (its own, and the other
+ * ranks' mapped into this device with dcp_exchange_open) and merges them with
+ * the dcp_merge formula.  The caller orders it after every shard's partial is
+ * complete (e.g. a stream-ordered NCCL collective between the partial and
+ * this call on every rank) and does not overwrite a buffer before every rank
+ * has read it.
+ *
+ *   partials     HOST array of num_shards DEVICE pointers; partials[s] is
+ *                shard s's [batch][num_heads][512] fp32 partial (16-byte
+ *                aligned), readable from the current device.
+ *   lses         HOST array of num_shards DEVICE pointers to [batch][num_heads]
+ *                fp32 LSEs.  Both tables are copied into the launch: the
+ *                host arrays may be reused as soon as the call returns.
+ *   num_shards   1 .. DCPMLA_MAX_MERGE_SHARDS.
+ *   head_begin, head_count: the merged slice, 0 <= head_begin,
+ *                1 <= head_count, head_begin + head_count <= num_heads.
+ *   out          [batch][head_count][512] fp32 (16-byte aligned): row
+ *                (b, i) is the merge of head head_begin + i of request b.
+ *   out_lse      [batch][head_count] fp32 merged LSE, or NULL.
+ *
+ * With head_begin = 0, head_count = num_heads and the shards' buffers laid
+ * out back to back this is exactly dcp_merge (same arithmetic, same order).
+ * Returns DCPMLA_OK or a negative code.
+ */
+#define DCPMLA_MAX_MERGE_SHARDS 64
+int dcp_merge_heads(const float* const* partials, const float* const* lses, int num_shards,
+                    int batch, int num_heads, int head_begin, int head_count, float* out,
+                    float* out_lse, void* stream);
+
+/*
+ * Exchange buffers: device memory another process (rank) can map.  The
+ * method's description has no counterpart to these calls; they are the
+ * plumbing dcp_merge_heads reads peers' partials through (CUDA IPC over
+ * NVLink / NVSwitch).  Unlike the compute calls they allocate, free and
+ * may synchronise the device.
+ *
+ *   dcp_exchange_alloc  allocates `bytes` on the current device; *dev_ptr
+ *                       receives the pointer (256-byte aligned) and
+ *                       ipc_handle (DCPMLA_IPC_HANDLE_BYTES bytes, caller
+ *                       owned) a handle other processes on this node pass to
+ *                       dcp_exchange_open.  Release with dcp_exchange_free
+ *                       after every mapping of it is closed.
+ *   dcp_exchange_open   maps another process's buffer into the current
+ *                       device (peer access enabled as needed); *dev_ptr
+ *                       receives its base.  A process cannot open its own
+ *                       handle: use its own pointer.  Close with
+ *                       dcp_exchange_close.
+ * Each returns DCPMLA_OK, DCPMLA_ERR_INVALID_ARGUMENT for a null pointer or a
+ * zero size, or DCPMLA_ERR_CUDA if the runtime refuses (out of memory, an
+ * invalid or own handle); *dev_ptr is NULL on failure.
+ */
+#define DCPMLA_IPC_HANDLE_BYTES 64
+int dcp_exchange_alloc(size_t bytes, void** dev_ptr, void* ipc_handle);
+int dcp_exchange_open(const void* ipc_handle, void** dev_ptr);
+int dcp_exchange_close(void* dev_ptr);
+int dcp_exchange_free(void* dev_ptr);
+
+/*
  * DCP cache write of new decode tokens: this shard writes the tokens it owns.
  *
  * "GLM-5.2 vLLM Decode Context Parallelism", section "Keep the current-main

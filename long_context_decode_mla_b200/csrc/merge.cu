@@ -1,68 +1,14 @@
 // LSE-weighted merges: the cross-shard DCP merge and the combine of split-KV
-// pieces inside one shard (the same formula applied one level down).
-//
-// With M = max_i LSE_i and w_i = exp(LSE_i - M):
-//   O = sum_i w_i O_i / sum_i w_i,   LSE = M + ln sum_i w_i,
-// and pieces with LSE = -inf weigh exactly zero; if all are -inf the result
-// is (0, -inf).  "GLM-5.2 vLLM Decode Context Parallelism", sections "See why
-// vLLM 0.26.0 fails" (partials combined with the softmax normalisation via
-// LSE) and "Separate the backend merge from stable" (the neutral (0, -inf)
-// pair of an empty shard drops out of the merge).
+// pieces inside one shard (the formula of merge_rows.cuh applied one level
+// down).
 #include "common.cuh"
 #include "kernels.h"
+#include "merge_rows.cuh"
 
 #include <math_constants.h>
 
 namespace dcpmla {
 namespace {
-
-// One warp merges `count` pieces of one (request, head) row.  Piece k has its
-// 512 outputs at o + (first + k * stride) * 512 and its LSE at
-// lse[first + k * stride].
-__device__ __forceinline__ void merge_warp(const float* __restrict__ o,
-                                           const float* __restrict__ lse, size_t first,
-                                           size_t stride, int count, float* __restrict__ out_o,
-                                           float* __restrict__ out_lse) {
-  const int lane = threadIdx.x & 31;
-  float M = -CUDART_INF_F;
-  for (int k = lane; k < count; k += 32) M = fmaxf(M, __ldg(lse + first + k * stride));
-#pragma unroll
-  for (int s = 16; s > 0; s >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, s));
-  float4 acc[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (M == -CUDART_INF_F) {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) reinterpret_cast<float4*>(out_o)[i * 32 + lane] = acc[i];
-    if (lane == 0 && out_lse) *out_lse = -CUDART_INF_F;
-    return;
-  }
-  float wsum = 0.f;
-  for (int k = 0; k < count; ++k) {
-    const size_t r = first + k * stride;
-    const float lk = __ldg(lse + r);
-    if (lk == -CUDART_INF_F) continue;
-    const float w = expf(lk - M);
-    wsum += w;
-    const float4* src = reinterpret_cast<const float4*>(o + r * kVDim);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float4 v = __ldg(src + i * 32 + lane);
-      acc[i].x = fmaf(w, v.x, acc[i].x);
-      acc[i].y = fmaf(w, v.y, acc[i].y);
-      acc[i].z = fmaf(w, v.z, acc[i].z);
-      acc[i].w = fmaf(w, v.w, acc[i].w);
-    }
-  }
-  const float inv = 1.f / wsum;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    float4 v = acc[i];
-    v.x *= inv; v.y *= inv; v.z *= inv; v.w *= inv;
-    reinterpret_cast<float4*>(out_o)[i * 32 + lane] = v;
-  }
-  if (lane == 0 && out_lse) *out_lse = M + logf(wsum);
-}
 
 constexpr int kMergeWarps = 8;
 
@@ -71,8 +17,8 @@ __global__ void __launch_bounds__(kMergeWarps * 32) dcp_merge_kernel(
     float* __restrict__ out, float* __restrict__ out_lse) {
   const int row = blockIdx.x * kMergeWarps + (threadIdx.x >> 5);
   if (row >= rows) return;
-  merge_warp(partials, lses, row, rows, nshards, out + (size_t)row * kVDim,
-             out_lse ? out_lse + row : nullptr);
+  merge_warp(StridedPieces{partials, lses, (size_t)row, (size_t)rows}, nshards,
+             out + (size_t)row * kVDim, out_lse ? out_lse + row : nullptr);
 }
 
 // Combine of the split pieces of each request.  Grid: one CTA per
@@ -120,8 +66,9 @@ __global__ void __launch_bounds__(256) split_combine_kernel(PartialParams p) {
     count = c_last - c_first + 1;
   }
   if (h < p.heads)
-    merge_warp(p.ws_o, p.ws_lse, (size_t)first_slot * p.heads + h, p.heads, count,
-               p.out + ((size_t)b * p.heads + h) * kVDim, p.out_lse + (size_t)b * p.heads + h);
+    merge_warp(StridedPieces{p.ws_o, p.ws_lse, (size_t)first_slot * p.heads + h, (size_t)p.heads},
+               count, p.out + ((size_t)b * p.heads + h) * kVDim,
+               p.out_lse + (size_t)b * p.heads + h);
 }
 
 }  // namespace

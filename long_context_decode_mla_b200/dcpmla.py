@@ -62,6 +62,16 @@ def lib() -> ctypes.CDLL:
     L.mla_kv_append.argtypes = [vp, vp, i32, vp, vp, vp, i32, i32, i32, i32, vp, i32, i64, i32,
                                 vp, vp]
     L.mla_kv_append.restype = i32
+    L.dcp_merge_heads.argtypes = [vp, vp, i32, i32, i32, i32, i32, vp, vp, vp]
+    L.dcp_merge_heads.restype = i32
+    L.dcp_exchange_alloc.argtypes = [sz, ctypes.POINTER(vp), vp]
+    L.dcp_exchange_alloc.restype = i32
+    L.dcp_exchange_open.argtypes = [vp, ctypes.POINTER(vp)]
+    L.dcp_exchange_open.restype = i32
+    L.dcp_exchange_close.argtypes = [vp]
+    L.dcp_exchange_close.restype = i32
+    L.dcp_exchange_free.argtypes = [vp]
+    L.dcp_exchange_free.restype = i32
     _lib = L
     return L
 
@@ -205,6 +215,58 @@ def dcp_merge(partials, lses, out, out_lse=None, stream=None):
     rc = lib().dcp_merge(_ptr(partials), _ptr(lses), N, B, H, _ptr(out), _ptr(out_lse),
                          _stream(stream))
     _check(rc, "dcp_merge")
+
+
+MAX_MERGE_SHARDS, IPC_HANDLE_BYTES = 64, 64   # DCPMLA_MAX_MERGE_SHARDS, DCPMLA_IPC_HANDLE_BYTES
+
+
+def _addr(x) -> int:
+    return x.data_ptr() if hasattr(x, "data_ptr") else int(x)
+
+
+def dcp_merge_heads(partials, lses, batch, num_heads, head_begin, head_count, out,
+                    out_lse=None, stream=None):
+    """Merge of one slice of heads over per-shard buffers (see include/dcpmla.h).
+
+    ``partials`` / ``lses``: one entry per shard, each a tensor or a raw device
+    address of that shard's [batch, num_heads, 512] / [batch, num_heads] fp32
+    buffer (another rank's, mapped with :func:`dcp_exchange_open`, included).
+    ``out`` is [batch, head_count, 512], ``out_lse`` [batch, head_count].
+    """
+    n = len(partials)
+    if len(lses) != n:
+        raise ValueError("one LSE buffer per partial buffer")
+    po = (ctypes.c_void_p * max(n, 1))(*[_addr(x) for x in partials])
+    pl = (ctypes.c_void_p * max(n, 1))(*[_addr(x) for x in lses])
+    rc = lib().dcp_merge_heads(po, pl, n, batch, num_heads, head_begin, head_count, _ptr(out),
+                               _ptr(out_lse), _stream(stream))
+    _check(rc, "dcp_merge_heads")
+
+
+def dcp_exchange_alloc(nbytes: int) -> tuple[int, bytes]:
+    """Device buffer other processes can map: returns (address, IPC handle bytes)."""
+    ptr = ctypes.c_void_p(0)
+    handle = ctypes.create_string_buffer(IPC_HANDLE_BYTES)
+    _check(lib().dcp_exchange_alloc(nbytes, ctypes.byref(ptr), handle), "dcp_exchange_alloc")
+    return int(ptr.value), handle.raw
+
+
+def dcp_exchange_open(handle: bytes) -> int:
+    """Map another process's exchange buffer into the current device: its address."""
+    if len(handle) != IPC_HANDLE_BYTES:
+        raise ValueError(f"an IPC handle has {IPC_HANDLE_BYTES} bytes, got {len(handle)}")
+    ptr = ctypes.c_void_p(0)
+    buf = ctypes.create_string_buffer(bytes(handle), IPC_HANDLE_BYTES)
+    _check(lib().dcp_exchange_open(buf, ctypes.byref(ptr)), "dcp_exchange_open")
+    return int(ptr.value)
+
+
+def dcp_exchange_close(address: int) -> None:
+    _check(lib().dcp_exchange_close(ctypes.c_void_p(address)), "dcp_exchange_close")
+
+
+def dcp_exchange_free(address: int) -> None:
+    _check(lib().dcp_exchange_free(ctypes.c_void_p(address)), "dcp_exchange_free")
 
 
 def check_inputs(block_tables, seq_lens, num_blocks: int, num_shards: int,

@@ -193,3 +193,42 @@ def test_multi_query_fails_closed_before_any_launch():
     assert call(shard=2) == EINVAL and call(kvd=3) == EINVAL and call(bs=16) == EUNSUP
     assert call(q=FAKE + 2) == EALIGN
     assert call(batch=0) == OK                               # nothing to do
+
+
+def test_merge_heads_fails_closed_before_any_launch():
+    L = dcpmla.lib()
+    P = ctypes.c_void_p * 2
+    ok = P(FAKE, FAKE + 4096)
+
+    def call(parts=ok, lses=ok, n=2, batch=1, heads=8, h0=0, hn=4, out=FAKE):
+        return L.dcp_merge_heads(parts, lses, n, batch, heads, h0, hn, out, None, None)
+
+    assert call(n=0) == EINVAL and call(n=dcpmla.MAX_MERGE_SHARDS + 1) == EINVAL
+    assert call(heads=0) == EINVAL and call(batch=-1) == EINVAL
+    assert call(h0=-1) == EINVAL and call(hn=0) == EINVAL and call(h0=5, hn=4) == EINVAL
+    assert call(parts=None) == EINVAL and call(lses=None) == EINVAL and call(out=None) == EINVAL
+    assert call(parts=P(FAKE, None)) == EINVAL and call(lses=P(None, FAKE)) == EINVAL
+    assert call(parts=P(FAKE, FAKE + 4)) == EALIGN and call(out=FAKE + 8) == EALIGN
+    assert call(batch=0, parts=None, lses=None, out=None) == OK      # nothing to do
+
+
+def test_merge_heads_limits_match_header():
+    text = open(HEADER).read()
+    assert re.search(r"#define DCPMLA_MAX_MERGE_SHARDS (\d+)", text).group(1) == \
+        str(dcpmla.MAX_MERGE_SHARDS)
+    assert re.search(r"#define DCPMLA_IPC_HANDLE_BYTES (\d+)", text).group(1) == \
+        str(dcpmla.IPC_HANDLE_BYTES)
+
+
+def test_exchange_calls_refuse_null_arguments():
+    L = dcpmla.lib()
+    h = ctypes.create_string_buffer(dcpmla.IPC_HANDLE_BYTES)
+    p = ctypes.c_void_p(0)
+    assert L.dcp_exchange_alloc(0, ctypes.byref(p), h) == EINVAL
+    assert L.dcp_exchange_alloc(1024, None, h) == EINVAL
+    assert L.dcp_exchange_alloc(1024, ctypes.byref(p), None) == EINVAL
+    assert L.dcp_exchange_open(None, ctypes.byref(p)) == EINVAL
+    assert L.dcp_exchange_open(h, None) == EINVAL
+    assert L.dcp_exchange_close(None) == EINVAL and L.dcp_exchange_free(None) == EINVAL
+    with pytest.raises(ValueError):
+        dcpmla.dcp_exchange_open(b"short")
