@@ -243,9 +243,13 @@ __device__ __forceinline__ __half2 e4m3x2_to_f16x2(uint32_t pair) {
 }
 
 // Scales outside the fp16 fast path (rare): fp32 products rounded once,
-// with clamping; returns true if a product was clamped.  Kept out of line
-// so the hot conversion code stays small.
-__device__ __noinline__ bool e4m3x16_to_f16_slow(const uint4 v, float sc, uint4& lo, uint4& hi) {
+// with clamping, stored to dst_lo / dst_hi; returns true if a product was
+// clamped.  Kept out of line so the hot conversion code stays small; it
+// stores its results itself so that the caller's values never need an
+// address (a by-reference result would put them in local memory on every
+// call, fast path included).
+__device__ __noinline__ bool e4m3x16_to_f16_slow(const uint4 v, float sc, uint4* dst_lo,
+                                                 uint4* dst_hi) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
   uint32_t o[8];
   float amax = 0.f;
@@ -259,12 +263,13 @@ __device__ __noinline__ bool e4m3x16_to_f16_slow(const uint4 v, float sc, uint4&
       o[2 * i + hw] = f16x2_sat(a, b);
     }
   }
-  lo = make_uint4(o[0], o[1], o[2], o[3]);
-  hi = make_uint4(o[4], o[5], o[6], o[7]);
+  *dst_lo = make_uint4(o[0], o[1], o[2], o[3]);
+  *dst_hi = make_uint4(o[4], o[5], o[6], o[7]);
   return amax > kF16Max;
 }
 
-// 16 e4m3 codes times `sc` -> 16 fp16 (two 16-byte units, dims in order).
+// 16 e4m3 codes times `sc` -> 16 fp16 stored as two 16-byte units (dims in
+// order) at dst_lo and dst_hi.
 // e4m3 -> fp16 is exact.  When every product stays a finite normal-range
 // fp16 number (2^-14 <= sc <= 65504 / 448) the product is taken in fp16 with
 // the scale split into sc_hi = fp16(sc) and sc_lo = fp16(sc - sc_hi):
@@ -273,8 +278,10 @@ __device__ __noinline__ bool e4m3x16_to_f16_slow(const uint4 v, float sc, uint4&
 // of a group, which moves large scores coherently.  Other scales take the
 // fp32 product, rounded once, with clamping.  Returns true if a product was
 // clamped (only possible off the fast path).
-__device__ __forceinline__ bool e4m3x16_to_f16(const uint4 v, float sc, uint4& lo, uint4& hi) {
-  if (!(sc >= 6.103515625e-05f && sc <= 146.0f)) return e4m3x16_to_f16_slow(v, sc, lo, hi);
+__device__ __forceinline__ bool e4m3x16_to_f16(const uint4 v, float sc, uint4* dst_lo,
+                                               uint4* dst_hi) {
+  if (!(sc >= 6.103515625e-05f && sc <= 146.0f))
+    return e4m3x16_to_f16_slow(v, sc, dst_lo, dst_hi);
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
   uint32_t o[8];
   const __half s_hi = __float2half_rn(sc);
@@ -289,8 +296,8 @@ __device__ __forceinline__ bool e4m3x16_to_f16(const uint4 v, float sc, uint4& l
       o[2 * i + hw] = *reinterpret_cast<const uint32_t*>(&r2);
     }
   }
-  lo = make_uint4(o[0], o[1], o[2], o[3]);
-  hi = make_uint4(o[4], o[5], o[6], o[7]);
+  *dst_lo = make_uint4(o[0], o[1], o[2], o[3]);
+  *dst_hi = make_uint4(o[4], o[5], o[6], o[7]);
   return false;
 }
 
@@ -727,10 +734,9 @@ __device__ __forceinline__ void stage_store_group(uint8_t* stage, int ct, const 
 #pragma unroll
   for (int i = 0; i < 2; ++i) {
     const int r = 32 * i + (ct >> 3);
-    uint4 lo, hi;
-    range_bad |= e4m3x16_to_f16(st.c[g][i], st.s[g][i], lo, hi);
-    *reinterpret_cast<uint4*>(dst + swz(r, (u & 3) * 2)) = lo;
-    *reinterpret_cast<uint4*>(dst + swz(r, (u & 3) * 2 + 1)) = hi;
+    range_bad |= e4m3x16_to_f16(st.c[g][i], st.s[g][i],
+                                reinterpret_cast<uint4*>(dst + swz(r, (u & 3) * 2)),
+                                reinterpret_cast<uint4*>(dst + swz(r, (u & 3) * 2 + 1)));
   }
 }
 
