@@ -50,7 +50,8 @@ def parse():
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the secondary at-64K measurement")
     ap.add_argument("--shard-streams", type=int, default=None,
-                    help="CUDA streams the N shard launches are spread over (default N; 1 = serial)")
+                    help="CUDA streams the N shard launches are spread over "
+                         "(default N; 1 = serial)")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's batch (smaller cases for profiling)")
     return ap.parse_args()

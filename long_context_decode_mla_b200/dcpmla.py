@@ -41,7 +41,8 @@ def lib() -> ctypes.CDLL:
             f"{LIB_PATH} is missing: build it with `python -m long_context_decode_mla_b200.build`"
             " (the decode path has no fallback)")
     L = ctypes.CDLL(LIB_PATH)
-    vp, i32, i64, f32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+    vp, i32, i64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
+    f32, sz = ctypes.c_float, ctypes.c_size_t
     L.mla_decode_workspace_size.argtypes = [i32, i32, i32, i32, ctypes.POINTER(sz)]
     L.mla_decode_workspace_size.restype = i32
     L.mla_decode_partial.argtypes = [vp, vp, i32, i64, i32, vp, i32, vp, i32, i32, i32, i32, vp,

@@ -42,8 +42,7 @@ from __future__ import annotations
 
 import numpy as np
 
-from .mla_decode import (BF16_ROW_BYTES, FP8_ROW_BYTES, LATENT_DIM, ROPE_DIM, decode_bf16,
-                         e4m3_value)
+from .mla_decode import BF16_ROW_BYTES, FP8_ROW_BYTES, LATENT_DIM, decode_bf16, e4m3_value
 
 BLOCK_ROWS = 64
 FLAG_BAD_BLOCK = 1
@@ -93,7 +92,8 @@ def quantize_fp8_row(latent_bits: np.ndarray, rope_bits: np.ndarray) -> np.ndarr
 
 def bf16_row(latent_bits: np.ndarray, rope_bits: np.ndarray) -> np.ndarray:
     """One 1152-byte bf16 row: the 576 values as given."""
-    bits = np.concatenate([np.asarray(latent_bits, dtype="<u2"), np.asarray(rope_bits, dtype="<u2")])
+    bits = np.concatenate([np.asarray(latent_bits, dtype="<u2"),
+                           np.asarray(rope_bits, dtype="<u2")])
     out = bits.view(np.uint8)
     assert out.size == BF16_ROW_BYTES
     return out

@@ -178,7 +178,8 @@ def test_kv_append_fails_closed_before_any_launch():
 def test_multi_query_fails_closed_before_any_launch():
     L = dcpmla.lib()
     f = L.mla_decode_partial_multi
-    vp, i32, i64, f32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+    vp, i32, i64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
+    f32, sz = ctypes.c_float, ctypes.c_size_t
     f.argtypes = [vp, vp, i32, i64, i32, vp, i32, vp, i32, i32, i32, i32, i32, f32, vp, vp, vp, sz,
                   i32, i32, vp]
     f.restype = i32

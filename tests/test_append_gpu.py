@@ -29,7 +29,8 @@ def _bits(x: torch.Tensor) -> np.ndarray:
 
 def _tokens(T, seed):
     g = torch.Generator().manual_seed(seed)
-    lat = torch.randn(T, 512, generator=g) * torch.exp(torch.randn(T, 4, generator=g) * 2).repeat_interleave(128, 1)
+    group_scale = torch.exp(torch.randn(T, 4, generator=g) * 2).repeat_interleave(128, 1)
+    lat = torch.randn(T, 512, generator=g) * group_scale
     lat[0, :128] = 0.0                       # an all-zero group
     lat[1, 128:256] = -0.0                   # negative zeros
     lat[2, 256:384] *= 1e-30                 # tiny values (bf16 subnormal range)
@@ -62,7 +63,8 @@ def _append_all_shards_gpu(pool, tables, lat, rope, pos, req, kv_dtype, N):
 def _append_all_shards_oracle(pool, tables, lat, rope, pos, req, kv_dtype, N):
     cache, flags = pool, 0
     for s in range(N):
-        cache, f = oracle.kv_append(cache, kv_dtype, _bits(lat), _bits(rope), pos, req, tables[s], s, N)
+        cache, f = oracle.kv_append(cache, kv_dtype, _bits(lat), _bits(rope), pos, req,
+                                    tables[s], s, N)
         flags |= f
     return cache, flags
 
@@ -95,7 +97,8 @@ def test_out_of_range_entries_are_flagged_and_skipped():
     bad = tables.copy()
     bad[0, 1, 0] = 10 ** 6                              # block outside the pool
     lat, rope = _tokens(4, seed=1)
-    pos = np.array([0, 2 * 64 * nblk, 2, 4], dtype=np.int32)     # ok, beyond the table, bad block, ok
+    # ok, beyond the table, bad block, ok
+    pos = np.array([0, 2 * 64 * nblk, 2, 4], dtype=np.int32)
     req = np.array([0, 0, 1, 5], dtype=np.int32)                  # last: request outside [0, B)
     d_pool = torch.from_numpy(pool.copy()).cuda()
     flags = torch.zeros(1, dtype=torch.int32, device="cuda")

@@ -26,7 +26,8 @@ def _compile(tmp_path):
         from long_context_decode_mla_b200 import build
         build.build()
     exe = str(tmp_path / "decode_from_c")
-    cmd = [cc, "-O2", "-std=c99", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"),
+    cmd = [cc, "-O2", "-std=c99", "-Wall", "-Wextra", "-Werror",
+           "-I", os.path.join(ROOT, "include"),
            "-I", os.path.join(CUDA, "include"), SRC, "-L", LIBDIR, "-ldcpmla",
            "-L", os.path.join(CUDA, "lib64"), "-lcudart", f"-Wl,-rpath,{LIBDIR}",
            f"-Wl,-rpath,{os.path.join(CUDA, 'lib64')}", "-o", exe]

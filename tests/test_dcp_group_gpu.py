@@ -15,7 +15,6 @@
 Ranks on several GPUs are not run here (one GPU); the peer mapping is the
 CUDA IPC path of ``dcp_exchange_open``.
 """
-import os
 import socket
 
 import numpy as np

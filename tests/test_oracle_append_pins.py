@@ -67,7 +67,8 @@ def test_matches_an_independent_library_cast():
 
 def test_quantised_row_layout_and_defining_properties():
     g = torch.Generator().manual_seed(11)
-    lat = torch.randn(512, generator=g) * torch.tensor([0.001, 1.0, 50.0, 0.0]).repeat_interleave(128)
+    group_scale = torch.tensor([0.001, 1.0, 50.0, 0.0]).repeat_interleave(128)
+    lat = torch.randn(512, generator=g) * group_scale
     rope = torch.randn(64, generator=g)
     lb, rb = _bf16_bits(lat), _bf16_bits(rope)
     row = oracle.quantize_fp8_row(lb, rb)
@@ -157,7 +158,8 @@ def test_skips_and_flags():
     rope = _bf16_bits(torch.ones(5, 64))
     bad = tables.copy()
     bad[0, 1, 0] = 10 ** 6
-    pos = np.array([-1, 0, 2 * 64 * nblk, 4, 1], dtype=np.int32)  # pad, ok, beyond table, bad block row, non-owner
+    # pad, ok, beyond the table, bad block row, non-owner
+    pos = np.array([-1, 0, 2 * 64 * nblk, 4, 1], dtype=np.int32)
     req = np.array([0, 0, 0, 1, 0], dtype=np.int32)
     out, flags = oracle.kv_append(pool, "fp8", lat, rope, pos, req, bad[0], 0, N)
     assert flags == ka.FLAG_BAD_LENGTH | ka.FLAG_BAD_BLOCK

@@ -11,7 +11,6 @@ import math
 
 import numpy as np
 import pytest
-import torch
 
 import oracle
 from oracle import multi_query as mq
@@ -104,7 +103,8 @@ def test_brute_force_over_logical_rows():
                 want_lse = m + math.log(z)
                 assert abs(lse[b, i, h] - want_lse) < 1e-10
                 for d in (0, 7, 300, 511):
-                    want = math.fsum(math.exp(s[t] - want_lse) * float(keys[t][d]) for t in range(n))
+                    want = math.fsum(math.exp(s[t] - want_lse) * float(keys[t][d])
+                                     for t in range(n))
                     assert abs(out[b, i, h, d] - want) < 1e-10
 
 

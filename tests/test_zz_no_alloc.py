@@ -52,7 +52,8 @@ def _no_alloc(prob, shard, num_splits, impl):
 
 
 def _close(a, b, kv_dtype):
-    (o, l), (o_ref, l_ref) = [(x.double().cpu().numpy(), y.double().cpu().numpy()) for x, y in (a, b)]
+    (o, l), (o_ref, l_ref) = [(x.double().cpu().numpy(), y.double().cpu().numpy())
+                              for x, y in (a, b)]
     fin = np.isfinite(l_ref)
     assert np.array_equal(fin, np.isfinite(l))
     assert not o[~fin].any()
