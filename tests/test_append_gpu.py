@@ -29,8 +29,8 @@ def _bits(x: torch.Tensor) -> np.ndarray:
 
 def _tokens(T, seed):
     g = torch.Generator().manual_seed(seed)
-    group_scale = torch.exp(torch.randn(T, 4, generator=g) * 2).repeat_interleave(128, 1)
-    lat = torch.randn(T, 512, generator=g) * group_scale
+    lat = torch.randn(T, 512, generator=g)
+    lat = lat * torch.exp(torch.randn(T, 4, generator=g) * 2).repeat_interleave(128, 1)
     lat[0, :128] = 0.0                       # an all-zero group
     lat[1, 128:256] = -0.0                   # negative zeros
     lat[2, 256:384] *= 1e-30                 # tiny values (bf16 subnormal range)
