@@ -109,21 +109,23 @@ class DcpRankDecoder:
     """This rank's share of a real multi-GPU DCP decode step (see module doc).
 
     ``group``: the DCP process group (NCCL, one rank per GPU, the current
-    device being this rank's).  ``batch`` and ``heads`` (gathered heads, a
-    multiple of the group size) fix the buffers; ``topk`` > 0 sizes the
-    workspace for sparse decode.  Results of :meth:`step` land in ``out``
-    [batch, H/N, 512] and ``out_lse`` [batch, H/N] for this rank's heads.
-    Call :meth:`close` on every rank before the group is destroyed.
+    device being this rank's, unless ``device`` names another).  ``batch``
+    and ``heads`` (gathered heads, a multiple of the group size) fix the
+    buffers; ``topk`` > 0 sizes the workspace for sparse decode.  Results of
+    :meth:`step` land in ``out`` [batch, H/N, 512] and ``out_lse`` [batch, H/N]
+    for this rank's heads.  Call :meth:`close` on every rank before the group
+    is destroyed.
     """
 
     def __init__(self, batch: int, heads: int, group=None, topk: int = 0, num_splits: int = 0,
-                 impl: str = "auto"):
+                 impl: str = "auto", device=None):
         self.group = group
         self.rank = dist.get_rank(group)
         self.world = dist.get_world_size(group)
         self.batch, self.heads, self.num_splits, self.impl = batch, heads, num_splits, impl
         self.head_begin, self.head_count = head_slice(self.rank, self.world, heads)
-        dev = torch.device("cuda", torch.cuda.current_device())
+        dev = (torch.device("cuda", torch.cuda.current_device()) if device is None
+               else torch.device(device))
         self._lse_off, self._slot_bytes = slot_layout(batch, heads)
         self._base, handle = dcpmla.dcp_exchange_alloc(2 * self._slot_bytes)
         self._mapped = []
@@ -180,15 +182,19 @@ class DcpRankDecoder:
         self.steps += 1
         return self.out, self.out_lse
 
+    def _sync(self):
+        if self.q.is_cuda:
+            torch.cuda.synchronize(self.q.device)
+
     def close(self):
         """Unmap the peers' buffers and free this rank's, once no rank reads it."""
         if self._base is None:
             return
-        torch.cuda.synchronize()
+        self._sync()
         for addr in self._mapped:
             dcpmla.dcp_exchange_close(addr)
         self._mapped = []
         dist.all_reduce(self._tick, group=self.group)      # every rank is done reading
-        torch.cuda.synchronize()
+        self._sync()
         dcpmla.dcp_exchange_free(self._base)
         self._base = None

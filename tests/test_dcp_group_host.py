@@ -94,3 +94,91 @@ def test_query_gather_and_handle_exchange_with_gloo_ranks(world):
             for h in range(world * hn):
                 r, i = divmod(h, hn)
                 assert bool((g[b, h] == 100 * r + 10 * i + b).all())
+
+
+def _decoder_worker(rank, world, port, out_q):
+    """One gloo rank running DcpRankDecoder with the library calls recorded
+    instead of executed (no GPU here): the step's collectives are real."""
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    from long_context_decode_mla_b200 import dcpmla
+    log = []
+    base = lambda r: 0x10000000 * (r + 1)                    # noqa: E731
+
+    def alloc(nbytes):
+        log.append(("alloc", nbytes))
+        return base(rank), bytes([rank]) * dcpmla.IPC_HANDLE_BYTES
+
+    def partial(q, kv, kvd, bt, lens, shard, nshards, idx, scale, o, l, ws, splits, impl, st, bs):
+        log.append(("partial", shard, nshards, o.data_ptr(), l.data_ptr(), q.tolist()))
+
+    def merge(parts, lses, B, H, h0, hn, out, out_lse):
+        log.append(("merge", list(parts), list(lses), B, H, h0, hn))
+
+    real_all_reduce = dist.all_reduce
+
+    def all_reduce(t, group=None):
+        log.append(("all_reduce",))
+        return real_all_reduce(t, group=group)
+
+    dcpmla.dcp_exchange_alloc = alloc
+    dcpmla.dcp_exchange_open = lambda h: (log.append(("open", h[0])), base(h[0]))[1]
+    dcpmla.dcp_exchange_close = lambda a: log.append(("close", a))
+    dcpmla.dcp_exchange_free = lambda a: log.append(("free", a))
+    dcpmla.mla_decode_partial = partial
+    dcpmla.dcp_merge_heads = merge
+    dcp_group.dist.all_reduce = all_reduce
+
+    B, H = 2, 4 * world
+    dec = dcp_group.DcpRankDecoder(B, H, topk=0, num_splits=4, device="cpu")
+    for step in range(3):
+        q_local = torch.full((B, H // world, 576), float(10 * step + rank), dtype=torch.bfloat16)
+        dec.step(q_local, None, "fp8", None, None, 0.1)
+    dec.close()
+    out_q.put((rank, log, dcp_group.slot_layout(B, H)))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_rank_decoder_schedule_with_gloo_ranks(world):
+    """Per rank: its own shard id, partials into alternating slots of its own
+    buffer, the all-reduce strictly between its partial and its merge, a merge
+    over every rank's slot of the same parity (rank order) for its own heads,
+    queries gathered in rank order, and unmap -> all-reduce -> free at close."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_decoder_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    results = {r: (log, lay) for r, log, lay in (q.get(timeout=180) for _ in procs)}
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    B, H, hn = 2, 4 * world, 4
+    base = lambda r: 0x10000000 * (r + 1)                    # noqa: E731
+    for rank in range(world):
+        log, (lse_off, slot) = results[rank]
+        assert log[0] == ("alloc", 2 * slot)
+        assert sorted(e[1] for e in log if e[0] == "open") == [r for r in range(world) if r != rank]
+        steps = [e for e in log if e[0] in ("partial", "all_reduce", "merge")]
+        body, tail = steps[:9], steps[9:]
+        for k in range(3):
+            part, red, mrg = body[3 * k:3 * k + 3]
+            par = k & 1
+            assert part[:5] == ("partial", rank, world, base(rank) + par * slot,
+                                base(rank) + par * slot + lse_off)
+            gathered = torch.tensor(part[5])
+            for r in range(world):
+                assert bool((gathered[:, r * hn:(r + 1) * hn] == 10 * k + r).all())
+            assert red == ("all_reduce",)
+            assert mrg == ("merge", [base(r) + par * slot for r in range(world)],
+                           [base(r) + par * slot + lse_off for r in range(world)], B, H,
+                           rank * hn, hn)
+        assert tail == [("all_reduce",)]
+        closes = [e for e in log if e[0] in ("close", "free")]
+        assert closes[:-1] == [("close", base(r)) for r in range(world) if r != rank]
+        assert closes[-1] == ("free", base(rank))
+        assert log.index(("free", base(rank))) > len(log) - 2
