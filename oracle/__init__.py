@@ -12,6 +12,6 @@ from .cache_write import (  # noqa: F401
     bf16_row, encode_e4m3, kv_append, quantize_fp8_row,
 )
 from .multi_query import dcp_decode_multi, mla_decode_partial_multi  # noqa: F401
-from .pcp_prefill import (  # noqa: F401
+from .pcp import (  # noqa: F401
     gather_prompt_rows, pcp_chunks, pcp_prefill, pcp_prefill_rank, pcp_rank_tokens,
 )

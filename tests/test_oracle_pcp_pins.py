@@ -1,4 +1,4 @@
-"""Pins of the PCP prefill oracle (``oracle/pcp_prefill.py``), on the CPU.
+"""Pins of the PCP prefill oracle (``oracle/pcp.py``), on the CPU.
 
 Each pin checks the oracle against something other than itself:
 
@@ -23,7 +23,7 @@ import pytest
 import torch
 
 import oracle
-from oracle import pcp_prefill as pcp
+from oracle import pcp
 from long_context_decode_mla_b200 import workload as wl
 
 
