@@ -127,16 +127,7 @@ class DcpRankDecoder:
         dev = (torch.device("cuda", torch.cuda.current_device()) if device is None
                else torch.device(device))
         self._lse_off, self._slot_bytes = slot_layout(batch, heads)
-        self._base, handle = dcpmla.dcp_exchange_alloc(2 * self._slot_bytes)
-        self._mapped = []
-        self._bases = []
-        for r, h in enumerate(exchange_handles(handle, group)):
-            if r == self.rank:
-                self._bases.append(self._base)
-            else:
-                addr = dcpmla.dcp_exchange_open(h)
-                self._mapped.append(addr)
-                self._bases.append(addr)
+        self._map_exchange_buffers()
         self.q = torch.empty(batch, heads, dcpmla.HEAD_DIM, dtype=torch.bfloat16, device=dev)
         self.out = torch.empty(batch, self.head_count, dcpmla.V_DIM, device=dev)
         self.out_lse = torch.empty(batch, self.head_count, device=dev)
@@ -144,6 +135,46 @@ class DcpRankDecoder:
         self.workspace = torch.zeros(nbytes, dtype=torch.uint8, device=dev)
         self._tick = torch.zeros(1, dtype=torch.int32, device=dev)
         self.steps = 0
+
+    def _map_exchange_buffers(self):
+        """Allocate this rank's buffer and map every peer's.  All ranks agree
+        on the outcome before returning: if any rank failed (allocation or a
+        mapping), every rank unmaps, frees and raises, so none is left
+        waiting in a later collective."""
+        self._base, self._mapped, self._bases = None, [], []
+        err = None
+        handle = b""
+        try:
+            self._base, handle = dcpmla.dcp_exchange_alloc(2 * self._slot_bytes)
+        except dcpmla.DcpMlaError as e:
+            err = e
+        handles = exchange_handles(handle, self.group)
+        if err is None and all(handles):
+            try:
+                for r, h in enumerate(handles):
+                    if r == self.rank:
+                        self._bases.append(self._base)
+                    else:
+                        addr = dcpmla.dcp_exchange_open(h)
+                        self._mapped.append(addr)
+                        self._bases.append(addr)
+            except dcpmla.DcpMlaError as e:
+                err = e
+        oks = [None] * self.world
+        dist.all_gather_object(oks, err is None, group=self.group)
+        if all(oks):
+            return
+        for addr in self._mapped:
+            dcpmla.dcp_exchange_close(addr)
+        self._mapped = []
+        done = [None] * self.world
+        dist.all_gather_object(done, True, group=self.group)   # every peer has unmapped
+        if self._base is not None:
+            dcpmla.dcp_exchange_free(self._base)
+            self._base = None
+        bad = [r for r, ok in enumerate(oks) if not ok]
+        raise RuntimeError(f"rank {self.rank}: DCP exchange buffers failed on rank(s) {bad}"
+                           + (f": {err}" if err is not None else "")) from err
 
     def slot(self, rank: int, parity: int) -> tuple[int, int]:
         """Device addresses (partial, LSEs) of ``rank``'s slot ``parity``."""

@@ -182,3 +182,58 @@ def test_rank_decoder_schedule_with_gloo_ranks(world):
         assert closes[:-1] == [("close", base(r)) for r in range(world) if r != rank]
         assert closes[-1] == ("free", base(rank))
         assert log.index(("free", base(rank))) > len(log) - 2
+
+
+def _failing_map_worker(rank, world, port, out_q):
+    """Rank 1 cannot map a peer's buffer (a fake of the failing call returns
+    an error code); every rank must unmap, free and raise, none may hang."""
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    from long_context_decode_mla_b200 import dcpmla
+    log = []
+    base = lambda r: 0x10000000 * (r + 1)                    # noqa: E731
+
+    def open_(h):
+        if rank == 1:
+            raise dcpmla.DcpMlaError(-5, "dcp_exchange_open")
+        log.append(("open", h[0]))
+        return base(h[0])
+
+    dcpmla.lib = lambda: None                                # error text without the library
+    dcpmla.error_string = lambda code: "CUDA runtime error"
+    dcpmla.dcp_exchange_alloc = lambda n: (base(rank), bytes([rank]) * dcpmla.IPC_HANDLE_BYTES)
+    dcpmla.dcp_exchange_open = open_
+    dcpmla.dcp_exchange_close = lambda a: log.append(("close", a))
+    dcpmla.dcp_exchange_free = lambda a: log.append(("free", a))
+    try:
+        dcp_group.DcpRankDecoder(2, 4 * world, num_splits=4, device="cpu")
+        msg = None
+    except RuntimeError as e:
+        msg = str(e)
+    out_q.put((rank, log, msg))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_a_failed_mapping_on_one_rank_fails_every_rank_cleanly():
+    world = 3
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_failing_map_worker, args=(r, world, port, q))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    results = {r: (log, msg) for r, log, msg in (q.get(timeout=180) for _ in procs)}
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    base = lambda r: 0x10000000 * (r + 1)                    # noqa: E731
+    for rank in range(world):
+        log, msg = results[rank]
+        assert msg is not None and "rank(s) [1]" in msg
+        opened = [e[1] for e in log if e[0] == "open"]
+        closed = [e[1] for e in log if e[0] == "close"]
+        assert closed == [base(r) for r in opened]          # every mapping made is undone
+        assert log[-1] == ("free", base(rank))               # and the own buffer is freed last
