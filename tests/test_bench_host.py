@@ -1,9 +1,12 @@
-"""Host-side logic of the benchmark's multi-rank path, on CPU ranks (gloo).
+"""Host-side logic of the benchmark, on the CPU (no GPU is touched).
 
 bench.py runs one process per GPU; every rank decodes its own batch (weak
 scaling, no data-path collective) and the timings are reduced as the max over
-ranks.  These tests run that reduction with two gloo ranks on the CPU and
-check the reference arm's rank behaviour; no GPU is touched.
+ranks.  These tests run that reduction with two gloo ranks and check the
+reference arm's rank behaviour; they also check the clock summary that decides
+whether a run's clocks were valid (timed window, throttle reasons), the key
+that ties the recorded DRAM traffic to the kernel source, and the KV byte
+counts the GB/s figures divide by.
 """
 import json
 import os
@@ -82,3 +85,75 @@ def test_ranks_draw_distinct_batches():
     b = workload.make_problem("tiny", seed=seed + 1000)
     assert not torch.equal(a.kv_cache, b.kv_cache)
     assert torch.equal(a.kv_cache, workload.make_problem("tiny", seed=seed).kv_cache)
+
+
+def _sampler(samples, t_on, t_off):
+    import bench
+    s = bench.ClockSampler(0)
+    s.samples, s.t_on, s.t_off = samples, t_on, t_off
+    return s
+
+
+def test_clock_summary_reads_the_timed_window_and_throttle_reasons():
+    row = "{mhz}, 1965, 700.5, 0x{act:x}, {hw}, Not Active, Not Active, {pc}"
+    samples = [
+        (0.0, row.format(mhz=1005, act=0, hw="Not Active", pc="Not Active")),   # before: ignored
+        (1.0, row.format(mhz=1900, act=4, hw="Not Active", pc="Active")),
+        (1.1, row.format(mhz=1860, act=4, hw="Not Active", pc="Active")),
+        (1.2, row.format(mhz=1965, act=0, hw="Not Active", pc="Not Active")),
+        (1.3, "[N/A], [N/A], [N/A], [N/A], [N/A], [N/A], [N/A], [N/A]"),        # unparsable
+        (9.0, row.format(mhz=300, act=8, hw="Active", pc="Not Active")),         # after: ignored
+    ]
+    s = _sampler(samples, 0.9, 1.35).summary()
+    assert s["window"] == "timed region"
+    assert s["samples"] == 3 and s["sm_mhz"] == 1900.0 and s["sm_max_mhz"] == 1965.0
+    assert s["reasons"] == ["sw_power_cap"]
+    # a throttle seen inside the window is reported by name
+    s = _sampler(samples, 0.9, 9.5).summary()
+    assert s["reasons"] == ["hw_slowdown", "sw_power_cap"]
+
+
+def test_clock_summary_falls_back_to_the_whole_run_when_the_window_is_empty():
+    samples = [(0.0, "1965, 1965, 500, 0x0, Not Active, Not Active, Not Active, Not Active")]
+    s = _sampler(samples, 5.0, 5.01).summary()
+    assert s["window"].startswith("whole run") and s["samples"] == 1
+    assert _sampler([], None, None).summary()["sm_mhz"] is None
+
+
+def test_traffic_key_ignores_comments_but_not_code():
+    import bench
+    csrc = os.path.join(ROOT, "long_context_decode_mla_b200", "csrc")
+
+    def read(name, edit=None):
+        with open(os.path.join(csrc, name), encoding="utf-8") as f:
+            text = f.read()
+        return edit(text) if edit and name == "partial_tc.cu" else text
+
+    base = bench.kernel_source_hash(read)
+    assert base == bench.kernel_source_hash()
+    recomment = lambda t: "// a new comment\n/* and a\n block */\n" + t.replace("\n", "  \n")  # noqa
+    commented = bench.kernel_source_hash(lambda n: read(n, recomment))
+    assert commented == base
+    changed = bench.kernel_source_hash(lambda n: read(n, lambda t: t + "\nstatic int x = 1;\n"))
+    assert changed != base
+
+
+def test_recorded_traffic_is_dropped_when_the_kernel_source_changes(monkeypatch):
+    import bench
+    with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+        entry = json.load(f)["agentic/auto"]
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda read=None: entry["source_hash"])
+    assert bench.recorded_traffic("agentic", "auto") == entry["bytes_per_launch"]
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda read=None: "0" * 16)
+    assert bench.recorded_traffic("agentic", "auto") is None
+    assert bench.recorded_traffic("no-such-workload", "auto") is None
+
+
+def test_shard_kv_bytes_add_up_to_the_step():
+    import bench
+    from long_context_decode_mla_b200 import workload
+    for name, over in (("tiny", {}), ("dense", dict(batch=3, seq_len=[700, 1, 0])),
+                       ("sparse", dict(batch=2, seq_len=[5000, 100], topk=256))):
+        for N in (1, 3, 8):
+            p = workload.make_problem(name, num_shards=N, **over)
+            assert sum(bench.shard_kv_bytes(p, s) for s in range(N)) == bench.kv_bytes(p)
