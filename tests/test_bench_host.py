@@ -131,7 +131,9 @@ def test_traffic_key_ignores_comments_but_not_code():
 
     base = bench.kernel_source_hash(read)
     assert base == bench.kernel_source_hash()
-    recomment = lambda t: "// a new comment\n/* and a\n block */\n" + t.replace("\n", "  \n")  # noqa
+    def recomment(t):
+        return "// a new comment\n/* and a\n block */\n" + t.replace("\n", "  \n")
+
     commented = bench.kernel_source_hash(lambda n: read(n, recomment))
     assert commented == base
     changed = bench.kernel_source_hash(lambda n: read(n, lambda t: t + "\nstatic int x = 1;\n"))
