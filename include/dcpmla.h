@@ -34,10 +34,12 @@
  *    is 64 rows.
  *
  * Conventions for every entry point:
- *  - All array pointers are DEVICE pointers owned by the caller.  The library
- *    allocates no memory, never synchronises, and only enqueues work on
- *    `stream` (a cudaStream_t; NULL means the legacy default stream).  The
- *    call returns once the work is enqueued.
+ *  - All array pointers are DEVICE pointers owned by the caller (except the
+ *    host pointer tables of dcp_merge_heads).  The compute calls allocate no
+ *    memory, never synchronise, and only enqueue work on `stream` (a
+ *    cudaStream_t; NULL means the legacy default stream); they return once the
+ *    work is enqueued.  The dcp_exchange_* calls are the exception: they
+ *    exist to allocate, map and free exchange buffers, and may synchronise.
  *  - Arguments are checked on the host, before anything is launched; a
  *    failed check returns a negative DCPMLA_ERR_* code and launches nothing
  *    (fail closed: nothing is clamped or guessed).  Device-side contents
