@@ -3,7 +3,8 @@
 Each pin checks the oracle against something other than itself:
 
 * the chunk plan against the definition (2P contiguous chunks in prompt
-  order, sizes within one) and the page's geometry (8 ranks -> 16 chunks);
+  order, sizes within one) and the page's geometry (``tests/golden/
+  pcp_geometry.json``: 8 ranks, 16 chunks, all 64 heads per rank);
 * the front/back pairing against its closed form: with c tokens per chunk,
   every rank's causal work sum_{i in rank}(i + 1) is (2P - 1) c^2 + c (c + 1),
   and the ranks add up to T (T + 1) / 2;
@@ -16,7 +17,9 @@ Each pin checks the oracle against something other than itself:
 * a planted off-by-one (a query that does not see itself) against the
   decode path, which it must fail.
 """
+import json
 import math
+import os
 
 import numpy as np
 import pytest
@@ -43,15 +46,25 @@ def test_chunk_plan_partitions_the_prompt(T, P):
 
 
 def test_page_geometry_and_pairing():
-    # 8 ranks, 16 chunks; rank r holds chunk r and chunk 15 - r
-    chunks = pcp.pcp_chunks(1600, 8)
-    assert len(chunks) == 16 and all(b - a == 100 for a, b in chunks)
-    for r in range(8):
-        tok = pcp.pcp_rank_tokens(1600, 8, r)
+    with open(os.path.join(os.path.dirname(__file__), "golden", "pcp_geometry.json")) as f:
+        g = json.load(f)
+    P, n = g["ranks"], g["chunks"]
+    T = 100 * n
+    chunks = pcp.pcp_chunks(T, P)
+    assert len(chunks) == n and all(b - a == 100 for a, b in chunks)
+    # rank r holds chunk r (front) and chunk n - 1 - r (back)
+    for r in range(P):
+        tok = pcp.pcp_rank_tokens(T, P, r)
         assert tok.tolist() == list(range(100 * r, 100 * r + 100)) + \
-            list(range(100 * (15 - r), 100 * (15 - r) + 100))
+            list(range(100 * (n - 1 - r), 100 * (n - 1 - r) + 100))
     with pytest.raises(ValueError):
-        pcp.pcp_rank_tokens(1600, 8, 8)
+        pcp.pcp_rank_tokens(T, P, P)
+    # every rank computes all heads for its tokens: the oracle's rank step
+    # returns every head of the query rows it is given
+    rows = np.random.default_rng(0).standard_normal((3, 576))
+    q = np.random.default_rng(1).standard_normal((3, g["heads_per_rank"], 576))
+    o, lse = pcp.pcp_prefill_rank(q, rows, np.array([0, 2]), 0.05)
+    assert o.shape == (2, g["heads_per_rank"], 512) and lse.shape == (2, g["heads_per_rank"])
 
 
 @pytest.mark.parametrize("P,c", [(1, 7), (2, 5), (8, 64), (8, 4096)])
