@@ -66,9 +66,16 @@ extern "C" {
 /* Kernel selection for mla_decode_partial. */
 #define DCPMLA_IMPL_AUTO 0   /* fastest available for the arguments */
 #define DCPMLA_IMPL_SIMT 1   /* plain CUDA-core kernel (any H <= 64) */
-#define DCPMLA_IMPL_TC 2     /* tcgen05 / TMEM tensor-core kernel */
-/* Test only, OR-ed into DCPMLA_IMPL_TC: the converter warps withhold their
- * first arrival, so every pipeline wait of every CTA runs out (about 2 s);
+#define DCPMLA_IMPL_TC 2     /* tcgen05 / TMEM tensor-core kernel: fp8 rows (dense,
+                                one query token) go to the kernel that multiplies
+                                the e4m3 codes directly; everything else to the
+                                fp16-operand kernel */
+#define DCPMLA_IMPL_TC_F16 3 /* the fp16-operand tensor-core kernel for every
+                                argument combination it supports (bf16 rows, fp8
+                                rows converted to fp16; kept for comparison) */
+/* Test only, OR-ed into DCPMLA_IMPL_TC or DCPMLA_IMPL_TC_F16: the kernel's
+ * first tile is never delivered, so every pipeline wait of every CTA runs
+ * out (about 2 s);
  * the kernel then drains, frees its tensor memory, sets
  * DCPMLA_FLAG_TIMEOUT and returns with invalid outputs.  Exercises the
  * timeout path; the context stays usable. */

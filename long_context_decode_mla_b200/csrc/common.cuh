@@ -18,6 +18,7 @@ constexpr int kMaxHeads = 64;
 constexpr int kRowBytesBf16 = 1152;
 constexpr int kRowBytesFp8 = 656;
 constexpr int kWsHeader = 256;    // workspace header: flag word + reserved
+constexpr int kMaxDevicesConfigured = 64;   // device ordinals the per-device caches cover
 
 enum : int { kKvBf16 = 0, kKvFp8 = 1 };
 enum : int { kFlagBadBlock = 1, kFlagBadLength = 2 };

@@ -114,13 +114,15 @@ int decode_partial(const void* q, const void* kv_cache, int kv_dtype, int64_t nu
   // ---- scalar checks (fail closed, nothing launched on error) ----
   const bool withhold = (impl & DCPMLA_TEST_WITHHOLD_ARRIVAL) != 0;
   impl &= ~DCPMLA_TEST_WITHHOLD_ARRIVAL;
-  if (withhold && impl != DCPMLA_IMPL_TC) return DCPMLA_ERR_INVALID_ARGUMENT;
+  if (withhold && impl != DCPMLA_IMPL_TC && impl != DCPMLA_IMPL_TC_F16)
+    return DCPMLA_ERR_INVALID_ARGUMENT;
   if (batch < 0 || num_heads < 1 || num_shards < 1 || shard_id < 0 || shard_id >= num_shards ||
       block_size < 1 || block_table_stride < 1 || num_blocks < 1 || num_splits < 0 ||
       topk < 0 || (sparse_idx && topk < 1) || !std::isfinite(softmax_scale))
     return DCPMLA_ERR_INVALID_ARGUMENT;
   if (kv_dtype != DCPMLA_KV_BF16 && kv_dtype != DCPMLA_KV_FP8) return DCPMLA_ERR_INVALID_ARGUMENT;
-  if (impl != DCPMLA_IMPL_AUTO && impl != DCPMLA_IMPL_SIMT && impl != DCPMLA_IMPL_TC)
+  if (impl != DCPMLA_IMPL_AUTO && impl != DCPMLA_IMPL_SIMT && impl != DCPMLA_IMPL_TC &&
+      impl != DCPMLA_IMPL_TC_F16)
     return DCPMLA_ERR_INVALID_ARGUMENT;
   if (num_heads > kMaxHeads || block_size != kBlock) return DCPMLA_ERR_UNSUPPORTED;
   if (batch == 0) return DCPMLA_OK;
@@ -165,12 +167,28 @@ int decode_partial(const void* q, const void* kv_cache, int kv_dtype, int64_t nu
   p.test_withhold = withhold ? 1 : 0;
 
   const bool tc_ok = tc_supports(p, kv_dtype);
-  if (impl == DCPMLA_IMPL_TC && !tc_ok) return DCPMLA_ERR_UNSUPPORTED;
-  const bool use_tc = impl == DCPMLA_IMPL_TC || (impl == DCPMLA_IMPL_AUTO && tc_ok);
-  if (q_len > 1 && !use_tc) return DCPMLA_ERR_UNSUPPORTED;   // causal rows: tensor-core kernel only
+  const bool f8_ok = f8_supports(p, kv_dtype);
+  enum { kSimt, kTc16, kTc8 } which;
+  if (impl == DCPMLA_IMPL_SIMT) {
+    which = kSimt;
+  } else if (impl == DCPMLA_IMPL_TC_F16) {
+    if (!tc_ok) return DCPMLA_ERR_UNSUPPORTED;
+    which = kTc16;
+  } else if (f8_ok) {
+    which = kTc8;
+  } else if (tc_ok) {
+    which = kTc16;
+  } else if (impl == DCPMLA_IMPL_TC) {
+    return DCPMLA_ERR_UNSUPPORTED;
+  } else {
+    which = kSimt;
+  }
+  if (q_len > 1 && which == kSimt) return DCPMLA_ERR_UNSUPPORTED;   // causal rows: tensor cores only
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  cudaError_t e = use_tc ? launch_partial_tc(p, kv_dtype, st) : launch_partial_simt(p, kv_dtype, st);
+  cudaError_t e = which == kTc8    ? launch_partial_f8(p, st)
+                  : which == kTc16 ? launch_partial_tc(p, kv_dtype, st)
+                                   : launch_partial_simt(p, kv_dtype, st);
   if (e != cudaSuccess) return DCPMLA_ERR_CUDA;
   e = launch_split_combine(p, st);
   return e == cudaSuccess ? DCPMLA_OK : DCPMLA_ERR_CUDA;

@@ -10,6 +10,8 @@ namespace dcpmla {
 cudaError_t launch_partial_simt(const PartialParams& p, int kv_dtype, cudaStream_t st);
 cudaError_t launch_partial_tc(const PartialParams& p, int kv_dtype, cudaStream_t st);
 bool tc_supports(const PartialParams& p, int kv_dtype);
+cudaError_t launch_partial_f8(const PartialParams& p, cudaStream_t st);
+bool f8_supports(const PartialParams& p, int kv_dtype);
 cudaError_t launch_split_combine(const PartialParams& p, cudaStream_t st);
 cudaError_t launch_dcp_merge(const float* partials, const float* lses, int num_shards, int batch,
                              int heads, float* out, float* out_lse, cudaStream_t st);

@@ -44,6 +44,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "schedule.cuh"
 #include "tc_ptx.cuh"
 
 namespace dcpmla {
@@ -59,7 +60,6 @@ constexpr int kNumSlots = 9;           // per stage: 8 latent chunks + rope (the
 constexpr int kRopeSlot = 8;
 constexpr int kStages = 2;
 constexpr int kQBytes = 9 * 8192;
-constexpr int kMaxSeg = 128;
 // A stage is filled, and its scores issued, in five parts: the four 128-value
 // scale groups of the latent row (two 64-value chunk slots each, 8 K-steps)
 // and the rope slot (4 K-steps).  The MMA starts on a part as soon as it
@@ -90,19 +90,12 @@ struct TcCtl {
   float lred[2][64];
   int sel_count;
   int warp_sums[16];
-  Segment seg[kMaxSeg];
+  Segment seg[kSchedMaxSeg];
 };
 
 constexpr size_t kSmemBytes =
     kQBytes + (size_t)kStages * kNumSlots * kSlotBytes + sizeof(TcCtl) + 1024;
 
-struct SegView {
-  int b;
-  int row_begin;   // first local row (dense); 0 (sparse, rows come from the list)
-  int nrows;
-  int ntiles;
-  bool whole;
-};
 
 __device__ __forceinline__ uint32_t swz(int row, int unit) {
   return (uint32_t)((row >> 3) * 1024 + (row & 7) * 128 + ((unit ^ (row & 7)) << 4));
@@ -112,23 +105,6 @@ __device__ __forceinline__ uint8_t* slot_ptr(uint8_t* sslot, int stage, int c) {
   return sslot + (stage * kNumSlots + c) * kSlotBytes;
 }
 
-__device__ __forceinline__ SegView seg_view(const PartialParams& p, const TcCtl& c, int k) {
-  SegView v;
-  if (p.sparse_idx) {
-    v.b = blockIdx.x / p.sparse_parts;
-    v.row_begin = 0;
-    v.nrows = c.sel_count;
-    v.whole = p.sparse_parts == 1;
-  } else {
-    const Segment s = c.seg[k];
-    v.b = s.b;
-    v.row_begin = s.t0 * kBlock;
-    v.nrows = min(s.n_rows, s.t1 * kBlock) - v.row_begin;
-    v.whole = s.t0 == 0 && s.t1 == s.nt;
-  }
-  v.ntiles = (v.nrows + kTileTok - 1) / kTileTok;
-  return v;
-}
 
 // Address of row r of tile `tile` of the segment, or nullptr if it is past
 // the end or its block-table entry is out of range (flagged).
@@ -198,33 +174,6 @@ __device__ __forceinline__ void prefetch_tile(const PartialParams& p, const SegV
   }
 }
 
-// Walks the CTA's tiles in order: segment k, tile t (segments without tiles
-// are skipped).  Returns false past the last tile.
-struct TileCursor {
-  int k, t, nseg;
-  SegView v;
-  __device__ __forceinline__ bool start(const PartialParams& p, const TcCtl& c, int n) {
-    nseg = n;
-    k = 0;
-    t = 0;
-    while (k < nseg) {
-      v = seg_view(p, c, k);
-      if (v.ntiles > 0) return true;
-      ++k;
-    }
-    return false;
-  }
-  __device__ __forceinline__ bool next(const PartialParams& p, const TcCtl& c) {
-    if (++t < v.ntiles) return true;
-    t = 0;
-    while (++k < nseg) {
-      v = seg_view(p, c, k);
-      if (v.ntiles > 0) return true;
-    }
-    return false;
-  }
-  __device__ __forceinline__ bool last_of_segment() const { return t == v.ntiles - 1; }
-};
 
 // fp32 pair -> fp16 pair (lo in the low half), rounded to nearest, clamped
 // to +-65504.
@@ -312,72 +261,6 @@ __device__ __forceinline__ uint4 bf16x8_to_f16(const uint4 v, float& amax) {
     o[i] = f16x2_sat(a, b);
   }
   return make_uint4(o[0], o[1], o[2], o[3]);
-}
-
-// ------------------------------------------------------------- segments ----
-
-// Collect this CTA's dense segments number [first, first + kMaxSeg) in request
-// order into c.seg.  Returns the total number of segments of the CTA.
-__device__ int collect_segments(const PartialParams& p, int lo, int hi, int first, TcCtl& c) {
-  int off = 0, seen = 0;
-  for (int base = 0; base < p.batch && off < hi; base += blockDim.x) {
-    const int b = base + threadIdx.x;
-    int n = 0, nt = 0;
-    if (b < p.batch) nt = request_tiles(p, b, &n);
-    int tot;
-    const int start = off + block_exclusive_scan(nt, c.warp_sums, &tot);
-    const int inter = (nt > 0 && start < hi && start + nt > lo) ? 1 : 0;
-    int tot_inter;
-    const int idx = seen + block_exclusive_scan(inter, c.warp_sums, &tot_inter);
-    if (inter && idx >= first && idx < first + kMaxSeg) {
-      Segment s;
-      s.b = b;
-      s.t0 = max(lo, start) - start;
-      s.t1 = min(hi, start + nt) - start;
-      s.n_rows = n;
-      s.nt = nt;
-      c.seg[idx - first] = s;
-    }
-    seen += tot_inter;
-    off += tot;
-  }
-  __syncthreads();
-  return seen;
-}
-
-// Sparse mode: this CTA's chunk of the index list, filtered to the positions
-// this shard owns, as local indices (in list order) into `list`.
-__device__ int compact_sparse(const PartialParams& p, int* list, TcCtl& c) {
-  const int b = blockIdx.x / p.sparse_parts, part = blockIdx.x % p.sparse_parts;
-  const int chunk = (p.topk + p.sparse_parts - 1) / p.sparse_parts;
-  const int i0 = part * chunk, i1 = min(p.topk, i0 + chunk);
-  int L = __ldg(p.seq_lens + b);
-  if (L < 0) {
-    if (threadIdx.x == 0 && p.flags) atomicOr(p.flags, kFlagBadLength);
-    L = 0;
-  }
-  int count = 0;
-  for (int base = i0; base < i1; base += blockDim.x) {
-    const int i = base + threadIdx.x;
-    int sel = 0, j = 0;
-    if (i < i1) {
-      const int t = __ldg(p.sparse_idx + (size_t)b * p.topk + i);
-      if (t >= 0 && t < L && t % p.nshards == p.shard) {
-        j = t / p.nshards;
-        if ((j >> 6) < p.bt_stride) {
-          sel = 1;
-        } else if (p.flags) {
-          atomicOr(p.flags, kFlagBadLength);
-        }
-      }
-    }
-    int tot;
-    const int pos = count + block_exclusive_scan(sel, c.warp_sums, &tot);
-    if (sel) list[pos] = j;
-    count += tot;
-  }
-  __syncthreads();
-  return count;
 }
 
 // ------------------------------------------------------------- roles -------
@@ -968,7 +851,7 @@ __global__ void __launch_bounds__(kThreads, 1) partial_tc_kernel(const PartialPa
       nseg = total = 1;
     } else {
       total = lo < hi ? collect_segments(p, lo, hi, first, c) : 0;
-      nseg = min(kMaxSeg, total - first);
+      nseg = min(kSchedMaxSeg, total - first);
     }
     if (nseg <= 0) break;
     if (warp < 4) {
@@ -983,7 +866,7 @@ __global__ void __launch_bounds__(kThreads, 1) partial_tc_kernel(const PartialPa
     }
     __syncthreads();
     if (c.abort) break;
-    first += kMaxSeg;
+    first += kSchedMaxSeg;
     if (p.sparse_idx || total <= first) break;
   }
   // Drain: every tcgen05.commit arrives on its mbarrier asynchronously.  The

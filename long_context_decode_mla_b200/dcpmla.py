@@ -18,7 +18,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libdcpmla.so")
 
 KV_DTYPES = {"bf16": 0, "fp8": 1}
-IMPLS = {"auto": 0, "simt": 1, "tc": 2}
+IMPLS = {"auto": 0, "simt": 1, "tc": 2, "tc16": 3}
 HEAD_DIM, V_DIM, BLOCK_SIZE, MAX_HEADS = 576, 512, 64, 64
 FLAG_BAD_BLOCK, FLAG_BAD_LENGTH, FLAG_TIMEOUT, FLAG_RANGE = 1, 2, 4, 8
 
