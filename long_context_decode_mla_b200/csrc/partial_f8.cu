@@ -15,7 +15,9 @@
 //  * Q (bf16, 8 significant bits) is split per head into two e4m3 terms in
 //    one power-of-two frame, q * 2^a = hi + lo.  That is exact for every
 //    element above 2^-9 of the head's largest (smaller ones lose low bits and
-//    weigh at most 2^-9 of it).  hi and lo are two MMAs into one accumulator.
+//    weigh at most 2^-9 of it).  hi and lo are two MMAs into one accumulator
+//    that share the key operand through a tensor-core collector buffer, so
+//    the codes are read from shared memory once.
 //  * Each 128-value scale group of the latent row has its own accumulator
 //    (weight-stationary M = 64 heads, N = 64 tokens): codes . (hi + lo) for
 //    that group.  The softmax threads multiply it by the token's fp32 group
@@ -24,26 +26,28 @@
 //  * A part takes 32 TMEM columns; eight part buffers hold more than a tile,
 //    so the scores of the next tile are computed while this one's softmax
 //    runs.
-//  * Online softmax in base 2 with a lazily updated running max (O is only
-//    rescaled when the max grows by more than 2^3).
+//  * Online softmax in base 2 with a lazily updated running max, decided per
+//    head (a head's O is rescaled only when its max grows by more than 2^3).
 //  * O += P V reads V as the same e4m3 codes.  The group scale multiplies P:
-//    for group g, P_g = p * s_tg * (8 / S_g), stored as two e4m3 terms (a
-//    Veltkamp split in fp16: hi keeps 4 leading bits, lo the rest rounded to
-//    4 bits; about 8 significant bits together) in a 64 x 64 K-major tile per
-//    term.  S_g is a per-request reference scale (the group's largest scale
-//    in the request's first tile, raised with an exact O rescale if a later
-//    tile holds a scale more than 4x larger), so P_g stays below 256 and the
-//    tokens that carry the softmax mass stay in the e4m3 normal range; the
-//    epilogue multiplies O_g back by S_g / 8.
+//    for group g, P_g = p * s_tg * (8 / S_g), stored as two e4m3 terms (hi:
+//    the 4 leading bits of the fp16 value, lo: the rest rounded to 4 bits;
+//    within 2^-7 of P_g together) in a 64 x 64 K-major tile per term; the two
+//    PV MMAs of a term pair share V through a collector buffer.  S_g is a
+//    per-request reference scale (the group's largest scale in the request's
+//    first tile, raised with an exact O rescale if a later tile holds a scale
+//    more than 4x larger), so P_g stays below 256 and the tokens that carry
+//    the softmax mass stay in the e4m3 normal range; the epilogue multiplies
+//    O_g back by S_g / 8.
 //  * O (64 heads x 512, fp32) stays in TMEM for the whole request, in the
 //    weight-stationary M = 64 layout (one N = 128 accumulator per group).
 //
 // Roles (16 warps): 0-7 softmax and epilogue (two warps per TMEM lane
 // quarter, one per 16-column half), 8 TMA producer, 9 and 15 issue the score
-// MMAs (parts 0, 2, 4 and parts 1, 3), 10 issues the PV MMAs, 11-14 prepare
-// Q (hi / lo split) per request.  Shared
-// memory: Q 72 KB, three stages of codes and scales (3 x 33 KB), two of rope
-// (2 x 8 KB), P 32 KB.  Every wait is bounded.
+// MMAs (parts 0, 2, 4 and parts 1, 3), 10 issues the PV MMAs, 11-14 stage
+// each tile's scales (raw and as P factors, with the reference scales), clear
+// the rows past a request's end and prepare Q (hi / lo split) per request.
+// Shared memory: Q 72 KB, three stages of codes and scales (3 x 33 KB), two
+// of rope (2 x 8 KB), P 32 KB.  Every wait is bounded.
 #include <cuda.h>
 #include <cuda_fp16.h>
 #include <math_constants.h>
@@ -56,13 +60,33 @@
 #include "tc_ptx.cuh"
 
 namespace dcpmla {
+
+// Optional clock trace of CTA 1 (event x index), compiled in only when
+// DCPMLA_F8_TRACE is defined; the product build leaves it out.
+#ifdef DCPMLA_F8_TRACE
+__device__ long long g_f8_trace[24][256];
+#define F8_TRACE(ev, idx)                                                        \
+  do {                                                                           \
+    if (blockIdx.x == 1 && (idx) < 256) g_f8_trace[ev][idx] = clock64();         \
+  } while (0)
+#else
+#define F8_TRACE(ev, idx) ((void)0)
+#endif
+
 namespace {
 
 constexpr int kThreads = 512;          // 16 warps
 constexpr int kSoftWarps = 8;
-constexpr int kProdWarp = 8, kQkWarp = 9, kPvWarp = 10, kQWarp0 = 11, kQkWarp2 = 15;
+constexpr int kProdWarp = 8, kQkWarp = 9, kPvWarp = 10, kStageWarp0 = 11, kQkWarp2 = 15;
 constexpr int kSoftThreads = 32 * kSoftWarps;
-constexpr int kQThreads = 128;
+constexpr int kStageThreads = 128;
+constexpr int kBarSoft = 1, kBarStage = 2, kBarBlock = 3;   // named barriers
+constexpr int kLaunchRegs = 128;             // 65,536 / kThreads
+constexpr int kSoftRegs = 184, kOtherRegs = 72;
+static_assert(kSoftWarps * 32 * kSoftRegs + (kThreads - kSoftWarps * 32) * kOtherRegs ==
+                  kThreads * kLaunchRegs,
+              "the register split must add up to what the launch holds");
+static_assert(kSoftWarps % 4 == 0, "setmaxnreg acts on whole warpgroups");
 
 constexpr uint32_t kChunk = 8192;                 // 64 rows x 128 B
 constexpr int kCodeStages = 3, kRopeStages = 2;
@@ -94,6 +118,9 @@ constexpr float kPNorm = 8.f;           // P_g = p * s * (kPNorm / S_g)
 constexpr float kScaleSlack = 4.f;      // a tile scale up to 4 S_g needs no rescale
 constexpr int kFlagTimeout = 4;
 
+// collector buffer of the PV issuer (the score MMAs gain nothing from one)
+constexpr int kCollPv = 2;
+
 // TMA box x offset inside a row: code chunks 0..3, then the rope
 __device__ __forceinline__ int box_x(int k) { return k < 4 ? 128 * k : 528; }
 
@@ -105,21 +132,26 @@ struct F8Params {
 
 struct F8Ctl {
   alignas(16) float sT[2][4][64];   // a tile's scales, [tile parity][group][row]
-  alignas(16) __half sTp[2][4][64]; // the same times the group's P normaliser (fp16)
+  alignas(16) __half sTp[2][4][64]; // the same times kPNorm / S_g (fp16), 0 for absent rows
+  alignas(16) float sc_r[2][4];     // per group: O rescale factor S_old / S_new at this tile
+  alignas(16) float sc_ref[2][4];   // per group: S_g in force for this tile
+  alignas(16) float gw[2][4][4];    // staging: per-warp group maxima of |scale|
   float qexp[64];                   // 2^-a per head (Q frame)
-  float gpart[2][kSoftWarps][4];    // per-warp group maxima of a tile's scales
-  float mred[4][64];                // per-thread-column maxima of the tile's scores, and in
-                                    // the epilogue the per-thread-column sums
+  float mred[2][4][64];             // [tile parity] per-thread-column maxima of the scores; in
+                                    // the epilogue (other parity) the per-thread-column sums
   uint64_t full[kCodeStages];       // TMA bytes of a tile landed
+  uint64_t staged[kCodeStages];     // the tile's scales staged and absent rows cleared
   uint64_t code_empty[kCodeStages]; // PV of the slot's tile done (commit)
   uint64_t rope_empty[kRopeStages]; // rope part of the slot's tile done (commit)
   uint64_t part_full[kParts];       // score part ready (commit)
   uint64_t part_empty[kParts];      // score part read (softmax arrivals)
+  uint64_t sc_empty[2];             // softmax done with a staged scale buffer
   uint64_t p_full;                  // P written (softmax arrivals)
   uint64_t p_empty;                 // PV done reading P (commit)
   uint64_t o_full;                  // a request's last PV done (commit)
-  uint64_t q_full;                  // Q of the next request staged (Q-warp arrivals)
-  uint64_t q_empty;                 // a request's last score MMA done (commit)
+  uint64_t q_full;                  // Q of the next request staged (staging arrivals)
+  uint64_t q_empty;                 // a request's last score MMA done (commits) and its Q
+                                    // frame read (softmax arrivals)
   int nv[kCodeStages];              // rows of the slot's tile that take part (producer)
   uint32_t tmem_base;
   int abort;
@@ -140,6 +172,14 @@ __device__ __forceinline__ uint32_t sw64(int r, int u) {
 
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, F8Ctl& c) {
   return ptx::mbar_wait(bar, parity, &c.abort);
+}
+
+// One arrival per warp, made by lane 0 once the whole warp got here (the
+// barrier's count is in warps).  Shared-memory atomics are scarce while the
+// tensor core streams its operands, so threads do not arrive one by one.
+__device__ __forceinline__ void warp_arrive(uint64_t* bar) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) ptx::mbar_arrive(bar);
 }
 
 __device__ __forceinline__ float ex2(float x) {
@@ -183,41 +223,42 @@ __device__ __forceinline__ uint32_t f16x2_rn(float lo, float hi) {
   asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
   return d;
 }
-__device__ __forceinline__ uint16_t f16_rn(float x) {
-  uint16_t d;
-  asm("cvt.rn.f16.f32 %0, %1;" : "=h"(d) : "f"(x));
-  return d;
-}
 __device__ __forceinline__ uint16_t f16_sat(float x) {
   uint16_t d;
   asm("cvt.rn.satfinite.f16.f32 %0, %1;" : "=h"(d) : "f"(x));
   return d;
 }
 
-// fp16 pair x (P_g of two tokens, 0 <= x < 256) -> e4m3 hi and lo terms
-// (2 bytes each, low byte = first token).  Veltkamp split in fp16:
-// gamma = x * (2^7 + 1), hi = gamma - (gamma - x) keeps the 4 leading bits of
-// x (exact for x * 129 < 65504), so its e4m3 encoding is exact in the normal
-// range; lo = x - hi is exact in fp16 and rounded to 4 bits by the encoding.
-__device__ __forceinline__ void split_hilo(uint32_t x, uint32_t& hi, uint32_t& lo) {
-  constexpr uint32_t k129 = 0x58085808u;          // fp16 129.0 in both halves
-  const uint32_t gam = hmul2_rn(x, k129);
-  const uint32_t h = hsub2_rn(gam, hsub2_rn(gam, x));
-  const uint32_t l = hsub2_rn(x, h);
-  uint16_t eh, el;
-  asm("cvt.rn.satfinite.e4m3x2.f16x2 %0, %1;" : "=h"(eh) : "r"(h));
-  asm("cvt.rn.satfinite.e4m3x2.f16x2 %0, %1;" : "=h"(el) : "r"(l));
-  hi = eh;
-  lo = el;
+// Two fp16 pairs x0, x1 (P_g of four tokens, |x| < 256) -> their e4m3 hi
+// and lo terms, four bytes each (first token in the low byte).  hi keeps the
+// sign, exponent and 3 leading mantissa bits of each fp16 value (4
+// significant bits, exact in e4m3 in its normal range); lo = x - hi is exact
+// in fp16 and below 2^-3 |x|, and its encoding rounds it to 4 bits.
+__device__ __forceinline__ void split_hilo4(uint32_t x0, uint32_t x1, uint32_t& hi,
+                                            uint32_t& lo) {
+  constexpr uint32_t kLead = 0xFF80FF80u;
+  const uint32_t h0 = x0 & kLead, h1 = x1 & kLead;
+  const uint32_t l0 = hsub2_rn(x0, h0), l1 = hsub2_rn(x1, h1);
+  asm("{\n .reg .b16 a, b;\n"
+      " cvt.rn.satfinite.e4m3x2.f16x2 a, %1;\n"
+      " cvt.rn.satfinite.e4m3x2.f16x2 b, %2;\n"
+      " mov.b32 %0, {a, b};\n}\n"
+      : "=r"(hi)
+      : "r"(h0), "r"(h1));
+  asm("{\n .reg .b16 a, b;\n"
+      " cvt.rn.satfinite.e4m3x2.f16x2 a, %1;\n"
+      " cvt.rn.satfinite.e4m3x2.f16x2 b, %2;\n"
+      " mov.b32 %0, {a, b};\n}\n"
+      : "=r"(lo)
+      : "r"(l0), "r"(l1));
 }
 
 // ---------------------------------------------------------------- roles ----
 
 // TMA producer (one thread): tile tau goes to code slot tau % 3 and rope
 // slot tau % 2.  A tile whose table entry is out of range (flagged) loads
-// block 0 instead; the softmax treats all of its rows as absent and clears
-// them before PV.
-__device__ void producer_role(const F8Params& P, const PartialParams& p, F8Ctl& c,
+// block 0 instead; it then has no valid rows.
+__device__ __forceinline__ void producer_role(const F8Params& P, const PartialParams& p, F8Ctl& c,
                               uint8_t* base, int nseg, uint32_t& tau,
                               uint32_t (&fills)[kCodeStages]) {
   TileCursor cur, pf;
@@ -240,9 +281,9 @@ __device__ void producer_role(const F8Params& P, const PartialParams& p, F8Ctl& 
       return;
     const int blk = tile_block(p, cur.v.b, (cur.v.row_begin >> 6) + cur.t);
     const int z = blk >= 0 ? blk : 0;
-    // the softmax reads the tile's valid rows with its bytes (the arrival
-    // below releases this write)
+    // read after the bytes land (the arrival below releases this write)
     c.nv[cs] = blk >= 0 ? cur.tile_valid_rows() : 0;
+    F8_TRACE(0, tau);
     // test only: withholding the very first tile makes every pipeline wait
     // of the CTA run out, which exercises the timeout path
     if (!(p.test_withhold && tau == 0)) {
@@ -271,74 +312,71 @@ __device__ __forceinline__ uint64_t dplus(uint64_t d, uint32_t byte_off) {
   return d + (uint64_t)(byte_off >> 4);
 }
 
-// One score part: four e4m3 K-steps of 32 (hi and lo MMAs into one
-// accumulator) for group kPart < 4, or four bf16 K-steps of 16 for the rope.
-template <int kPart>
-__device__ __forceinline__ void issue_part(uint32_t d, uint64_t dqh, uint64_t dql, uint64_t dqr,
-                                           uint64_t dcode, uint64_t drope) {
+// Score MMAs.  Two threads share them: side 0 issues parts 0, 2 and 4 (the
+// rope) of each tile, side 1 parts 1 and 3; part p of tile tau is number
+// 5 tau + p and goes to part buffer (5 tau + p) % 8 (weight-stationary
+// M = 64 heads, N = 64 tokens, 32 columns).  A group part is four e4m3
+// K-steps of 32, each a hi and a lo MMA into one accumulator; the rope part
+// is four bf16 K-steps of 16.  One loop serves both sides (a small
+// instruction footprint matters more here than constant offsets).
+__device__ __forceinline__ void qk_role(int side, const PartialParams& p, F8Ctl& c, uint8_t* base,
+                                        int nseg, uint32_t& tau, uint32_t& sigma) {
   constexpr uint32_t kIdF8 = ptx::idesc_make(64, 64, 0, false, false);
   constexpr uint32_t kIdBf = ptx::idesc_make(64, 64, 1, false, false);
-  if constexpr (kPart < 4) {
-#pragma unroll
-    for (int ks = 0; ks < 4; ++ks) {
-      const uint64_t bk = dplus(dcode, kPart * kChunk + ks * 32);
-      ptx::mma_ws_f8(d, dplus(dqh, kPart * kChunk + ks * 32), bk, kIdF8, ks > 0);
-      ptx::mma_ws_f8(d, dplus(dql, kPart * kChunk + ks * 32), bk, kIdF8, 1u);
-    }
-  } else {
-#pragma unroll
-    for (int ks = 0; ks < 4; ++ks)
-      ptx::mma_ws_f16(d, dplus(dqr, ks * 32), dplus(drope, ks * 32), kIdBf, ks > 0);
-  }
-}
-
-// Score MMAs.  Two threads share them: kSide 0 issues parts 0, 2 and 4 (the
-// rope) of each tile, kSide 1 parts 1 and 3; part p of tile tau is number
-// 5 tau + p and goes to part buffer (5 tau + p) % 8 (weight-stationary
-// M = 64 heads, N = 64 tokens, 32 columns).
-template <int kSide>
-__device__ void qk_role(const PartialParams& p, F8Ctl& c, uint8_t* base, int nseg,
-                        uint32_t& tau, uint32_t& sigma) {
   const uint64_t dqh = ptx::sdesc(ptx::smem_addr(base + kOffQh), 16, 1024, ptx::kSwizzle128B);
   const uint64_t dql = ptx::sdesc(ptx::smem_addr(base + kOffQl), 16, 1024, ptx::kSwizzle128B);
   const uint64_t dqr = ptx::sdesc(ptx::smem_addr(base + kOffQr), 16, 1024, ptx::kSwizzle128B);
   const uint64_t dc0 = ptx::sdesc(ptx::smem_addr(base + kOffCode), 16, 1024, ptx::kSwizzle128B);
   const uint64_t dr0 = ptx::sdesc(ptx::smem_addr(base + kOffRope), 16, 1024, ptx::kSwizzle128B);
+  const int nparts = side == 0 ? 3 : 2;
   TileCursor cur;
   if (!cur.start(p, c, nseg)) return;
   while (true) {
     const uint32_t cs = tau % kCodeStages, rs = tau % kRopeStages;
     if (cur.t == 0 && !wait_or_abort(&c.q_full, sigma & 1, c)) return;
-    if (!wait_or_abort(&c.full[cs], (tau / kCodeStages) & 1, c)) return;
-    // stay at most one tile ahead of PV: the scores of tile tau are issued
-    // once the PV of tile tau - 2 is done (the release of its code slot, a
-    // barrier that cannot complete its next phase before these scores), so
-    // that a PV never waits behind score MMAs of tiles far ahead
-    if (tau >= 2 &&
-        !wait_or_abort(&c.code_empty[(tau - 2) % kCodeStages], ((tau - 2) / kCodeStages) & 1, c))
+    // the tile's bytes and scales are staged; and stay at most one tile
+    // ahead of PV: the scores of tile tau are issued once the PV of tile
+    // tau - 2 is done (the release of its code slot, a barrier that cannot
+    // complete its next phase before these scores), so that a PV never
+    // waits behind score MMAs of tiles far ahead
+    const uint32_t tp = tau - 2;
+    uint64_t* thr = tau >= 2 ? &c.code_empty[tp % kCodeStages] : &c.staged[cs];
+    const uint32_t thr_par = tau >= 2 ? (tp / kCodeStages) & 1 : (tau / kCodeStages) & 1;
+    if (!ptx::mbar_wait3(&c.staged[cs], (tau / kCodeStages) & 1, thr, thr_par, thr, thr_par,
+                         &c.abort))
       return;
+    if (side == 0) F8_TRACE(1, tau);
     const uint64_t dcode = dplus(dc0, cs * kCodeStage), drope = dplus(dr0, rs * kChunk);
-    constexpr int kNum = kSide == 0 ? 3 : 2;
-#pragma unroll
-    for (int k = 0; k < kNum; ++k) {
-      const int part = kSide + 2 * k;
+#pragma unroll 1
+    for (int k = 0; k < nparts; ++k) {
+      const int part = side + 2 * k;
       const uint32_t pi = 5 * tau + part, buf = pi % kParts;
       if (pi >= (uint32_t)kParts &&
           !wait_or_abort(&c.part_empty[buf], ((pi / kParts) + 1) & 1, c))
         return;
       ptx::tc_fence_after();
+      F8_TRACE(12, pi);
       const uint32_t d = c.tmem_base + kColPart + 32 * buf;
-      if (kSide == 0) {
-        if (k == 0) issue_part<0>(d, dqh, dql, dqr, dcode, drope);
-        if (k == 1) issue_part<2>(d, dqh, dql, dqr, dcode, drope);
-        if (k == 2) issue_part<4>(d, dqh, dql, dqr, dcode, drope);
+      if (part < 4) {
+        const uint32_t off = part * kChunk;
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+          const uint64_t bk = dplus(dcode, off + ks * 32);
+          ptx::mma_ws_f8(d, dplus(dqh, off + ks * 32), bk, kIdF8, ks > 0);
+          ptx::mma_ws_f8(d, dplus(dql, off + ks * 32), bk, kIdF8, 1u);
+        }
       } else {
-        if (k == 0) issue_part<1>(d, dqh, dql, dqr, dcode, drope);
-        if (k == 1) issue_part<3>(d, dqh, dql, dqr, dcode, drope);
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+          ptx::mma_ws_f16(d, dplus(dqr, ks * 32), dplus(drope, ks * 32), kIdBf, ks > 0);
       }
       ptx::mma_commit(&c.part_full[buf]);
+      F8_TRACE(13, pi);
     }
-    if (kSide == 0) ptx::mma_commit(&c.rope_empty[rs]);
+    if (side == 0) {
+      ptx::mma_commit(&c.rope_empty[rs]);
+      F8_TRACE(2, tau);
+    }
     if (cur.last_of_segment()) {
       ptx::mma_commit(&c.q_empty);
       ++sigma;
@@ -350,8 +388,9 @@ __device__ void qk_role(const PartialParams& p, F8Ctl& c, uint8_t* base, int nse
 
 // PV MMAs (one thread): O_g += P_g,hi V_g + P_g,lo V_g per group, weight
 // stationary M = 64 heads, N = 128 values, K = 32 tokens; V_g is the code
-// chunk g of the tile's slot read MN-major.
-__device__ void pv_role(const PartialParams& p, F8Ctl& c, uint8_t* base, int nseg, uint32_t& tau,
+// chunk g of the tile's slot read MN-major, kept in a collector buffer
+// between the hi and lo MMAs.
+__device__ __forceinline__ void pv_role(const PartialParams& p, F8Ctl& c, uint8_t* base, int nseg, uint32_t& tau,
                         uint32_t (&uses)[kCodeStages], uint32_t& o_commits) {
   constexpr uint32_t kIdPv = ptx::idesc_make(64, 128, 0, false, true);
   const uint64_t dv0 = ptx::sdesc(ptx::smem_addr(base + kOffCode), 4096, 1024, ptx::kSwizzle128B);
@@ -362,6 +401,7 @@ __device__ void pv_role(const PartialParams& p, F8Ctl& c, uint8_t* base, int nse
     const uint32_t cs = tau % kCodeStages;
     if (!wait_or_abort(&c.p_full, tau & 1, c)) return;
     ptx::tc_fence_after();
+    F8_TRACE(3, tau);
     const uint64_t dv = dplus(dv0, cs * kCodeStage);
     const uint32_t acc0 = cur.t == 0 ? 0u : 1u;
 #pragma unroll
@@ -370,12 +410,16 @@ __device__ void pv_role(const PartialParams& p, F8Ctl& c, uint8_t* base, int nse
 #pragma unroll
       for (int ks = 0; ks < 2; ++ks) {
         const uint64_t bv = dplus(dv, g * kChunk + ks * 4096);
-        ptx::mma_ws_f8(d, dplus(dp, (2 * g) * kPVar + ks * 32), bv, kIdPv, ks == 0 ? acc0 : 1u);
-        ptx::mma_ws_f8(d, dplus(dp, (2 * g + 1) * kPVar + ks * 32), bv, kIdPv, 1u);
+        ptx::mma_ws_f8_coll<kCollPv, ptx::kFill>(d, dplus(dp, (2 * g) * kPVar + ks * 32), bv,
+                                                 kIdPv, ks == 0 ? acc0 : 1u);
+        ptx::mma_ws_f8_coll<kCollPv, ptx::kLastUse>(d, dplus(dp, (2 * g + 1) * kPVar + ks * 32),
+                                                    bv, kIdPv, 1u);
       }
+      F8_TRACE(14, 4 * tau + g);
     }
     ptx::mma_commit(&c.p_empty);
     ptx::mma_commit(&c.code_empty[cs]);
+    F8_TRACE(10, tau);
     ++uses[cs];
     if (cur.last_of_segment()) {
       ptx::mma_commit(&c.o_full);
@@ -386,109 +430,177 @@ __device__ void pv_role(const PartialParams& p, F8Ctl& c, uint8_t* base, int nse
   }
 }
 
-// Q of each request (128 threads): thread q handles head q / 2 and half the
-// latent (256 values) and rope (32 values).  Writes the hi and lo A operands
-// (64 rows each), the rope A operand and 2^-a per head.
-__device__ void q_role(const PartialParams& p, F8Ctl& c, uint8_t* base, int nseg,
-                       uint32_t& sigma) {
-  const int q = threadIdx.x - kQWarp0 * 32;   // 0..127
-  const int hq = q >> 1, part = q & 1;
+// Q of request b (the 128 staging threads): thread u handles head u / 2 and
+// half the latent (256 values) and rope (32 values).  Writes the hi and lo A
+// operands (64 rows each), the rope A operand and 2^-a per head, once the
+// previous request's score MMAs are done and its softmax read its Q frame.
+__device__ __forceinline__ bool prepare_q(const PartialParams& p, F8Ctl& c, uint8_t* base, int b,
+                          uint32_t sigma) {
+  const int u = threadIdx.x - kStageWarp0 * 32;   // 0..127
+  const int hq = u >> 1, part = u & 1;
   uint8_t* qh = base + kOffQh;
   uint8_t* ql = base + kOffQl;
   uint8_t* qr = base + kOffQr;
-  TileCursor cur;
-  if (!cur.start(p, c, nseg)) return;
-  while (true) {
-    if (sigma > 0 && !wait_or_abort(&c.q_empty, (sigma - 1) & 1, c)) return;
-    const bool live = hq < p.heads;
-    const uint4* src = reinterpret_cast<const uint4*>(
-        p.q + ((size_t)cur.v.b * p.heads + (live ? hq : 0)) * kHeadDim);
-    float amax = 0.f;
+  if (sigma > 0 && !wait_or_abort(&c.q_empty, (sigma - 1) & 1, c)) return false;
+  const bool live = hq < p.heads;
+  const uint4* src =
+      reinterpret_cast<const uint4*>(p.q + ((size_t)b * p.heads + (live ? hq : 0)) * kHeadDim);
+  float amax = 0.f;
 #pragma unroll 4
-    for (int u = 0; u < 32; ++u) {
-      const uint4 v = live ? __ldg(src + part * 32 + u) : make_uint4(0, 0, 0, 0);
+  for (int k = 0; k < 32; ++k) {
+    const uint4 v = live ? __ldg(src + part * 32 + k) : make_uint4(0, 0, 0, 0);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(w[e] << 16)),
+                               fabsf(__uint_as_float(w[e] & 0xFFFF0000u))));
+  }
+  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+  // frame: q * 2^a with max |q * 2^a| in [128, 256)
+  int a = 0;
+  if (amax > 0.f) {
+    const int e = (int)((__float_as_uint(amax) >> 23) & 0xFF) - 127;
+    a = min(120, max(-120, 7 - e));
+  }
+  const float fa = __uint_as_float((uint32_t)(127 + a) << 23);
+  if (part == 0) c.qexp[hq] = __uint_as_float((uint32_t)(127 - a) << 23);
+  // latent: 16 output units of 16 codes (two groups of 128 values) per term
+  // (not unrolled: these warps keep a small register budget)
+#pragma unroll 1
+  for (int uo = 0; uo < 16; ++uo) {
+    const int g = 2 * part + (uo >> 3), un = uo & 7;
+    uint32_t hw[4], lw[4];
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const uint4 v = live ? __ldg(src + part * 32 + 2 * uo + k) : make_uint4(0, 0, 0, 0);
       const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-      for (int e = 0; e < 4; ++e)
-        amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(w[e] << 16)),
-                                 fabsf(__uint_as_float(w[e] & 0xFFFF0000u))));
-    }
-    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-    // frame: q * 2^a with max |q * 2^a| in [128, 256)
-    int a = 0;
-    if (amax > 0.f) {
-      const int e = (int)((__float_as_uint(amax) >> 23) & 0xFF) - 127;
-      a = min(120, max(-120, 7 - e));
-    }
-    const float fa = __uint_as_float((uint32_t)(127 + a) << 23);
-    if (part == 0) c.qexp[hq] = __uint_as_float((uint32_t)(127 - a) << 23);
-    // latent: 16 output units of 16 codes (two groups of 128 values) per term
-#pragma unroll 2
-    for (int uo = 0; uo < 16; ++uo) {
-      const int g = 2 * part + (uo >> 3), u = uo & 7;
-      uint32_t hw[4], lw[4];
-#pragma unroll
-      for (int k = 0; k < 2; ++k) {
-        const uint4 v = live ? __ldg(src + part * 32 + 2 * uo + k) : make_uint4(0, 0, 0, 0);
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int e = 0; e < 4; e += 2) {
-          // four bf16 values -> one word of hi codes and one of lo codes
-          const float f0 = __uint_as_float(w[e] << 16) * fa;
-          const float f1 = __uint_as_float(w[e] & 0xFFFF0000u) * fa;
-          const float f2 = __uint_as_float(w[e + 1] << 16) * fa;
-          const float f3 = __uint_as_float(w[e + 1] & 0xFFFF0000u) * fa;
-          const uint32_t h01 = e4m3x2_f32(f0, f1), h23 = e4m3x2_f32(f2, f3);
-          const float2 b01 = e4m3x2_to_f32(h01), b23 = e4m3x2_to_f32(h23);
-          const uint32_t l01 = e4m3x2_f32(f0 - b01.x, f1 - b01.y);
-          const uint32_t l23 = e4m3x2_f32(f2 - b23.x, f3 - b23.y);
-          hw[2 * k + e / 2] = h01 | (h23 << 16);
-          lw[2 * k + e / 2] = l01 | (l23 << 16);
-        }
+      for (int e = 0; e < 4; e += 2) {
+        // four bf16 values -> one word of hi codes and one of lo codes
+        const float f0 = __uint_as_float(w[e] << 16) * fa;
+        const float f1 = __uint_as_float(w[e] & 0xFFFF0000u) * fa;
+        const float f2 = __uint_as_float(w[e + 1] << 16) * fa;
+        const float f3 = __uint_as_float(w[e + 1] & 0xFFFF0000u) * fa;
+        const uint32_t h01 = e4m3x2_f32(f0, f1), h23 = e4m3x2_f32(f2, f3);
+        const float2 b01 = e4m3x2_to_f32(h01), b23 = e4m3x2_to_f32(h23);
+        const uint32_t l01 = e4m3x2_f32(f0 - b01.x, f1 - b01.y);
+        const uint32_t l23 = e4m3x2_f32(f2 - b23.x, f3 - b23.y);
+        hw[2 * k + e / 2] = h01 | (h23 << 16);
+        lw[2 * k + e / 2] = l01 | (l23 << 16);
       }
-      *reinterpret_cast<uint4*>(qh + g * kChunk + sw128(hq, u)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-      *reinterpret_cast<uint4*>(ql + g * kChunk + sw128(hq, u)) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
     }
-    // rope: 32 bf16 values = 4 units
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const uint4 v = live ? __ldg(src + 64 + part * 4 + u) : make_uint4(0, 0, 0, 0);
-      *reinterpret_cast<uint4*>(qr + sw128(hq, part * 4 + u)) = v;
-    }
-    ptx::fence_proxy_async();
-    ptx::mbar_arrive(&c.q_full);
-    ++sigma;
-    // next segment
-    cur.t = cur.v.ntiles - 1;
-    if (!cur.next(p, c)) break;
+    *reinterpret_cast<uint4*>(qh + g * kChunk + sw128(hq, un)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+    *reinterpret_cast<uint4*>(ql + g * kChunk + sw128(hq, un)) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
   }
+  // rope: 32 bf16 values = 4 units
+#pragma unroll
+  for (int un = 0; un < 4; ++un) {
+    const uint4 v = live ? __ldg(src + 64 + part * 4 + un) : make_uint4(0, 0, 0, 0);
+    *reinterpret_cast<uint4*>(qr + sw128(hq, part * 4 + un)) = v;
+  }
+  ptx::fence_proxy_async();
+  warp_arrive(&c.q_full);
+  return true;
 }
 
-// The scales of one tile, moved into the control block by the softmax
-// threads: [group][row] copies (raw, and times the P normaliser of the
-// current reference scales) and per-warp group maxima over the valid rows.
-// Thread T moves the entry (row T / 4, group T % 4).
-__device__ __forceinline__ void stage_scales(F8Ctl& c, const uint8_t* code, int nv, int buf,
-                                             const float (&sref)[4], int T) {
-  const int stok = T >> 2, sg = T & 3, w = T >> 5, i = T & 31;
-  const float sv = *reinterpret_cast<const float*>(code + kScalesOff + stok * 16 + sg * 4);
-  c.sT[buf][sg][stok] = sv;
-  const float ref = sg == 0 ? sref[0] : sg == 1 ? sref[1] : sg == 2 ? sref[2] : sref[3];
-  reinterpret_cast<uint16_t*>(c.sTp[buf][sg])[stok] =
-      f16_sat(stok < nv ? sv * (kPNorm / ref) : 0.f);
-  float m = stok < nv ? fabsf(sv) : 0.f;
+// Staging (4 warps): per request, its Q; per tile, once its bytes landed,
+// the scales as [group][row] copies (raw, and times kPNorm / S_g as fp16),
+// the reference scales S_g with the O rescale factor a raised reference
+// implies, and zeros over the codes of rows past the request's end (their
+// bytes are whatever the block holds and must not reach PV).  Thread u
+// handles row u / 2, groups 2 (u % 2) and 2 (u % 2) + 1.
+__device__ __forceinline__ void staging_role(const PartialParams& p, F8Ctl& c, uint8_t* base, int nseg,
+                             uint32_t& tau, uint32_t& sigma) {
+  const int u = threadIdx.x - kStageWarp0 * 32;   // 0..127
+  const int sw = u >> 5, lane = u & 31;
+  const int row = u >> 1, gp = (u & 1) * 2;
+  TileCursor cur;
+  if (!cur.start(p, c, nseg)) return;
+  float sref[4] = {1.f, 1.f, 1.f, 1.f};
+  while (true) {
+    const uint32_t cs = tau % kCodeStages;
+    const int b = tau & 1;
+    const bool first = cur.t == 0;
+    if (first) {
+      if (!prepare_q(p, c, base, cur.v.b, sigma)) return;
+      ++sigma;
+    }
+    if (!wait_or_abort(&c.full[cs], (tau / kCodeStages) & 1, c)) return;
+    // buffer b was last read by the softmax of tile tau - 2
+    if (tau >= 2 && !wait_or_abort(&c.sc_empty[b], ((tau / 2) + 1) & 1, c)) return;
+    const int nv = c.nv[cs];
+    uint8_t* code = base + kOffCode + cs * kCodeStage;
+    const float2 sv = *reinterpret_cast<const float2*>(code + kScalesOff + row * 16 + gp * 4);
+    const bool valid = row < nv;
+    float m0 = valid ? fabsf(sv.x) : 0.f, m1 = valid ? fabsf(sv.y) : 0.f;
 #pragma unroll
-  for (int o = 4; o < 32; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-  if (i < 4) c.gpart[buf][w][i] = m;
+    for (int o = 2; o < 32; o <<= 1) {
+      m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, o));
+      m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, o));
+    }
+    if (lane < 2) {
+      c.gw[b][sw][gp] = m0;
+      c.gw[b][sw][gp + 1] = m1;
+    }
+    ptx::named_bar(kBarStage, kStageThreads);
+    float gm[4];
+    {
+      const float4 w0 = *reinterpret_cast<const float4*>(c.gw[b][0]);
+      const float4 w1 = *reinterpret_cast<const float4*>(c.gw[b][1]);
+      const float4 w2 = *reinterpret_cast<const float4*>(c.gw[b][2]);
+      const float4 w3 = *reinterpret_cast<const float4*>(c.gw[b][3]);
+      gm[0] = fmaxf(fmaxf(w0.x, w1.x), fmaxf(w2.x, w3.x));
+      gm[1] = fmaxf(fmaxf(w0.y, w1.y), fmaxf(w2.y, w3.y));
+      gm[2] = fmaxf(fmaxf(w0.z, w1.z), fmaxf(w2.z, w3.z));
+      gm[3] = fmaxf(fmaxf(w0.w, w1.w), fmaxf(w2.w, w3.w));
+    }
+    float r[4] = {1.f, 1.f, 1.f, 1.f};
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      if (first) {
+        sref[g] = gm[g] > 0.f ? gm[g] : 1.f;
+      } else if (gm[g] > kScaleSlack * sref[g]) {
+        r[g] = sref[g] / gm[g];
+        sref[g] = gm[g];
+      }
+    }
+    if (u == 0) {
+      *reinterpret_cast<float4*>(c.sc_r[b]) = make_float4(r[0], r[1], r[2], r[3]);
+      *reinterpret_cast<float4*>(c.sc_ref[b]) = make_float4(sref[0], sref[1], sref[2], sref[3]);
+    }
+    const float ref0 = gp == 0 ? sref[0] : sref[2], ref1 = gp == 0 ? sref[1] : sref[3];
+    c.sT[b][gp][row] = sv.x;
+    c.sT[b][gp + 1][row] = sv.y;
+    reinterpret_cast<uint16_t*>(c.sTp[b][gp])[row] = f16_sat(valid ? sv.x * (kPNorm / ref0) : 0.f);
+    reinterpret_cast<uint16_t*>(c.sTp[b][gp + 1])[row] =
+        f16_sat(valid ? sv.y * (kPNorm / ref1) : 0.f);
+    if (nv < kTileRows) {
+      for (int k = u; k < (kTileRows - nv) * 32; k += kStageThreads) {
+        const int rr = nv + k / 32, g = (k & 31) >> 3, un = k & 7;
+        *reinterpret_cast<uint4*>(code + g * kChunk + sw128(rr, un)) = make_uint4(0, 0, 0, 0);
+      }
+      ptx::fence_proxy_async();
+    }
+    warp_arrive(&c.staged[cs]);
+    ++tau;
+    if (!cur.next(p, c)) break;
+  }
 }
 
 // Softmax, P and the epilogue (8 warps).  Parts and O share the weight-
 // stationary M = 64 layout: TMEM lane L holds head L % 64 for the first
 // (L < 64) or second half of the columns.  Warp w reads lane quarter
 // q = w % 4 and the 16-column half th = w / 4 of each part, so thread (w, i)
-// owns 16 tokens of head h = (32 q + i) % 64.  One named barrier per tile
-// publishes the maxima of this tile and the scales of the next one.
-__device__ void softmax_role(const PartialParams& p, F8Ctl& c, uint8_t* base, int nseg,
+// owns 16 tokens of head h = (32 q + i) % 64.
+//
+// While the tensor core streams its operands, every shared-memory round trip
+// of these threads costs a few hundred cycles, so each tile takes as few as
+// possible: one for its barriers, one for the parts (TMEM) and scales
+// together, one for P.  The running max of a head is shared by its four
+// threads; a barrier-wide vote tells whether any thread's tile maximum
+// exceeds the max in use by more than 2^3, and only then are the maxima
+// exchanged through shared memory.
+__device__ __forceinline__ void softmax_role(const PartialParams& p, F8Ctl& c, uint8_t* base, int nseg,
                              uint32_t& tau, uint32_t& sigma, uint32_t& pi) {
   const int T = threadIdx.x;                 // 0..255
   const int w = T >> 5, i = T & 31;
@@ -501,176 +613,138 @@ __device__ void softmax_role(const PartialParams& p, F8Ctl& c, uint8_t* base, in
   const float sl2 = p.scale * kLog2e;
   const int odh = tq * 64 + th * 32;         // O: this thread's 32 values of each group
 
-  // sparse CTAs whose list is empty write the neutral pair and stop
-  if (p.sparse_idx && seg_view(p, c, 0).ntiles == 0) {
-    const SegView v = seg_view(p, c, 0);
-    const size_t slot = seg_slot(p, v);
-    if (h < p.heads) {
-      float* o = (v.whole ? p.out : p.ws_o) + (slot * p.heads + h) * kVDim;
-      for (int g = 0; g < 4; ++g)
-        for (int e = 0; e < 32; e += 4)
-          *reinterpret_cast<float4*>(o + 128 * g + odh + e) = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (col == 0) (v.whole ? p.out_lse : p.ws_lse)[slot * p.heads + h] = -CUDART_INF_F;
-    }
-    return;
-  }
-
   TileCursor cur;
   if (!cur.start(p, c, nseg)) return;
   float m_used = -CUDART_INF_F, l = 0.f, kq = 0.f, two_a = 1.f;
-  float sref[4] = {1.f, 1.f, 1.f, 1.f};      // reference scales of the current request
   uint8_t* pbuf = base + kOffP;
-  // scales of the batch's first tile
-  {
-    const uint32_t cs = tau % kCodeStages;
-    if (!wait_or_abort(&c.full[cs], (tau / kCodeStages) & 1, c)) return;
-    stage_scales(c, base + kOffCode + cs * kCodeStage, c.nv[cs], tau & 1, sref, T);
-    ptx::named_bar(1, kSoftThreads);
-  }
   while (true) {
     const uint32_t cs = tau % kCodeStages;
-    const int buf = tau & 1;
-    uint8_t* code = base + kOffCode + cs * kCodeStage;
+    const int b = tau & 1;
     const bool first_blk = cur.t == 0;
+    if (T == 0) F8_TRACE(4, tau);
     if (first_blk) {
       if (!wait_or_abort(&c.q_full, sigma & 1, c)) return;
       const float qe = c.qexp[h];
+      warp_arrive(&c.q_empty);               // the Q frame is read
       kq = qe * sl2;
       two_a = 1.f / qe;                      // exact: a power of two
       m_used = -CUDART_INF_F;
       l = 0.f;
     }
+    // ---- the tile's staged scales and its five score parts (side 1's
+    // commit of part 3 and side 0's of part 4 cover all of them)
+    if (!ptx::mbar_wait3(&c.staged[cs], (tau / kCodeStages) & 1, &c.part_full[(pi + 3) % kParts],
+                         ((pi + 3) / kParts) & 1, &c.part_full[(pi + 4) % kParts],
+                         ((pi + 4) / kParts) & 1, &c.abort))
+      return;
+    if (T == 0) F8_TRACE(19, tau);
+    __syncwarp();
+    ptx::tc_fence_after();
     // rows of the tile that take part (none if its table entry is bad: the
-    // producer flagged it and loaded a stand-in block)
+    // producer flagged it and loaded a stand-in block), the group rescale
+    // factors, the reference scales and this thread's 16 token scales; then
+    // the parts in two TMEM loads (registers bound the batch)
     const int nv = c.nv[cs];
-    // ---- reference scales (S_g) of this tile.  The staged P scales were
-    // made with the references of the previous tile: a request's first tile
-    // restages them (one more barrier, once per request); a raised reference
-    // (factor r < 1/4) is applied to P as it is formed.
-    float r[4] = {1.f, 1.f, 1.f, 1.f};
-    bool need_g = false;
+    const float4 rr = *reinterpret_cast<const float4*>(c.sc_r[b]);
+    const float4 sref = *reinterpret_cast<const float4*>(c.sc_ref[b]);
+    float4 s4[4][4];
 #pragma unroll
-    for (int g = 0; g < 4; ++g) {
-      float gm = 0.f;
+    for (int g = 0; g < 4; ++g)
 #pragma unroll
-      for (int k = 0; k < kSoftWarps; ++k) gm = fmaxf(gm, c.gpart[buf][k][g]);
-      if (first_blk) {
-        sref[g] = gm > 0.f ? gm : 1.f;
-      } else if (gm > kScaleSlack * sref[g]) {
-        r[g] = sref[g] / gm;
-        sref[g] = gm;
-        need_g = true;
-      }
-    }
-    if (first_blk) {
-      const int stok = T >> 2, sg = T & 3;
-      const float ref = sg == 0 ? sref[0] : sg == 1 ? sref[1] : sg == 2 ? sref[2] : sref[3];
-      reinterpret_cast<uint16_t*>(c.sTp[buf][sg])[stok] =
-          f16_rn(stok < nv ? c.sT[buf][sg][stok] * (kPNorm / ref) : 0.f);
-      ptx::named_bar(1, kSoftThreads);
-    }
-    // ---- score parts: 16 tokens of head h.  The loads of a batch of parts
-    // (0-2, then 3-4) are issued back to back and waited for once.
+      for (int j = 0; j < 4; ++j) s4[g][j] = reinterpret_cast<const float4*>(&c.sT[b][g][tok0])[j];
     float x[16];
     {
       uint32_t xa[3][16];
 #pragma unroll
-      for (int part = 0; part < 3; ++part) {
-        const uint32_t bp = (pi + part) % kParts;
-        if (!wait_or_abort(&c.part_full[bp], ((pi + part) / kParts) & 1, c)) return;
-        __syncwarp();
-        ptx::tc_fence_after();
-        ptx::tmem_ld16(lane_base + kColPart + 32 * bp + 16 * th, xa[part]);
-      }
+      for (int part = 0; part < 3; ++part)
+        ptx::tmem_ld16(lane_base + kColPart + 32 * ((pi + part) % kParts) + 16 * th, xa[part]);
       ptx::tmem_wait_ld();
-      ptx::tc_fence_before();
+      if (T == 0) F8_TRACE(16, tau);
 #pragma unroll
-      for (int part = 0; part < 3; ++part) ptx::mbar_arrive(&c.part_empty[(pi + part) % kParts]);
+      for (int j = 0; j < 4; ++j) {
 #pragma unroll
-      for (int g = 0; g < 3; ++g) {
-        const float4* s4 = reinterpret_cast<const float4*>(&c.sT[buf][g][tok0]);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const float4 s = s4[j];
-          const float a0 = __uint_as_float(xa[g][4 * j]), a1 = __uint_as_float(xa[g][4 * j + 1]);
-          const float a2 = __uint_as_float(xa[g][4 * j + 2]), a3 = __uint_as_float(xa[g][4 * j + 3]);
-          x[4 * j] = g == 0 ? s.x * a0 : fmaf(s.x, a0, x[4 * j]);
-          x[4 * j + 1] = g == 0 ? s.y * a1 : fmaf(s.y, a1, x[4 * j + 1]);
-          x[4 * j + 2] = g == 0 ? s.z * a2 : fmaf(s.z, a2, x[4 * j + 2]);
-          x[4 * j + 3] = g == 0 ? s.w * a3 : fmaf(s.w, a3, x[4 * j + 3]);
+        for (int e = 0; e < 4; ++e) {
+          const int k = 4 * j + e;
+          const float s0 = e == 0 ? s4[0][j].x : e == 1 ? s4[0][j].y : e == 2 ? s4[0][j].z : s4[0][j].w;
+          const float s1 = e == 0 ? s4[1][j].x : e == 1 ? s4[1][j].y : e == 2 ? s4[1][j].z : s4[1][j].w;
+          const float s2 = e == 0 ? s4[2][j].x : e == 1 ? s4[2][j].y : e == 2 ? s4[2][j].z : s4[2][j].w;
+          float v = s0 * __uint_as_float(xa[0][k]);
+          v = fmaf(s1, __uint_as_float(xa[1][k]), v);
+          x[k] = fmaf(s2, __uint_as_float(xa[2][k]), v);
         }
       }
     }
     {
       uint32_t xb[2][16];
 #pragma unroll
-      for (int part = 3; part < 5; ++part) {
-        const uint32_t bp = (pi + part) % kParts;
-        if (!wait_or_abort(&c.part_full[bp], ((pi + part) / kParts) & 1, c)) return;
-        __syncwarp();
-        ptx::tc_fence_after();
-        ptx::tmem_ld16(lane_base + kColPart + 32 * bp + 16 * th, xb[part - 3]);
-      }
+      for (int part = 3; part < 5; ++part)
+        ptx::tmem_ld16(lane_base + kColPart + 32 * ((pi + part) % kParts) + 16 * th,
+                       xb[part - 3]);
       ptx::tmem_wait_ld();
       ptx::tc_fence_before();
+      __syncwarp();
+      if (i == 0)
 #pragma unroll
-      for (int part = 3; part < 5; ++part) ptx::mbar_arrive(&c.part_empty[(pi + part) % kParts]);
-      const float4* s4 = reinterpret_cast<const float4*>(&c.sT[buf][3][tok0]);
+        for (int part = 0; part < 5; ++part) ptx::mbar_arrive(&c.part_empty[(pi + part) % kParts]);
+      // x = sum_g s_g part_g + 2^a rope (times 2^-a scale log2(e) below)
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const float4 s = s4[j];
-        x[4 * j] = fmaf(s.x, __uint_as_float(xb[0][4 * j]), x[4 * j]);
-        x[4 * j + 1] = fmaf(s.y, __uint_as_float(xb[0][4 * j + 1]), x[4 * j + 1]);
-        x[4 * j + 2] = fmaf(s.z, __uint_as_float(xb[0][4 * j + 2]), x[4 * j + 2]);
-        x[4 * j + 3] = fmaf(s.w, __uint_as_float(xb[0][4 * j + 3]), x[4 * j + 3]);
-      }
-      // rope, brought into the Q frame: the sum is multiplied by 2^-a * scale below
 #pragma unroll
-      for (int j = 0; j < 16; ++j) x[j] = fmaf(__uint_as_float(xb[1][j]), two_a, x[j]);
+        for (int e = 0; e < 4; ++e) {
+          const int k = 4 * j + e;
+          const float s3 = e == 0 ? s4[3][j].x : e == 1 ? s4[3][j].y : e == 2 ? s4[3][j].z : s4[3][j].w;
+          const float v = fmaf(s3, __uint_as_float(xb[0][k]), x[k]);
+          x[k] = fmaf(__uint_as_float(xb[1][k]), two_a, v);
+        }
+      }
     }
     pi += 5;
+    const bool need_g = !first_blk && (rr.x != 1.f || rr.y != 1.f || rr.z != 1.f || rr.w != 1.f);
+    // the P factors of this thread's tokens (consumed after the exponentials)
+    uint4 sp[4][2];
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      sp[g][0] = *reinterpret_cast<const uint4*>(&c.sTp[b][g][tok0]);
+      sp[g][1] = *reinterpret_cast<const uint4*>(&c.sTp[b][g][tok0 + 8]);
+    }
     float mloc = -CUDART_INF_F;
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
       x[j] = (tok0 + j < nv) ? x[j] * kq : -CUDART_INF_F;
       mloc = fmaxf(mloc, x[j]);
     }
-    c.mred[col][h] = mloc;
-    // ---- the next tile's scales, published by the barrier below
-    {
-      TileCursor nx = cur;
-      if (nx.next(p, c)) {
-        const uint32_t ns = (tau + 1) % kCodeStages;
-        if (!wait_or_abort(&c.full[ns], ((tau + 1) / kCodeStages) & 1, c)) return;
-        stage_scales(c, base + kOffCode + ns * kCodeStage, c.nv[ns], buf ^ 1, sref, T);
+    if (T == 0) F8_TRACE(5, tau);
+    // ---- lazy max, per head.  The vote is a barrier without shared-memory
+    // traffic; the exchange runs only if some thread needs a larger max.
+    const bool grow = mloc > m_used + kRescaleLog2;
+    float alpha = 1.f;
+    if (ptx::named_bar_or(kBarSoft, kSoftThreads, grow)) {
+      float (*mr)[64] = c.mred[b];
+      mr[col][h] = mloc;
+      ptx::named_bar(kBarSoft, kSoftThreads);
+      const float mt = fmaxf(fmaxf(mr[0][h], mr[1][h]), fmaxf(mr[2][h], mr[3][h]));
+      if (first_blk) {
+        m_used = mt;
+      } else if (mt > m_used + kRescaleLog2) {
+        alpha = m_used == -CUDART_INF_F ? 0.f : ex2(m_used - mt);
+        m_used = mt;
       }
     }
-    // ---- lazy rescale of O (running max grew by > 2^3, or a group's scale
-    // reference was raised); decided for the whole CTA
-    const bool grow = !first_blk && mloc > m_used + kRescaleLog2;
-    const bool any = ptx::named_bar_or(1, kSoftThreads, grow || need_g);
-    const float mt = fmaxf(fmaxf(c.mred[0][h], c.mred[1][h]), fmaxf(c.mred[2][h], c.mred[3][h]));
-    float m_new = m_used;
-    if (first_blk) {
-      m_used = mt;
-      m_new = mt;
-    } else if (mt > m_used + kRescaleLog2) {
-      m_new = mt;
-    }
+    if (T == 0) F8_TRACE(6, tau);
+    l *= alpha;
     bool waited_pv = false;
-    if (any) {
-      const float alpha = (m_new == m_used) ? 1.f
-                          : (m_used == -CUDART_INF_F ? 0.f : ex2(m_used - m_new));
-      l *= alpha;
-      m_used = m_new;
-      // the previous tile's PV must have landed in O before it is rescaled
+    if (__any_sync(0xffffffffu, alpha != 1.f || need_g)) {
+      // O of the previous tiles is rescaled once the previous PV has landed;
+      // a raised group reference scales its O by r_g as well
       if (!wait_or_abort(&c.p_empty, (tau - 1) & 1, c)) return;
       waited_pv = true;
+      if (T == 0) F8_TRACE(11, tau);
       __syncwarp();
       ptx::tc_fence_after();
-#pragma unroll
+#pragma unroll 1
       for (int g = 0; g < 4; ++g) {
-        const float f = alpha * r[g];
+        const float rg = g == 0 ? rr.x : g == 1 ? rr.y : g == 2 ? rr.z : rr.w;
+        const float f = need_g ? alpha * rg : alpha;
         uint32_t v[32];
         const uint32_t addr = lane_base + 64 * g + 32 * th;
         ptx::tmem_ld32(addr, v);
@@ -688,65 +762,56 @@ __device__ void softmax_role(const PartialParams& p, F8Ctl& c, uint8_t* base, in
     uint32_t pp[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      const float a = ex2(x[2 * j] - mu), b = ex2(x[2 * j + 1] - mu);
-      sum += a + b;
-      pp[j] = f16x2_rn(a, b);
+      const float a = ex2(x[2 * j] - mu), bb = ex2(x[2 * j + 1] - mu);
+      sum += a + bb;
+      pp[j] = f16x2_rn(a, bb);
     }
     l += sum;
-    // ---- P (and the tile's invalid rows) may be written once the previous PV is done
+    // ---- P may be written once the previous PV is done with it
     if (!waited_pv && tau > 0 && !wait_or_abort(&c.p_empty, (tau - 1) & 1, c)) return;
-    if (nv < kTileRows) {
-      // rows past the end must not reach PV (their bytes are whatever the
-      // block holds): zero their codes
-      for (int k = T; k < (kTileRows - nv) * 32; k += kSoftThreads) {
-        const int row = nv + k / 32, g = (k & 31) >> 3, u = k & 7;
-        *reinterpret_cast<uint4*>(code + g * kChunk + sw128(row, u)) = make_uint4(0, 0, 0, 0);
-      }
-    }
+    if (T == 0) F8_TRACE(7, tau);
     const int unit = tok0 >> 4;              // my 16 tokens: one 16-byte unit of a P row
 #pragma unroll
     for (int g = 0; g < 4; ++g) {
-      const uint4 sa = *reinterpret_cast<const uint4*>(&c.sTp[buf][g][tok0]);
-      const uint4 sb = *reinterpret_cast<const uint4*>(&c.sTp[buf][g][tok0 + 8]);
-      uint32_t sw[8] = {sa.x, sa.y, sa.z, sa.w, sb.x, sb.y, sb.z, sb.w};
-      if (need_g) {
-        const uint32_t f2 = f16x2_rn(r[g], r[g]);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) sw[j] = hmul2_rn(sw[j], f2);
-      }
+      const uint32_t swv[8] = {sp[g][0].x, sp[g][0].y, sp[g][0].z, sp[g][0].w,
+                               sp[g][1].x, sp[g][1].y, sp[g][1].z, sp[g][1].w};
       uint32_t hw[4], lw[4];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        uint32_t h0, l0, h1, l1;
-        split_hilo(hmul2_rn(pp[2 * j], sw[2 * j]), h0, l0);
-        split_hilo(hmul2_rn(pp[2 * j + 1], sw[2 * j + 1]), h1, l1);
-        hw[j] = h0 | (h1 << 16);
-        lw[j] = l0 | (l1 << 16);
-      }
+      for (int j = 0; j < 4; ++j)
+        split_hilo4(hmul2_rn(pp[2 * j], swv[2 * j]), hmul2_rn(pp[2 * j + 1], swv[2 * j + 1]),
+                    hw[j], lw[j]);
       *reinterpret_cast<uint4*>(pbuf + (2 * g) * kPVar + sw64(h, unit)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
       *reinterpret_cast<uint4*>(pbuf + (2 * g + 1) * kPVar + sw64(h, unit)) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
     }
     ptx::fence_proxy_async();
-    ptx::mbar_arrive(&c.p_full);
+    __syncwarp();
+    if (i == 0) {
+      ptx::mbar_arrive(&c.p_full);
+      ptx::mbar_arrive(&c.sc_empty[b]);
+    }
+    if (T == 0) F8_TRACE(8, tau);
     // ---- epilogue after the request's last tile
     if (cur.last_of_segment()) {
       const SegView& v = cur.v;
       const size_t slot = seg_slot(p, v);
-      c.mred[col][h] = l;
+      // the other parity's maxima were read before this tile's vote
+      float (*ls)[64] = c.mred[b ^ 1];
+      ls[col][h] = l;
       // o_full completes once per request, after its last PV
       if (!wait_or_abort(&c.o_full, sigma & 1, c)) return;
-      ptx::named_bar(1, kSoftThreads);
+      ptx::named_bar(kBarSoft, kSoftThreads);
       __syncwarp();
       ptx::tc_fence_after();
-      const float ltot = (c.mred[0][h] + c.mred[1][h]) + (c.mred[2][h] + c.mred[3][h]);
+      const float ltot = (ls[0][h] + ls[1][h]) + (ls[2][h] + ls[3][h]);
       if (col == 0 && h < p.heads)
         (v.whole ? p.out_lse : p.ws_lse)[slot * p.heads + h] =
             ltot > 0.f ? (m_used + log2f(ltot)) * kLn2 : -CUDART_INF_F;
       const float il = ltot > 0.f ? 1.f / ltot : 0.f;
       float* o_base = (v.whole ? p.out : p.ws_o) + (slot * p.heads + h) * kVDim + odh;
-#pragma unroll
+#pragma unroll 1
       for (int g = 0; g < 4; ++g) {
-        const float f = il * (sref[g] / kPNorm);
+        const float sg = g == 0 ? sref.x : g == 1 ? sref.y : g == 2 ? sref.z : sref.w;
+        const float f = il * (sg * (1.f / kPNorm));
         uint32_t v32[32];
         ptx::tmem_ld32(lane_base + 64 * g + 32 * th, v32);
         ptx::tmem_wait_ld();
@@ -760,7 +825,7 @@ __device__ void softmax_role(const PartialParams& p, F8Ctl& c, uint8_t* base, in
         }
       }
       ptx::tc_fence_before();
-      ptx::named_bar(1, kSoftThreads);
+      ptx::named_bar(kBarSoft, kSoftThreads);
       ++sigma;
     }
     ++tau;
@@ -768,10 +833,84 @@ __device__ void softmax_role(const PartialParams& p, F8Ctl& c, uint8_t* base, in
   }
 }
 
-template <bool kSparse>
+// Barrier over the whole block, written out so that the two warpgroup
+// branches below (which never rejoin until the end) can both use it.
+__device__ __forceinline__ void block_bar() { ptx::named_bar(kBarBlock, kThreads); }
+
+// The batch loop of one side of the register split: kSoft runs the softmax
+// warps, !kSoft every other role and, at the end, the drains of the
+// asynchronous arrivals.  Both sides take the same block barriers.
+template <bool kSoft>
+__device__ __forceinline__ void run_roles(const F8Params& P, const PartialParams& p, F8Ctl& c,
+                                          uint8_t* base, int lo, int hi) {
+  const int warp = threadIdx.x >> 5;
+  uint32_t tau = 0, sigma = 0, pi = 0, o_commits = 0;
+  uint32_t uses[kCodeStages] = {0, 0, 0}, fills[kCodeStages] = {0, 0, 0};
+  int first = 0;
+  while (true) {
+    // the control block holds kMaxSegF8 segments: collect them in batches
+    const int total = lo < hi ? collect_segments_n(p, lo, hi, first, kMaxSegF8, c) : 0;
+    const int nseg = min(kMaxSegF8, total - first);
+    if (nseg <= 0) break;
+    if constexpr (kSoft) {
+      softmax_role(p, c, base, nseg, tau, sigma, pi);
+    } else {
+      if (warp == kProdWarp) {
+        if ((threadIdx.x & 31) == 0) producer_role(P, p, c, base, nseg, tau, fills);
+      } else if (warp == kQkWarp || warp == kQkWarp2) {
+        if ((threadIdx.x & 31) == 0) qk_role(warp == kQkWarp ? 0 : 1, p, c, base, nseg, tau, sigma);
+      } else if (warp == kPvWarp) {
+        if ((threadIdx.x & 31) == 0) pv_role(p, c, base, nseg, tau, uses, o_commits);
+      } else {
+        staging_role(p, c, base, nseg, tau, sigma);
+      }
+    }
+    block_bar();
+    if (c.abort) break;
+    first += kMaxSegF8;
+    if (total <= first) break;
+  }
+  if constexpr (!kSoft) {
+    // Drain: every asynchronous arrival must land before the CTA exits (it
+    // could otherwise hit the next CTA's barriers at the same addresses).
+    // Normally only the last slot, P and Q releases are unconsumed; after a
+    // timeout any commit or TMA fill may be.  Each wait is for the latest
+    // phase of its barrier, so the parity is unambiguous.
+    if (threadIdx.x == kPvWarp * 32) {
+      uint32_t n = 0;
+      for (int s = 0; s < kCodeStages; ++s) {
+        if (uses[s] > 0) wait_or_abort(&c.code_empty[s], (uses[s] - 1) & 1, c);
+        n += uses[s];
+      }
+      if (n > 0) wait_or_abort(&c.p_empty, (n - 1) & 1, c);
+      if (o_commits > 0) wait_or_abort(&c.o_full, (o_commits - 1) & 1, c);
+    }
+    if (threadIdx.x == kQkWarp * 32 || threadIdx.x == kQkWarp2 * 32) {
+      // tau counts the tiles this issuer handled; parts 5 tau of them,
+      // commits on buffer k for every part number below 5 tau congruent to k
+      if (sigma > 0) wait_or_abort(&c.q_empty, (sigma - 1) & 1, c);
+      if (threadIdx.x == kQkWarp * 32)
+        for (uint32_t s = 0; s < (uint32_t)kRopeStages; ++s) {
+          const uint32_t n = tau > s ? (tau - s + kRopeStages - 1) / kRopeStages : 0;
+          if (n > 0) wait_or_abort(&c.rope_empty[s], (n - 1) & 1, c);
+        }
+      const uint32_t parts = 5 * tau;
+      for (uint32_t k = 0; k < (uint32_t)kParts; ++k) {
+        const uint32_t n = parts > k ? (parts - k + kParts - 1) / kParts : 0;
+        if (n > 0) wait_or_abort(&c.part_full[k], (n - 1) & 1, c);
+      }
+    }
+    if (threadIdx.x == kProdWarp * 32)
+      for (int s = 0; s < kCodeStages; ++s)
+        if (fills[s] > 0) wait_or_abort(&c.full[s], (fills[s] - 1) & 1, c);
+  }
+}
+
 __global__ void __launch_bounds__(kThreads, 1) partial_f8_kernel(const __grid_constant__ F8Params P) {
+  // dense only: a known-null index list lets the compiler drop the sparse
+  // branches of the shared schedule
   PartialParams p = P.p;
-  if constexpr (!kSparse) p.sparse_idx = nullptr;
+  p.sparse_idx = nullptr;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -781,18 +920,21 @@ __global__ void __launch_bounds__(kThreads, 1) partial_f8_kernel(const __grid_co
   if (threadIdx.x == 0) {
     for (int s = 0; s < kCodeStages; ++s) {
       ptx::mbar_init(&c.full[s], 1);
+      ptx::mbar_init(&c.staged[s], kStageThreads / 32);
       ptx::mbar_init(&c.code_empty[s], 1);
     }
     for (int s = 0; s < kRopeStages; ++s) ptx::mbar_init(&c.rope_empty[s], 1);
     for (int k = 0; k < kParts; ++k) {
       ptx::mbar_init(&c.part_full[k], 1);
-      ptx::mbar_init(&c.part_empty[k], kSoftThreads);
+      ptx::mbar_init(&c.part_empty[k], kSoftWarps);
     }
-    ptx::mbar_init(&c.p_full, kSoftThreads);
+    for (int s = 0; s < 2; ++s) ptx::mbar_init(&c.sc_empty[s], kSoftWarps);
+    ptx::mbar_init(&c.p_full, kSoftWarps);
     ptx::mbar_init(&c.p_empty, 1);
     ptx::mbar_init(&c.o_full, 1);
-    ptx::mbar_init(&c.q_full, kQThreads);
-    ptx::mbar_init(&c.q_empty, 2);        // one commit from each score issuer
+    ptx::mbar_init(&c.q_full, kStageThreads / 32);
+    // one commit from each score issuer, one arrival per softmax warp
+    ptx::mbar_init(&c.q_empty, 2 + kSoftWarps);
     c.abort = 0;
     ptx::fence_mbar_init();
   }
@@ -803,7 +945,7 @@ __global__ void __launch_bounds__(kThreads, 1) partial_f8_kernel(const __grid_co
   ptx::tc_fence_after();
 
   int lo = 0, hi = 0;
-  if (!p.sparse_idx) {
+  {
     const int T = total_tiles(p, c.warp_sums);
     const int tpc = T > 0 ? (T + p.num_ctas - 1) / p.num_ctas : 0;
     lo = blockIdx.x * tpc;
@@ -811,72 +953,21 @@ __global__ void __launch_bounds__(kThreads, 1) partial_f8_kernel(const __grid_co
   }
   __syncthreads();
 
-  uint32_t tau = 0, sigma = 0, pi = 0, o_commits = 0;
-  uint32_t uses[kCodeStages] = {0, 0, 0}, fills[kCodeStages] = {0, 0, 0};
-  int first = 0;
-  while (true) {
-    int nseg, total;
-    if (p.sparse_idx) {
-      nseg = total = 1;
-    } else {
-      // the control block holds kMaxSegF8 segments: collect them in batches
-      total = lo < hi ? collect_segments_n(p, lo, hi, first, kMaxSegF8, c) : 0;
-      nseg = min(kMaxSegF8, total - first);
-    }
-    if (nseg <= 0) break;
-    if (warp < kSoftWarps) {
-      softmax_role(p, c, base, nseg, tau, sigma, pi);
-    } else if (warp == kProdWarp) {
-      if ((threadIdx.x & 31) == 0) producer_role(P, p, c, base, nseg, tau, fills);
-    } else if (warp == kQkWarp) {
-      if ((threadIdx.x & 31) == 0) qk_role<0>(p, c, base, nseg, tau, sigma);
-    } else if (warp == kQkWarp2) {
-      if ((threadIdx.x & 31) == 0) qk_role<1>(p, c, base, nseg, tau, sigma);
-    } else if (warp == kPvWarp) {
-      if ((threadIdx.x & 31) == 0) pv_role(p, c, base, nseg, tau, uses, o_commits);
-    } else {
-      q_role(p, c, base, nseg, sigma);
-    }
-    __syncthreads();
-    if (c.abort) break;
-    first += kMaxSegF8;
-    if (p.sparse_idx || total <= first) break;
+  // Register split: the launch gives every thread kLaunchRegs registers
+  // (65,536 in all); the two softmax warpgroups take kSoftRegs and the two
+  // others keep kOtherRegs.  Every warpgroup executes its adjustment here,
+  // before any role can return, and the two branches stay apart until the
+  // end so that each is compiled within its own budget.
+  if (warp < kSoftWarps) {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftRegs));
+    run_roles<true>(P, p, c, base, lo, hi);
+  } else {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kOtherRegs));
+    run_roles<false>(P, p, c, base, lo, hi);
   }
-  // Drain: every asynchronous arrival must land before the CTA exits (it
-  // could otherwise hit the next CTA's barriers at the same addresses).
-  // Normally only the last slot, P and Q releases are unconsumed; after a
-  // timeout any commit or TMA fill may be.  Each wait is for the latest phase
-  // of its barrier, so the parity is unambiguous.
-  if (threadIdx.x == kPvWarp * 32) {
-    uint32_t n = 0;
-    for (int s = 0; s < kCodeStages; ++s) {
-      if (uses[s] > 0) wait_or_abort(&c.code_empty[s], (uses[s] - 1) & 1, c);
-      n += uses[s];
-    }
-    if (n > 0) wait_or_abort(&c.p_empty, (n - 1) & 1, c);
-    if (o_commits > 0) wait_or_abort(&c.o_full, (o_commits - 1) & 1, c);
-  }
-  if (threadIdx.x == kQkWarp * 32 || threadIdx.x == kQkWarp2 * 32) {
-    // tau counts the tiles this issuer handled; parts 5 tau of them, commits
-    // on buffer k for every part number below 5 tau congruent to k
-    if (sigma > 0) wait_or_abort(&c.q_empty, (sigma - 1) & 1, c);
-    if (threadIdx.x == kQkWarp * 32)
-      for (uint32_t s = 0; s < (uint32_t)kRopeStages; ++s) {
-        const uint32_t n = tau > s ? (tau - s + kRopeStages - 1) / kRopeStages : 0;
-        if (n > 0) wait_or_abort(&c.rope_empty[s], (n - 1) & 1, c);
-      }
-    const uint32_t parts = 5 * tau;
-    for (uint32_t k = 0; k < (uint32_t)kParts; ++k) {
-      const uint32_t n = parts > k ? (parts - k + kParts - 1) / kParts : 0;
-      if (n > 0) wait_or_abort(&c.part_full[k], (n - 1) & 1, c);
-    }
-  }
-  if (threadIdx.x == kProdWarp * 32)
-    for (int s = 0; s < kCodeStages; ++s)
-      if (fills[s] > 0) wait_or_abort(&c.full[s], (fills[s] - 1) & 1, c);
   if (c.abort && threadIdx.x == 0 && p.flags) atomicOr(p.flags, kFlagTimeout);
   ptx::tc_fence_before();
-  __syncthreads();
+  block_bar();
   ptx::tc_fence_after();
   if (warp == 0) ptx::tmem_dealloc(c.tmem_base, kTmemCols);
 }
@@ -946,14 +1037,28 @@ cudaError_t launch_partial_f8(const PartialParams& p, cudaStream_t st) {
     // (including ones captured into a CUDA graph) are plain launches
     std::lock_guard<std::mutex> lock(g_attr_mutex);
     if (!g_attr_done[dev]) {
-      e = cudaFuncSetAttribute(partial_f8_kernel<false>,
+      // the in-kernel register split assumes exactly kLaunchRegs registers
+      // per thread at launch; with fewer, the softmax warpgroups' increase
+      // could never be granted
+      cudaFuncAttributes fa;
+      e = cudaFuncGetAttributes(&fa, partial_f8_kernel);
+      if (e != cudaSuccess) return e;
+      if (fa.numRegs != kLaunchRegs || fa.maxThreadsPerBlock < kThreads)
+        return cudaErrorInvalidDeviceFunction;
+      e = cudaFuncSetAttribute(partial_f8_kernel,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
       if (e != cudaSuccess) return e;
       g_attr_done[dev] = true;
     }
   }
-  partial_f8_kernel<false><<<p.num_ctas, kThreads, smem, st>>>(fp);
+  partial_f8_kernel<<<p.num_ctas, kThreads, smem, st>>>(fp);
   return cudaGetLastError();
 }
 
 }  // namespace dcpmla
+
+#ifdef DCPMLA_F8_TRACE
+extern "C" int f8_trace_read(long long* host) {
+  return (int)cudaMemcpyFromSymbol(host, dcpmla::g_f8_trace, sizeof(long long) * 24 * 256);
+}
+#endif

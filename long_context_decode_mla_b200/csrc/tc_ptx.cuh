@@ -1,6 +1,7 @@
-// Thin inline-PTX wrappers for the sm_100a features the tensor-core kernel
-// uses: mbarriers, cp.async, tcgen05 (TMEM allocation, MMA, commit, loads
-// and stores) and shared-memory matrix descriptors.  Every wait is bounded:
+// Thin inline-PTX wrappers for the sm_100a features the tensor-core kernels
+// use: mbarriers, cp.async and TMA tensor loads, tcgen05 (TMEM allocation,
+// MMA, collector buffers, commit, loads and stores) and shared-memory matrix
+// descriptors.  Every wait is bounded:
 // it gives up after a clock budget and reports failure to the caller.
 #pragma once
 
@@ -70,6 +71,37 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
       return false;
     }
   }
+}
+
+// Tests three phases with one shared-memory round trip (the three tests are
+// issued back to back; while the tensor core streams its operands a single
+// round trip of the load/store unit costs a few hundred cycles).  Returns a
+// bit mask of the completed ones (bit k for barrier k).
+__device__ __forceinline__ uint32_t mbar_test3(uint64_t* b0, uint32_t p0, uint64_t* b1,
+                                               uint32_t p1, uint64_t* b2, uint32_t p2) {
+  uint32_t m;
+  asm volatile(
+      "{\n .reg .pred q0, q1, q2;\n .reg .b32 t0, t1, t2;\n"
+      " mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 q0, [%1], %2;\n"
+      " mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 q1, [%3], %4;\n"
+      " mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 q2, [%5], %6;\n"
+      " selp.b32 t0, 1, 0, q0;\n selp.b32 t1, 2, 0, q1;\n selp.b32 t2, 4, 0, q2;\n"
+      " or.b32 t0, t0, t1;\n or.b32 %0, t0, t2;\n}\n"
+      : "=r"(m)
+      : "r"(smem_addr(b0)), "r"(p0), "r"(smem_addr(b1)), "r"(p1), "r"(smem_addr(b2)), "r"(p2)
+      : "memory");
+  return m;
+}
+
+// mbar_wait for three phases at once (any of them may repeat a barrier).
+__device__ __forceinline__ bool mbar_wait3(uint64_t* b0, uint32_t p0, uint64_t* b1, uint32_t p1,
+                                           uint64_t* b2, uint32_t p2, volatile int* abort) {
+  const uint32_t m = mbar_test3(b0, p0, b1, p1, b2, p2);
+  if (m == 7u) return true;
+  if (!(m & 1u) && !mbar_wait(b0, p0, abort)) return false;
+  if (!(m & 2u) && !mbar_wait(b1, p1, abort)) return false;
+  if (!(m & 4u) && !mbar_wait(b2, p2, abort)) return false;
+  return true;
 }
 
 // ------------------------------------------------------------- cp.async ----
@@ -184,6 +216,45 @@ __device__ __forceinline__ void mma_ws_f8(uint32_t d_tmem, uint64_t a_desc, uint
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+
+// Weight-stationary MMAs that keep the B operand in one of the tensor
+// core's four collector buffers: kFill reads B from shared memory and keeps
+// it, kUse / kLastUse read the kept copy (kLastUse releases it) instead of
+// shared memory.  The B descriptor passed with kUse / kLastUse must describe
+// the same operand that was filled.  Two consecutive MMAs that share B (the
+// hi and lo terms of one product) then read it from shared memory once.
+enum CollectorOp { kFill = 0, kUse = 1, kLastUse = 2 };
+
+#define DCPMLA_MMA_WS_COLL(KIND, BUF, OP)                                                  \
+  asm volatile("{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"                              \
+               " tcgen05.mma.ws.cta_group::1.kind::" KIND ".collector::b" #BUF "::" OP  \
+               " [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),                               \
+               "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)                     \
+               : "memory")
+
+template <int kBuf, int kOp>
+__device__ __forceinline__ void mma_ws_f8_coll(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                               uint32_t idesc, uint32_t accumulate) {
+  static_assert(kBuf >= 0 && kBuf < 4, "collector buffers b0..b3");
+  if constexpr (kBuf == 0) {
+    if constexpr (kOp == kFill) DCPMLA_MMA_WS_COLL("f8f6f4", 0, "fill");
+    else if constexpr (kOp == kUse) DCPMLA_MMA_WS_COLL("f8f6f4", 0, "use");
+    else DCPMLA_MMA_WS_COLL("f8f6f4", 0, "lastuse");
+  } else if constexpr (kBuf == 1) {
+    if constexpr (kOp == kFill) DCPMLA_MMA_WS_COLL("f8f6f4", 1, "fill");
+    else if constexpr (kOp == kUse) DCPMLA_MMA_WS_COLL("f8f6f4", 1, "use");
+    else DCPMLA_MMA_WS_COLL("f8f6f4", 1, "lastuse");
+  } else if constexpr (kBuf == 2) {
+    if constexpr (kOp == kFill) DCPMLA_MMA_WS_COLL("f8f6f4", 2, "fill");
+    else if constexpr (kOp == kUse) DCPMLA_MMA_WS_COLL("f8f6f4", 2, "use");
+    else DCPMLA_MMA_WS_COLL("f8f6f4", 2, "lastuse");
+  } else {
+    if constexpr (kOp == kFill) DCPMLA_MMA_WS_COLL("f8f6f4", 3, "fill");
+    else if constexpr (kOp == kUse) DCPMLA_MMA_WS_COLL("f8f6f4", 3, "use");
+    else DCPMLA_MMA_WS_COLL("f8f6f4", 3, "lastuse");
+  }
+}
+#undef DCPMLA_MMA_WS_COLL
 
 // cta_group::1 kind::f16 (non weight-stationary), used with bf16 operands.
 __device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
