@@ -103,7 +103,9 @@ extern "C" {
 /*
  * Bytes of workspace that mla_decode_partial needs for these sizes.
  *
- *   batch, num_heads: as passed to mla_decode_partial.
+ *   batch, num_heads: as passed to mla_decode_partial (for
+ *               mla_decode_partial_multi, num_heads * q_len; up to
+ *               DCPMLA_MAX_HEADS * 64 rows, else DCPMLA_ERR_UNSUPPORTED).
  *   num_splits: as passed to mla_decode_partial (0 = automatic, which uses
  *               the SM count of the current device).
  *   topk: length of each sparse index list, 0 for dense decode.
@@ -163,14 +165,22 @@ int mla_decode_partial(const void* q, const void* kv_cache, int kv_dtype, int64_
  * position L_b - q_len + i and attends to every cached t <= that position.
  *
  *   q            [batch][q_len][num_heads][576] bf16 (16-byte aligned).
- *   num_heads    query heads per token; num_heads * q_len <= 64 (the rows of
- *                the tensor-core tile), else DCPMLA_ERR_UNSUPPORTED.
+ *   num_heads    query heads per token, 1..64 (else DCPMLA_ERR_UNSUPPORTED);
+ *                q_len 1..64 (else DCPMLA_ERR_INVALID_ARGUMENT).  The rows
+ *                (query, head) run in passes over the cache, each pass one
+ *                tile of at most 64 rows and whole queries: with an fp8 cache
+ *                (exact e4m3 kernel) and with DCPMLA_IMPL_SIMT one query per
+ *                pass, otherwise as many queries as fit 64 rows.  A pass over
+ *                queries [k, k + n) attends over the cache less its last
+ *                q_len - k - n tokens; each pass reads that part of the
+ *                cache again, so q_len passes read about q_len times the
+ *                bytes of one decode.
  *   out_partial  [batch][q_len][num_heads][512] fp32; out_lse
  *                [batch][q_len][num_heads] fp32; queries that see no token of
  *                this shard give (0, -inf).
  *   workspace    mla_decode_workspace_size(batch, num_heads * q_len, ...).
- *   impl         DCPMLA_IMPL_AUTO or DCPMLA_IMPL_TC (the CUDA-core kernel has
- *                no causal rows: DCPMLA_ERR_UNSUPPORTED when q_len > 1).
+ *   impl         any DCPMLA_IMPL_* (the CUDA-core kernel runs one query per
+ *                pass).
  * Other arguments as in mla_decode_partial (no sparse variant).  The merge is
  * dcp_merge with num_heads * q_len rows.
  */
@@ -184,8 +194,15 @@ int mla_decode_partial_multi(const void* q, const void* kv_cache, int kv_dtype,
 
 /*
  * Bytes of the scratch array built into the library for
- * mla_decode_partial_noalloc (32 MiB per device that calls it; enough for
- * batch 64 x 64 heads x 148 splits, about 27.8 MB).
+ * mla_decode_partial_noalloc: 32 MiB per device, enough for batch 64 x 64
+ * heads x 148 splits (about 27.8 MB).  Of the five workloads the tiny,
+ * dense, agentic and million-token ones fit; the sparse one (batch 128 with
+ * several index-list parts per request) does not and is refused with
+ * DCPMLA_ERR_WORKSPACE.  The array is part of the library's device module:
+ * with CUDA's lazy module loading (the default) it takes device memory only
+ * on devices where the module is loaded, i.e. that call into the library;
+ * with eager loading (CUDA_MODULE_LOADING=EAGER) it is reserved on every
+ * device the process initialises.
  */
 #define DCPMLA_NOALLOC_SCRATCH_BYTES (32u << 20)
 
@@ -217,6 +234,11 @@ int mla_decode_partial_multi(const void* q, const void* kv_cache, int kv_dtype,
  *    setup: it looks the scratch array up with cudaGetSymbolAddress, which
  *    may load the library's module, and enqueues the first clear of the flag
  *    word.  Make that first call before any stream capture begins.
+ *  - The looked-up address is kept for the life of the process: the setup
+ *    must not outlive the device's context (no cudaDeviceReset, no teardown
+ *    of the primary context, between calls).
+ *  - Query heads only (num_heads <= 64, else DCPMLA_ERR_UNSUPPORTED); there
+ *    is no multi-query or sparse-beyond-the-scratch variant.
  *
  * Returns DCPMLA_OK or a negative DCPMLA_ERR_* code (DCPMLA_ERR_CUDA if the
  * setup fails).

@@ -15,6 +15,7 @@ constexpr int kVDim = 512;
 constexpr int kRopeDim = 64;
 constexpr int kBlock = 64;        // rows per cache block
 constexpr int kMaxHeads = 64;
+constexpr int kMaxQueryLen = 64;   // query tokens per request of a multi-query call
 constexpr int kRowBytesBf16 = 1152;
 constexpr int kRowBytesFp8 = 656;
 constexpr int kWsHeader = 256;    // workspace header: flag word + reserved
@@ -25,14 +26,15 @@ enum : int { kFlagBadBlock = 1, kFlagBadLength = 2 };
 
 // Everything one shard's partial-attention launch needs.
 struct PartialParams {
-  const __nv_bfloat16* q;     // [B][H][576]; multi-query: [B][q_len][H / q_len][576]
+  const __nv_bfloat16* q;     // [B][rows_q][576], the first `heads` rows of each request;
+                              // multi-query: query-major rows (query i, head h)
   const uint8_t* kv;          // [num_blocks][64][row_bytes]
   long long num_blocks;
   const int* block_table;     // [B][bt_stride] this shard's table
   int bt_stride;
   const int* seq_lens;        // [B] global lengths
   int batch;
-  int heads;                  // rows per request: query heads x q_len (<= 64)
+  int heads;                  // rows per request in this pass: query heads x q_len (<= 64)
   int q_len;                  // query tokens per request (1 = plain decode); row r is
                               // query r / (heads / q_len), causal at L_b - q_len + that
   int shard;
@@ -41,8 +43,12 @@ struct PartialParams {
   int topk;
   int sparse_parts;           // index-list chunks per request (sparse mode)
   float scale;                // softmax scale
-  float* out;                 // [B][H][512]
-  float* out_lse;             // [B][H]
+  float* out;                 // [B][rows_o][512] (the first `heads` rows of each request)
+  float* out_lse;             // [B][rows_o]
+  int rows_q;                 // rows between consecutive requests in q (>= heads)
+  int rows_o;                 // rows between consecutive requests in out / out_lse
+  int len_delta;              // subtracted from every valid length (a query pass that
+                              // sits len_delta tokens before the request's end)
   int* flags;                 // workspace flag word
   float* ws_o;                // [slots][H][512]
   float* ws_lse;              // [slots][H]
@@ -66,8 +72,15 @@ __host__ __device__ __forceinline__ int local_len(int L, int s, int N) {
 
 // Tiles of request b on this shard, with the range checks on the length and
 // on the block-table row; sets flag bits instead of reading out of range.
+// Length request b is attended over: its cached length, less len_delta (a
+// negative length stays negative: it is flagged by the callers).
+__device__ __forceinline__ int seq_len_of(const PartialParams& p, int b) {
+  const int L = __ldg(p.seq_lens + b);
+  return L < 0 ? L : max(L - p.len_delta, 0);
+}
+
 __device__ __forceinline__ int request_tiles(const PartialParams& p, int b, int* n_rows) {
-  int L = __ldg(p.seq_lens + b);
+  int L = seq_len_of(p, b);
   if (L < 0) {
     if (p.flags) atomicOr(p.flags, kFlagBadLength);
     L = 0;

@@ -91,7 +91,8 @@ int mla_decode_workspace_size(int batch, int num_heads, int num_splits, int topk
                               size_t* bytes) {
   if (!bytes || batch < 0 || num_heads < 1 || num_splits < 0 || topk < 0)
     return DCPMLA_ERR_INVALID_ARGUMENT;
-  if (num_heads > kMaxHeads) return DCPMLA_ERR_UNSUPPORTED;
+  // rows: query heads, or (query, head) pairs of a multi-query call
+  if (num_heads > kMaxHeads * kMaxQueryLen) return DCPMLA_ERR_UNSUPPORTED;
   int ctas = 0;
   int rc = resolve_ctas(num_splits, &ctas);
   if (rc != DCPMLA_OK) return rc;
@@ -104,13 +105,17 @@ int mla_decode_workspace_size(int batch, int num_heads, int num_splits, int topk
 namespace {
 
 // Shared body of mla_decode_partial (q_len = 1) and mla_decode_partial_multi:
-// num_heads here counts rows (query heads x q_len).
+// num_heads here counts rows (query heads x q_len).  rows_q / rows_o are the
+// rows between consecutive requests in q and in the outputs (num_heads for a
+// plain call), len_delta is subtracted from every length (a pass over the
+// earlier queries of a multi-query call).
 int decode_partial(const void* q, const void* kv_cache, int kv_dtype, int64_t num_blocks,
                    int block_size, const int32_t* block_table, int block_table_stride,
                    const int32_t* seq_lens, int batch, int num_heads, int q_len, int shard_id,
                    int num_shards, const int32_t* sparse_idx, int topk, float softmax_scale,
                    float* out_partial, float* out_lse, void* workspace, size_t workspace_bytes,
-                   int num_splits, int impl, void* stream) {
+                   int num_splits, int impl, void* stream, int rows_q, int rows_o,
+                   int len_delta) {
   // ---- scalar checks (fail closed, nothing launched on error) ----
   const bool withhold = (impl & DCPMLA_TEST_WITHHOLD_ARRIVAL) != 0;
   impl &= ~DCPMLA_TEST_WITHHOLD_ARRIVAL;
@@ -158,6 +163,9 @@ int decode_partial(const void* q, const void* kv_cache, int kv_dtype, int64_t nu
   p.scale = softmax_scale;
   p.out = out_partial;
   p.out_lse = out_lse;
+  p.rows_q = rows_q;
+  p.rows_o = rows_o;
+  p.len_delta = len_delta;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   p.flags = reinterpret_cast<int*>(ws);
   p.ws_o = reinterpret_cast<float*>(ws + ws_o_offset());
@@ -208,7 +216,7 @@ int mla_decode_partial(const void* q, const void* kv_cache, int kv_dtype, int64_
   return decode_partial(q, kv_cache, kv_dtype, num_blocks, block_size, block_table,
                         block_table_stride, seq_lens, batch, num_heads, 1, shard_id, num_shards,
                         sparse_idx, topk, softmax_scale, out_partial, out_lse, workspace,
-                        workspace_bytes, num_splits, impl, stream);
+                        workspace_bytes, num_splits, impl, stream, num_heads, num_heads, 0);
 }
 
 int mla_decode_partial_multi(const void* q, const void* kv_cache, int kv_dtype,
@@ -218,12 +226,40 @@ int mla_decode_partial_multi(const void* q, const void* kv_cache, int kv_dtype,
                              float softmax_scale, float* out_partial, float* out_lse,
                              void* workspace, size_t workspace_bytes, int num_splits, int impl,
                              void* stream) {
-  if (q_len < 1 || num_heads < 1) return DCPMLA_ERR_INVALID_ARGUMENT;
-  if ((long long)num_heads * q_len > kMaxHeads) return DCPMLA_ERR_UNSUPPORTED;
-  return decode_partial(q, kv_cache, kv_dtype, num_blocks, block_size, block_table,
-                        block_table_stride, seq_lens, batch, num_heads * q_len, q_len, shard_id,
-                        num_shards, nullptr, 0, softmax_scale, out_partial, out_lse, workspace,
-                        workspace_bytes, num_splits, impl, stream);
+  if (q_len < 1 || num_heads < 1 || q_len > kMaxQueryLen) return DCPMLA_ERR_INVALID_ARGUMENT;
+  if (num_heads > kMaxHeads) return DCPMLA_ERR_UNSUPPORTED;
+  const int rows = num_heads * q_len;
+  const int base_impl = impl & ~DCPMLA_TEST_WITHHOLD_ARRIVAL;
+  // Queries per pass.  A pass is one decode over the cache whose rows fit
+  // one 64-row tile: the fp8 cache and the CUDA-core kernel take one query
+  // per pass (plain decode rows: the e4m3-direct kernel's exact scores, and
+  // no causal rows for the CUDA-core kernel); the fp16-operand kernel takes
+  // as many whole queries as fit its tile.
+  int qpp = kMaxHeads / num_heads;
+  if (base_impl == DCPMLA_IMPL_SIMT ||
+      (kv_dtype == DCPMLA_KV_FP8 && base_impl != DCPMLA_IMPL_TC_F16))
+    qpp = 1;
+  if (qpp >= q_len)
+    return decode_partial(q, kv_cache, kv_dtype, num_blocks, block_size, block_table,
+                          block_table_stride, seq_lens, batch, rows, q_len, shard_id,
+                          num_shards, nullptr, 0, softmax_scale, out_partial, out_lse, workspace,
+                          workspace_bytes, num_splits, impl, stream, rows, rows, 0);
+  // Several passes, in order on the stream (they share the workspace).
+  // Pass k covers queries [k0, k0 + n): rows k0 * num_heads onward of every
+  // request, over the cache less its last q_len - k0 - n tokens, which puts
+  // its last query at the end of the shortened cache.
+  for (int k0 = 0; k0 < q_len; k0 += qpp) {
+    const int n = q_len - k0 < qpp ? q_len - k0 : qpp;
+    const size_t r0 = (size_t)k0 * num_heads;
+    const int rc = decode_partial(
+        static_cast<const uint8_t*>(q) + r0 * kHeadDim * sizeof(__nv_bfloat16), kv_cache,
+        kv_dtype, num_blocks, block_size, block_table, block_table_stride, seq_lens, batch,
+        n * num_heads, n, shard_id, num_shards, nullptr, 0, softmax_scale,
+        out_partial + r0 * kVDim, out_lse + r0, workspace, workspace_bytes, num_splits, impl,
+        stream, rows, rows, q_len - k0 - n);
+    if (rc != DCPMLA_OK) return rc;
+  }
+  return DCPMLA_OK;
 }
 
 int dcp_merge(const float* partials, const float* lses, int num_shards, int batch,

@@ -53,9 +53,9 @@ __global__ void __launch_bounds__(256) split_combine_kernel(PartialParams p) {
     const int start = sh_start, nt_b = sh_nt;
     if (nt_b == 0) {
       if (h < p.heads) {
-        float* o = p.out + ((size_t)b * p.heads + h) * kVDim;
+        float* o = p.out + ((size_t)b * p.rows_o + h) * kVDim;
         for (int i = threadIdx.x & 31; i < kVDim; i += 32) o[i] = 0.f;
-        if ((threadIdx.x & 31) == 0) p.out_lse[(size_t)b * p.heads + h] = -CUDART_INF_F;
+        if ((threadIdx.x & 31) == 0) p.out_lse[(size_t)b * p.rows_o + h] = -CUDART_INF_F;
       }
       return;
     }
@@ -67,8 +67,8 @@ __global__ void __launch_bounds__(256) split_combine_kernel(PartialParams p) {
   }
   if (h < p.heads)
     merge_warp(StridedPieces{p.ws_o, p.ws_lse, (size_t)first_slot * p.heads + h, (size_t)p.heads},
-               count, p.out + ((size_t)b * p.heads + h) * kVDim,
-               p.out_lse + (size_t)b * p.heads + h);
+               count, p.out + ((size_t)b * p.rows_o + h) * kVDim,
+               p.out_lse + (size_t)b * p.rows_o + h);
 }
 
 }  // namespace

@@ -58,7 +58,9 @@ extern "C" int mla_decode_partial_noalloc(
     float softmax_scale, float* out_partial, float* out_lse, int32_t* out_flags,
     int num_splits, int impl, void* stream) {
   // Size check first: a request that does not fit is refused before any
-  // work is enqueued.
+  // work is enqueued.  (The size function also sizes multi-query rows; this
+  // entry point takes query heads only.)
+  if (num_heads > DCPMLA_MAX_HEADS) return DCPMLA_ERR_UNSUPPORTED;
   size_t need = 0;
   int rc = mla_decode_workspace_size(batch, num_heads, num_splits, sparse_idx ? topk : 0, &need);
   if (rc != DCPMLA_OK) return rc;
@@ -69,14 +71,17 @@ extern "C" int mla_decode_partial_noalloc(
   rc = scratch_for_current_device(st, &scratch);
   if (rc != DCPMLA_OK) return rc;
 
-  // The flag word is zero here: cleared at setup and after every call.
+  // The flag word is zero here: cleared at setup and after every call.  Once
+  // setup succeeded, the clear is queued on every return path, errors
+  // included (best effort), so a failed call leaves no bits for the next.
   rc = mla_decode_partial(q, kv_cache, kv_dtype, num_blocks, block_size, block_table,
                           block_table_stride, seq_lens, batch, num_heads, shard_id, num_shards,
                           sparse_idx, topk, softmax_scale, out_partial, out_lse, scratch,
                           (size_t)DCPMLA_NOALLOC_SCRATCH_BYTES, num_splits, impl, stream);
-  if (rc != DCPMLA_OK) return rc;
-  if (out_flags &&
+  if (rc == DCPMLA_OK && out_flags &&
       cudaMemcpyAsync(out_flags, scratch, kFlagBytes, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
-    return DCPMLA_ERR_CUDA;
-  return cudaMemsetAsync(scratch, 0, kFlagBytes, st) == cudaSuccess ? DCPMLA_OK : DCPMLA_ERR_CUDA;
+    rc = DCPMLA_ERR_CUDA;
+  const bool cleared = cudaMemsetAsync(scratch, 0, kFlagBytes, st) == cudaSuccess;
+  if (rc != DCPMLA_OK) return rc;
+  return cleared ? DCPMLA_OK : DCPMLA_ERR_CUDA;
 }

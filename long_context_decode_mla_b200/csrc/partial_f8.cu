@@ -444,7 +444,7 @@ __device__ __forceinline__ bool prepare_q(const PartialParams& p, F8Ctl& c, uint
   if (sigma > 0 && !wait_or_abort(&c.q_empty, (sigma - 1) & 1, c)) return false;
   const bool live = hq < p.heads;
   const uint4* src =
-      reinterpret_cast<const uint4*>(p.q + ((size_t)b * p.heads + (live ? hq : 0)) * kHeadDim);
+      reinterpret_cast<const uint4*>(p.q + ((size_t)b * p.rows_q + (live ? hq : 0)) * kHeadDim);
   float amax = 0.f;
 #pragma unroll 4
   for (int k = 0; k < 32; ++k) {
@@ -804,10 +804,11 @@ __device__ __forceinline__ void softmax_role(const PartialParams& p, F8Ctl& c, u
       ptx::tc_fence_after();
       const float ltot = (ls[0][h] + ls[1][h]) + (ls[2][h] + ls[3][h]);
       if (col == 0 && h < p.heads)
-        (v.whole ? p.out_lse : p.ws_lse)[slot * p.heads + h] =
+        (v.whole ? p.out_lse : p.ws_lse)[slot * (v.whole ? p.rows_o : p.heads) + h] =
             ltot > 0.f ? (m_used + log2f(ltot)) * kLn2 : -CUDART_INF_F;
       const float il = ltot > 0.f ? 1.f / ltot : 0.f;
-      float* o_base = (v.whole ? p.out : p.ws_o) + (slot * p.heads + h) * kVDim + odh;
+      float* o_base = (v.whole ? p.out : p.ws_o) +
+                      (slot * (v.whole ? p.rows_o : p.heads) + h) * kVDim + odh;
 #pragma unroll 1
       for (int g = 0; g < 4; ++g) {
         const float sg = g == 0 ? sref.x : g == 1 ? sref.y : g == 2 ? sref.z : sref.w;

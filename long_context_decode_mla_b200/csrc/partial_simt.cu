@@ -177,7 +177,7 @@ __device__ void attend_rows(const PartialParams& p, SimtSmem& sm, int n, RowOf r
 }
 
 __device__ void load_q(const PartialParams& p, SimtSmem& sm, int b) {
-  const uint4* src = reinterpret_cast<const uint4*>(p.q + (size_t)b * p.heads * kHeadDim);
+  const uint4* src = reinterpret_cast<const uint4*>(p.q + (size_t)b * p.rows_q * kHeadDim);
   for (int i = threadIdx.x; i < p.heads * 72; i += kThreads) {
     const int h = i / 72, c = i % 72;
     *reinterpret_cast<uint4*>(sm.q + h * kQPad + 8 * c) = src[i];
@@ -236,8 +236,8 @@ __global__ void __launch_bounds__(kThreads, 1) partial_simt_dense(PartialParams 
     }, acc);
     const bool whole = s.t0 == 0 && s.t1 == s.nt;
     const size_t slot = whole ? (size_t)s.b : (size_t)blockIdx.x + s.b;
-    float* o_base = (whole ? p.out : p.ws_o) + slot * p.heads * kVDim;
-    float* l_base = (whole ? p.out_lse : p.ws_lse) + slot * p.heads;
+    float* o_base = (whole ? p.out : p.ws_o) + slot * (whole ? p.rows_o : p.heads) * kVDim;
+    float* l_base = (whole ? p.out_lse : p.ws_lse) + slot * (whole ? p.rows_o : p.heads);
     store_result(p, sm, acc, o_base, l_base);
   });
 }
@@ -251,7 +251,7 @@ __global__ void __launch_bounds__(kThreads, 1) partial_simt_sparse(PartialParams
   if (b >= p.batch) return;
   const int chunk = (p.topk + p.sparse_parts - 1) / p.sparse_parts;
   const int i0 = part * chunk, i1 = min(p.topk, i0 + chunk);
-  int L = __ldg(p.seq_lens + b);
+  int L = seq_len_of(p, b);
   if (L < 0) {
     if (p.flags) atomicOr(p.flags, kFlagBadLength);
     L = 0;
@@ -286,8 +286,8 @@ __global__ void __launch_bounds__(kThreads, 1) partial_simt_sparse(PartialParams
   }, acc);
   const bool whole = p.sparse_parts == 1;
   const size_t slot = whole ? (size_t)b : (size_t)blockIdx.x;
-  float* o_base = (whole ? p.out : p.ws_o) + slot * p.heads * kVDim;
-  float* l_base = (whole ? p.out_lse : p.ws_lse) + slot * p.heads;
+  float* o_base = (whole ? p.out : p.ws_o) + slot * (whole ? p.rows_o : p.heads) * kVDim;
+  float* l_base = (whole ? p.out_lse : p.ws_lse) + slot * (whole ? p.rows_o : p.heads);
   store_result(p, sm, acc, o_base, l_base);
 }
 

@@ -403,10 +403,11 @@ __device__ __forceinline__ void softmax_role(const PartialParams& p, TcCtl& c, u
     const SegView v = seg_view(p, c, 0);
     const size_t slot = v.whole ? (size_t)v.b : (size_t)blockIdx.x;
     if (h < p.heads) {
-      float* o = (v.whole ? p.out : p.ws_o) + (slot * p.heads + h) * kVDim;
+      const size_t row = slot * (v.whole ? p.rows_o : p.heads) + h;
+      float* o = (v.whole ? p.out : p.ws_o) + row * kVDim;
       for (int i = half; i < kVDim / 4; i += 2)
         reinterpret_cast<float4*>(o)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (half == 0) (v.whole ? p.out_lse : p.ws_lse)[slot * p.heads + h] = -CUDART_INF_F;
+      if (half == 0) (v.whole ? p.out_lse : p.ws_lse)[row] = -CUDART_INF_F;
     }
     return;
   }
@@ -430,7 +431,7 @@ __device__ __forceinline__ void softmax_role(const PartialParams& p, TcCtl& c, u
       // Causal rows: row h is query i = h / (heads / q_len) at global position
       // L_b - q_len + i; it sees local rows j with j * N + shard <= that.
       if (cur.t == 0) {
-        const int lim = max(__ldg(p.seq_lens + cur.v.b), 0) - p.q_len + h / (p.heads / p.q_len);
+        const int lim = max(seq_len_of(p, cur.v.b), 0) - p.q_len + h / (p.heads / p.q_len);
         jmax = lim >= p.shard ? (lim - p.shard) / p.nshards : -1;
       }
       const int cmax = jmax - (cur.v.row_begin + cur.t * kTileTok + half * 32);
@@ -512,8 +513,9 @@ __device__ __forceinline__ void softmax_role(const PartialParams& p, TcCtl& c, u
       const SegView& v = cur.v;
       const size_t slot = v.whole ? (size_t)v.b
                                   : (p.sparse_idx ? (size_t)blockIdx.x : (size_t)blockIdx.x + v.b);
-      float* o_base = (v.whole ? p.out : p.ws_o) + (slot * p.heads + h) * kVDim;
-      float* l_base = (v.whole ? p.out_lse : p.ws_lse) + slot * p.heads + h;
+      const size_t row = slot * (v.whole ? p.rows_o : p.heads) + h;
+      float* o_base = (v.whole ? p.out : p.ws_o) + row * kVDim;
+      float* l_base = (v.whole ? p.out_lse : p.ws_lse) + row;
       // o_full completes once per request, after its last PV (and so after
       // all of its PVs).  Earlier phases were consumed by earlier epilogues and
       // the next one needs this thread's P, so the parity wait is unambiguous.
@@ -679,7 +681,7 @@ __device__ __forceinline__ void stage_store_half1(uint8_t* stage, int ct, const 
 // Q of request b into the Q region: 64 rows x 72 units of fp16, heads >= H zero.
 __device__ __forceinline__ void load_q(const PartialParams& p, int b, uint8_t* sq, int ct,
                                        bool& range_bad) {
-  const uint4* qb = reinterpret_cast<const uint4*>(p.q + (size_t)b * p.heads * kHeadDim);
+  const uint4* qb = reinterpret_cast<const uint4*>(p.q + (size_t)b * p.rows_q * kHeadDim);
   float amax = 0.f;
 #pragma unroll 6
   for (int i = 0; i < 18; ++i) {

@@ -134,7 +134,7 @@ __device__ int compact_sparse(const PartialParams& p, int* list, Ctl& c) {
   const int b = blockIdx.x / p.sparse_parts, part = blockIdx.x % p.sparse_parts;
   const int chunk = (p.topk + p.sparse_parts - 1) / p.sparse_parts;
   const int i0 = part * chunk, i1 = min(p.topk, i0 + chunk);
-  int L = __ldg(p.seq_lens + b);
+  int L = seq_len_of(p, b);
   if (L < 0) {
     if (threadIdx.x == 0 && p.flags) atomicOr(p.flags, kFlagBadLength);
     L = 0;

@@ -58,7 +58,9 @@ def test_workspace_size_rejects_bad_arguments():
     n = ctypes.c_size_t(0)
     assert L.mla_decode_workspace_size(-1, 64, 1, 0, ctypes.byref(n)) == EINVAL
     assert L.mla_decode_workspace_size(1, 0, 1, 0, ctypes.byref(n)) == EINVAL
-    assert L.mla_decode_workspace_size(1, 65, 1, 0, ctypes.byref(n)) == EUNSUP
+    # rows: 64 heads, or (query, head) pairs of a multi-query call, up to 64 x 64
+    assert L.mla_decode_workspace_size(1, 64 * 64 + 1, 1, 0, ctypes.byref(n)) == EUNSUP
+    assert L.mla_decode_workspace_size(1, 256, 1, 0, ctypes.byref(n)) == 0
     assert L.mla_decode_workspace_size(1, 8, 1, 0, None) == EINVAL
 
 
@@ -189,8 +191,10 @@ def test_multi_query_fails_closed_before_any_launch():
                  FAKE, FAKE, FAKE, 0, 4, impl, None)
 
     assert call(q_len=0) == EINVAL and call(heads=0) == EINVAL
-    assert call(heads=16, q_len=5) == EUNSUP                 # 80 rows > 64
-    assert call(heads=64, q_len=2) == EUNSUP
+    # more than 64 rows run as passes over the cache: accepted, and then the
+    # (empty) workspace is refused before anything is launched
+    assert call(heads=16, q_len=5) == EWS and call(heads=64, q_len=4) == EWS
+    assert call(heads=65) == EUNSUP and call(q_len=65) == EINVAL
     assert call(shard=2) == EINVAL and call(kvd=3) == EINVAL and call(bs=16) == EUNSUP
     assert call(q=FAKE + 2) == EALIGN
     assert call(batch=0) == OK                               # nothing to do

@@ -28,7 +28,9 @@ from long_context_decode_mla_b200 import workload as wl
 
 pytestmark = pytest.mark.gpu
 
-TOL = {"bf16": (2e-3, 1e-4), "fp8": (2e-2, 5e-3)}
+# fp8 LSE: 1e-3 on the exact dense path; the sparse fp8 path runs on the
+# fp16-operand kernel (e4m3 * scale rounded to fp16 before the MMA), 5e-3
+TOL = {"bf16": (2e-3, 1e-4), "fp8": (2e-2, 1e-3), "fp8-sparse": (2e-2, 5e-3)}
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -98,7 +100,8 @@ def test_merge_heads_over_exchange_buffers(name, N, H, lens):
                                                    ni["softmax_scale"],
                                                    sparse_idx=ni["sparse_idx"])
         _compare(out.double().cpu().numpy(), out_lse.double().cpu().numpy(), o_ref, l_ref,
-                 prob.kv_dtype)
+                 prob.kv_dtype + ("-sparse" if prob.kv_dtype == "fp8" and prob.sparse_idx is not None
+                                  else ""))
     finally:
         torch.cuda.synchronize()
         for a in bufs:

@@ -2,14 +2,14 @@
 
 Tolerances, applied to every shard's partials and to the merged result: bf16
 cache max|dO| <= 2e-3 * max|O| and |dLSE| <= 1e-4, fp8 cache max|dO| <=
-2e-2 * max|O| (the required accuracy of the decode path).  No LSE bound is
-given for fp8 rows; it is derived from the arithmetic: the tensor cores read
-e4m3 * scale rounded once to fp16 (relative error <= 2^-11 per value,
-independent across values; the scale itself is carried as an fp16 hi + lo
-pair so no error is shared by a whole group), so a score moves by about
-0.072 * 2^-11 * sqrt(sum_d q_d^2 k_d^2) ~ 0.9e-3 (rms, N(0,1) data, 512
-latent values); the LSE, a softmax-weighted mean of score errors, stays
-within 5e-3 over all heads and requests, large scores included.
+2e-2 * max|O| (the required accuracy of the decode path) and |dLSE| <= 1e-3.
+The fp8 dense path multiplies the e4m3 codes exactly and applies each
+per-128 scale in fp32, so its scores carry only fp32 accumulation error (the
+CUDA-core kernel likewise).  The sparse fp8 path still runs on the
+fp16-operand kernel, which rounds e4m3 * scale once to fp16 before the MMA
+(relative error <= 2^-11 per value, independent across values), so a score
+moves by about 0.072 * 2^-11 * sqrt(sum_d q_d^2 k_d^2) ~ 0.9e-3 (rms, N(0,1)
+data, 512 latent values); its LSE bound stays 5e-3.
 Empty shards must return exactly (0, -inf).  Addressing and sparse selection
 are checked bit-exactly with id-coded rows.
 """
@@ -25,7 +25,14 @@ from long_context_decode_mla_b200 import workload as wl
 
 pytestmark = pytest.mark.gpu
 
-TOL = {"bf16": (2e-3, 1e-4), "fp8": (2e-2, 5e-3)}
+TOL = {"bf16": (2e-3, 1e-4), "fp8": (2e-2, 1e-3)}
+TOL_FP8_FP16_OPERANDS = (2e-2, 5e-3)     # sparse fp8: the fp16-operand kernel
+
+
+def _tol(kv_dtype, impl, sparse):
+    if kv_dtype == "fp8" and sparse and impl != "simt":
+        return TOL_FP8_FP16_OPERANDS
+    return TOL[kv_dtype]
 IMPLS = ["simt", "auto"]
 
 
@@ -55,8 +62,8 @@ def _oracle(prob, batch_ids=None):
                              ni["sparse_idx"], ni["block_size"], batch_ids)
 
 
-def _compare(o, l, o_ref, l_ref, kv_dtype, what):
-    rel_o, abs_l = TOL[kv_dtype]
+def _compare(o, l, o_ref, l_ref, kv_dtype, what, tol=None):
+    rel_o, abs_l = TOL[kv_dtype] if tol is None else tol
     fin = np.isfinite(l_ref)
     assert np.array_equal(fin, np.isfinite(l)), f"{what}: -inf pattern differs"
     assert np.all(np.isneginf(l[~fin])), f"{what}: empty rows must have LSE -inf"
@@ -76,9 +83,10 @@ def _check_problem(prob, impl="auto", batch_ids=None, num_splits=0, streams=None
     parts, lses, out, lse = _run(prob, impl, num_splits, streams)
     rp, rl, ro, rlse = _oracle(prob, batch_ids)
     ids = list(range(prob.batch)) if batch_ids is None else list(batch_ids)
+    tol = _tol(prob.kv_dtype, impl, prob.sparse_idx is not None)
     for s in range(prob.num_shards):
-        _compare(parts[s, ids], lses[s, ids], rp[s], rl[s], prob.kv_dtype, f"shard {s}")
-    return _compare(out[ids], lse[ids], ro, rlse, prob.kv_dtype, "merged")
+        _compare(parts[s, ids], lses[s, ids], rp[s], rl[s], prob.kv_dtype, f"shard {s}", tol)
+    return _compare(out[ids], lse[ids], ro, rlse, prob.kv_dtype, "merged", tol)
 
 
 # --------------------------------------------------------------- small ------

@@ -1,7 +1,8 @@
 """The bounded-wait (timeout) path of the tensor-core kernel, on the GPU.
 
-With DCPMLA_TEST_WITHHOLD_ARRIVAL the converter warps withhold their first
-arrival, so nothing ever completes the first stage: every waiting role of
+With DCPMLA_TEST_WITHHOLD_ARRIVAL the fp16-operand kernel's converter warps
+withhold their first arrival (the e4m3 kernel's producer withholds its first
+tile), so nothing ever completes the first stage: every waiting role of
 every CTA gives up after its clock budget (about 2 s), the CTA drains, frees
 its tensor memory and sets DCPMLA_FLAG_TIMEOUT.  No trap, fault or unbounded
 wait is involved, and the context must stay usable: a normal call right after
@@ -51,6 +52,34 @@ def test_withheld_arrival_times_out_and_the_context_survives():
                                            ni["seq_lens"], 2, ni["softmax_scale"])
     out = dec.out.double().cpu().numpy()
     assert np.abs(out - ref).max() <= 2e-3 * np.abs(ref).max()
+
+
+def test_withheld_tile_times_out_on_the_e4m3_kernel():
+    # fp8 single-token decode runs on the e4m3-direct kernel: the producer
+    # withholds every CTA's first tile, so staging, scores, softmax and PV
+    # waits run out; the CTAs drain, free TMEM and flag the timeout
+    prob = wl.make_problem("agentic", num_shards=2, batch=3, seq_len=[1500, 300, 64],
+                           seed=41).to("cuda")
+    B, H = prob.batch, prob.heads
+    o = torch.empty(B, H, 512, device="cuda")
+    l = torch.empty(B, H, device="cuda")
+    ws = torch.zeros(dcpmla.mla_decode_workspace_size(B, H, 6), dtype=torch.uint8, device="cuda")
+    dcpmla.mla_decode_partial(prob.q, prob.kv_cache, "fp8", prob.block_tables[0], prob.seq_lens,
+                              0, 2, None, prob.softmax_scale, o, l, ws, 6,
+                              dcpmla.IMPLS["tc"] | WITHHOLD)
+    torch.cuda.synchronize()
+    assert int(ws[:4].view(torch.int32).item()) & dcpmla.FLAG_TIMEOUT
+
+    dec = dcpmla.DcpDecoder(B, H, 2, impl="tc")
+    dec.step(prob)
+    torch.cuda.synchronize()
+    assert dec.flags() == 0
+    ni = wl.make_problem("agentic", num_shards=2, batch=3, seq_len=[1500, 300, 64],
+                         seed=41).numpy_inputs()
+    _, _, ref, ref_lse = oracle.dcp_decode(ni["q"], ni["kv_cache"], "fp8", ni["block_tables"],
+                                           ni["seq_lens"], 2, ni["softmax_scale"])
+    assert np.abs(dec.out.double().cpu().numpy() - ref).max() <= 2e-2 * np.abs(ref).max()
+    assert np.abs(dec.out_lse.double().cpu().numpy() - ref_lse).max() <= 1e-3
 
 
 def test_withhold_needs_the_tensor_core_kernel():

@@ -3,8 +3,9 @@
 The no-alloc entry point runs the same kernels on a scratch array built into
 the library (one per device) instead of a caller's workspace.  This file is
 named to be collected last, so that it runs both alone and after every other
-GPU test in the same process.  Tolerances are the parity tests' (bf16 cache:
-max|dO| <= 2e-3 max|O|, |dLSE| <= 1e-4; fp8 cache: 2e-2 and 5e-3).
+GPU test in the same process.  Both entry points run the same kernels, so
+the parity tests' tolerances hold with room (bf16 cache: max|dO| <= 2e-3
+max|O|, |dLSE| <= 1e-4; fp8 cache: 2e-2 and 1e-3).
 """
 import numpy as np
 import pytest
@@ -15,7 +16,7 @@ from long_context_decode_mla_b200 import workload as wl
 
 pytestmark = pytest.mark.gpu
 
-TOL = {"bf16": (2e-3, 1e-4), "fp8": (2e-2, 5e-3)}
+TOL = {"bf16": (2e-3, 1e-4), "fp8": (2e-2, 1e-3)}
 
 
 @pytest.fixture(scope="module", autouse=True)
