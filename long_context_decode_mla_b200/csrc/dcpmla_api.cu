@@ -2,6 +2,7 @@
 // The entry points are declared (and their contracts stated) in dcpmla.h.
 #include "dcpmla.h"
 
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 
@@ -16,15 +17,18 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 int sm_count_current(int* out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return DCPMLA_ERR_CUDA;
-  static int cache[64] = {0};
-  if (dev >= 0 && dev < 64 && cache[dev] > 0) {
-    *out = cache[dev];
+  if (dev < 0 || dev >= kMaxDevicesConfigured) return DCPMLA_ERR_UNSUPPORTED;
+  // per-device cache; host threads may ask at once, so each entry is atomic
+  static std::atomic<int> cache[kMaxDevicesConfigured];
+  const int c = cache[dev].load(std::memory_order_relaxed);
+  if (c > 0) {
+    *out = c;
     return DCPMLA_OK;
   }
   int n = 0;
   if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
     return DCPMLA_ERR_CUDA;
-  if (dev >= 0 && dev < 64) cache[dev] = n;
+  cache[dev].store(n, std::memory_order_relaxed);
   *out = n;
   return DCPMLA_OK;
 }

@@ -42,6 +42,8 @@
 #include <cuda_fp8.h>
 #include <math_constants.h>
 
+#include <mutex>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "schedule.cuh"
@@ -908,15 +910,21 @@ cudaError_t launch_partial_tc(const PartialParams& p, int kv_dtype, cudaStream_t
                     : (sparse ? partial_tc_kernel<kKvFp8, true> : partial_tc_kernel<kKvFp8, false>);
   // Raise the shared-memory limit once per kernel and device, so that later
   // launches (including ones captured into a CUDA graph) are plain launches.
-  static int configured[4][64] = {};
+  // The record is guarded: host threads may make their first calls at once.
+  static std::mutex mu;
+  static bool configured[4][kMaxDevicesConfigured] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  int& done = configured[(kv_dtype == kKvBf16 ? 0 : 2) + (sparse ? 1 : 0)][dev & 63];
-  if (!done) {
-    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    done = 1;
+  if (dev < 0 || dev >= kMaxDevicesConfigured) return cudaErrorInvalidDevice;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    bool& done = configured[(kv_dtype == kKvBf16 ? 0 : 2) + (sparse ? 1 : 0)][dev];
+    if (!done) {
+      e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      if (e != cudaSuccess) return e;
+      done = true;
+    }
   }
   kernel<<<grid, kThreads, smem, st>>>(p);
   return cudaGetLastError();
