@@ -54,6 +54,13 @@ def parse():
                          "(default N; 1 = serial)")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's batch (smaller cases for profiling)")
+    ap.add_argument("--million-layers", type=int, default=83,
+                    help="resident layer caches of the million-token leg (83: the model)")
+    ap.add_argument("--replicas", action="store_true",
+                    help="with several GPUs: independent replicas of the emulated step "
+                         "instead of the real DCP step across the GPUs")
+    ap.add_argument("--dcp", action="store_true",
+                    help="run the real DCP step (one shard per GPU, NCCL) even on one GPU")
     return ap.parse_args()
 
 
@@ -165,7 +172,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "50"],
+                 "--format=csv,noheader,nounits", "-lms", "20"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
@@ -268,13 +275,25 @@ def run_ours(args, rank, world, local):
         dist.barrier()
     torch.cuda.synchronize(dev)
     sampler.mark(True)
-    ms_step = timed_replays(step_graph, args.steps, stream, flush)
+    st_step = replay_stats(step_graph, args.steps, stream, flush)
     sampler.mark(False)
+    # the same steps for about a second more (untimed), so that the clock
+    # record under this load has enough samples even when K steps are short
+    load = ClockSampler(local)
+    load.samples = sampler.samples
+    load.mark(True)
+    t_end = time.time() + 1.0
+    while time.time() < t_end:
+        for _ in range(20):
+            step_graph.replay()
+        torch.cuda.synchronize(dev)
+    load.mark(False)
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
     # the partial kernels alone (N shard launches + their split combines)
-    ms_partials = timed_replays(partial_graph, args.steps, stream, flush)
+    st_part = replay_stats(partial_graph, args.steps, stream, flush)
+    ms_step, ms_partials = st_step["mean"], st_part["mean"]
 
     # end to end through the public API, host buffers in pinned memory
     h_q = prob.q.cpu().pin_memory()
@@ -311,6 +330,8 @@ def run_ours(args, rank, world, local):
     sampler.stop()
 
     ms_step, e2e_ms, ms_partials = max_over_ranks([ms_step, e2e_ms, ms_partials])
+    st_step = dict(zip(st_step, max_over_ranks(list(st_step.values()))))
+    st_part = dict(zip(st_part, max_over_ranks(list(st_part.values()))))
     gpu_launches = args.steps * (N * (1 if (prob.sparse_idx is not None) else 2) + 1)
     peak, peak_kind = measured_peaks()
     result = None
@@ -320,11 +341,12 @@ def run_ours(args, rank, world, local):
         achieved = (kvb + N * other_per_launch) / (ms_partials * 1e-3) / 1e9
         traffic = recorded_traffic(args.workload, args.kernel)
         clocks = sampler.summary()
+        clocks["under_load_1s"] = load.summary()
         result = {
             "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": round(ms_step, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "bf16" if args.kernel != "simt" else "f32",
+            "dtype": dtype_label(prob.kv_dtype, args.kernel),
             "data": "synthetic (seeded; no public trace or checkpoint available)",
             "config": {
                 "workload": describe(args.workload, prob), "global_batch": B * world,
@@ -346,6 +368,8 @@ def run_ours(args, rank, world, local):
                                    "launches of a step (one stream each, overlapping), algorithmic "
                                    "bytes / device time of that phase, CUDA-graph replay"},
             "ms_partials_per_step": round(ms_partials, 4),
+            "ms_step_stats": ms_summary(st_step),
+            "ms_partials_stats": ms_summary(st_part),
             "e2e": {"value": round(world * kvb / (e2e_ms * 1e-3) / 1e9, 1), "unit": UNIT,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": round(e2e_ms, 4),
@@ -357,9 +381,15 @@ def run_ours(args, rank, world, local):
     # secondary measurements (same rank layout; every rank runs them, rank 0 reports)
     extras = {}
     if args.workload == "agentic" and not args.no_extras:
-        extras["at_64k"] = time_other_workload("agentic64k", dev, rank, world, args, streams_for=N)
-    if prob.sparse_idx is None and prob.heads % 4 == 0:
-        extras["multi_query"] = time_multi_query(prob, dev, args, q_len=4)
+        # every configuration, each timed as its own graph-replayed steps
+        extras["at_64k"] = time_other_workload("agentic64k", dev, rank, world, args)
+        legs = {"dense": lambda: time_other_workload("dense", dev, rank, world, args),
+                "sparse": lambda: time_other_workload("sparse", dev, rank, world, args),
+                "million": lambda: time_million_layers(dev, rank, world, args,
+                                                       layers=args.million_layers)}
+        extras["configs"] = {k: f() for k, f in legs.items()}
+    if prob.sparse_idx is None and not args.no_extras:
+        extras["multi_query"] = time_multi_query(prob, dev, args, q_len=4, world=world)
     extras["kv_append"] = time_append(prob, dev, max(20, args.steps // 4))
     if H % N == 0:
         extras["merge_heads"] = time_merge_heads(dec, dev, max(20, args.steps // 4))
@@ -374,91 +404,193 @@ def run_ours(args, rank, world, local):
 L2_BYTES = 126 << 20
 
 
-def timed_replays(graph, steps, stream, flush=None):
-    """Mean device time (ms) of `steps` graph replays on `stream`.  With a
-    flush buffer, each replay is timed alone after overwriting the buffer."""
+def replay_stats(graph, steps, stream, flush=None):
+    """Device times (ms) of `steps` graph replays on `stream`, each between
+    its own pair of CUDA events: mean, median, min and max.  Replays run back
+    to back; with a flush buffer, each replay follows an overwrite of the
+    buffer (outside its events)."""
     import torch
-    if flush is None:
-        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        t0.record(stream)
-        for _ in range(steps):
-            graph.replay()
-        t1.record(stream)
-        t1.synchronize()
-        return t0.elapsed_time(t1) / steps
     pairs = []
     for i in range(steps):
-        flush.fill_(i & 0xFF)
+        if flush is not None:
+            flush.fill_(i & 0xFF)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         graph.replay()
         b.record(stream)
         pairs.append((a, b))
     pairs[-1][1].synchronize()
-    return sum(a.elapsed_time(b) for a, b in pairs) / steps
+    t = [a.elapsed_time(b) for a, b in pairs]
+    return {"mean": sum(t) / len(t), "median": statistics.median(t), "min": min(t),
+            "max": max(t)}
 
 
-def time_other_workload(name, dev, rank, world, args, streams_for):
-    """Graph-replayed steps of another workload (for "steps/s at 64K context")."""
+def timed_replays(graph, steps, stream, flush=None):
+    """Mean device time (ms) of `steps` graph replays (see replay_stats)."""
+    return replay_stats(graph, steps, stream, flush)["mean"]
+
+
+def ms_summary(st):
+    return {k: round(v, 4) for k, v in st.items()}
+
+
+def step_bytes(prob, kvb=None):
+    """Algorithmic bytes of one emulated DCP step: the KV rows read once
+    (sparse: the selected rows), and for each of the N shard launches its
+    query (bf16), index list (sparse) and partial O + LSE (fp32) written,
+    then the merge reading the N partials and writing the result."""
+    B, H, N = prob.batch, prob.heads, prob.num_shards
+    kvb = kv_bytes(prob) if kvb is None else kvb
+    idx = 0 if prob.sparse_idx is None else prob.sparse_idx.numel() * 4
+    per_launch = B * H * 576 * 2 + B * H * 513 * 4 + idx
+    return kvb + N * per_launch + (N + 1) * B * H * 513 * 4
+
+
+def leg(name, prob, stats, world, kvb=None, total=None, extra=None):
+    """One secondary measurement: device-time statistics of graph-replayed
+    steps, KV GB/s and total algorithmic GB/s (both whole job), and the
+    fraction of the HBM peak."""
+    peak, _ = measured_peaks()
+    kvb = kv_bytes(prob) if kvb is None else kvb
+    total = step_bytes(prob, kvb) if total is None else total
+    ms = stats["mean"]
+    d = {"workload": describe(name, prob), "ms_per_step": ms_summary(stats),
+         "steps_per_s": round(world * 1e3 / ms, 2),
+         "kv_GBps": round(world * kvb / (ms * 1e-3) / 1e9, 1),
+         "total_GBps": round(world * total / (ms * 1e-3) / 1e9, 1),
+         "frac": round(total / (ms * 1e-3) / 1e9 / peak, 4), "unit": UNIT,
+         "kv_bytes_per_step": kvb, "total_bytes_per_step": total}
+    if extra:
+        d.update(extra)
+    return d
+
+
+def time_other_workload(name, dev, rank, world, args, streams_for=None):
+    """Graph-replayed steps of another workload, each step timed alone (L2
+    flushed first when the step reads less than 4x the L2)."""
     import torch
     from long_context_decode_mla_b200 import dcpmla, workload
     cfg = dict(workload.CONFIGS[name])
     prob = workload.make_problem(name, device=dev, kv_device=dev, seed=cfg["seed"] + 1000 * rank)
     N = prob.num_shards
+    topk = 0 if prob.sparse_idx is None else prob.sparse_idx.shape[1]
     streams = [torch.cuda.Stream(device=dev) for _ in range(N)]
-    dec = dcpmla.DcpDecoder(prob.batch, prob.heads, N, device=dev, impl=args.kernel,
-                            streams=streams)
+    splits = max(1, dcpmla.device_sm_count() // N) if name == "million" else 0
+    dec = dcpmla.DcpDecoder(prob.batch, prob.heads, N, topk=topk, num_splits=splits, device=dev,
+                            impl=args.kernel, streams=streams)
     graph = dec.capture(prob)
+    kvb = kv_bytes(prob)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if kvb < 4 * L2_BYTES else None
     for _ in range(max(3, args.warmup)):
         graph.replay()
     torch.cuda.synchronize(dev)
     steps = max(20, args.steps // 4)
     stream = torch.cuda.current_stream(dev)
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    t0.record(stream)
-    for _ in range(steps):
-        graph.replay()
-    t1.record(stream)
-    t1.synchronize()
+    st = replay_stats(graph, steps, stream, flush)
     assert dec.flags() == 0, "device flags set"
-    ms = max_over_ranks([t0.elapsed_time(t1) / steps])[0]
-    kvb = kv_bytes(prob)
-    desc = describe(name, prob)
-    del graph, dec, prob
+    st = dict(zip(st, max_over_ranks(list(st.values()))))
+    d = leg(name, prob, st, world, kvb,
+            extra={"steps": steps,
+                   "l2": "256 MB written before every step" if flush is not None else "no flush"})
+    if prob.sparse_idx is not None:
+        d["note"] = ("kv_GBps counts the selected rows read (each once); total_GBps adds the "
+                     "queries, the index lists (read by every shard), partials and the merge")
+    del graph, dec, prob, flush
     torch.cuda.empty_cache()
-    return {"workload": desc, "steps_per_s": round(world * 1e3 / ms, 2),
-            "ms_per_step": round(ms, 4), "value": round(world * kvb / (ms * 1e-3) / 1e9, 1),
-            "unit": UNIT, "steps": steps}
+    return d
 
 
-def time_multi_query(prob, dev, args, q_len):
-    """The same cache and rows as the headline step, read as heads / q_len
-    heads x q_len query tokens with causal limits (speculative verification):
-    KV bytes per step are unchanged, query tokens per step are q_len x."""
+def time_million_layers(dev, rank, world, args, layers=83):
+    """The million-token configuration as one model step: `layers` resident
+    layer caches of the 1M-token request (about 53 GiB of fp8 rows), each
+    layer one emulated DCP step over its own cache, all captured in one CUDA
+    graph.  The caches are copies of one seeded layer in distinct memory
+    (their contents do not change the work)."""
     import torch
-    from long_context_decode_mla_b200 import dcpmla
-    B, N, H = prob.batch, prob.num_shards, prob.heads // q_len
+    from long_context_decode_mla_b200 import dcpmla, workload
+    cfg = dict(workload.CONFIGS["million"])
+    prob = workload.make_problem("million", device=dev, kv_device=dev,
+                                 seed=cfg["seed"] + 1000 * rank)
+    N = prob.num_shards
+    caches = [prob.kv_cache] + [prob.kv_cache.clone() for _ in range(layers - 1)]
+    cache_bytes = sum(c.numel() for c in caches)
     streams = [torch.cuda.Stream(device=dev) for _ in range(N)]
-    dec = dcpmla.DcpDecoder(B, H, N, device=dev, impl=args.kernel, streams=streams, q_len=q_len)
-    graph = dec.capture(prob)
+    splits = max(1, dcpmla.device_sm_count() // N)
+    dec = dcpmla.DcpDecoder(prob.batch, prob.heads, N, num_splits=splits, device=dev,
+                            impl=args.kernel, streams=streams)
+    views = [workload.DecodeProblem(prob.q, c, prob.kv_dtype, prob.block_tables, prob.seq_lens,
+                                    N) for c in caches]
+    side = torch.cuda.Stream(device=dev)
+    side.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(side):
+        dec.step(views[0], side)
+    torch.cuda.current_stream(dev).wait_stream(side)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=side):
+        for v in views:
+            dec.step(v, side)
     for _ in range(3):
         graph.replay()
     torch.cuda.synchronize(dev)
-    steps = max(20, args.steps // 4)
-    stream = torch.cuda.current_stream(dev)
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    t0.record(stream)
-    for _ in range(steps):
-        graph.replay()
-    t1.record(stream)
-    t1.synchronize()
+    steps = max(5, args.steps // 20)
+    st = replay_stats(graph, steps, torch.cuda.current_stream(dev))
     assert dec.flags() == 0, "device flags set"
-    ms = t0.elapsed_time(t1) / steps
+    st = dict(zip(st, max_over_ranks(list(st.values()))))
+    kvb = layers * kv_bytes(prob)
+    total = layers * step_bytes(prob)
+    d = leg("million", prob, st, world, kvb, total,
+            extra={"layers": layers, "resident_cache_GiB": round(cache_bytes / 2**30, 2),
+                   "model_steps_per_s": round(world * 1e3 / st["mean"], 2), "steps": steps,
+                   "note": f"one model step = {layers} layers x (N shard partials + merge) in one "
+                           "CUDA graph; caches far larger than L2, no flush"})
+    del graph, dec, views, caches, prob
+    torch.cuda.empty_cache()
+    return d
+
+
+def time_multi_query(prob, dev, args, q_len, world=1):
+    """Multi-query decode (speculative verification) over the headline cache
+    at the models' head count: every request carries q_len query tokens of
+    all its heads (q_len x 64 rows), causal at the cache end.  Rows beyond one
+    64-row tile run as one pass per query over the cache, so each step reads
+    the cache about q_len times: kv_GBps counts every pass's rows,
+    cache_GBps the distinct cache once."""
+    import torch
+    from long_context_decode_mla_b200 import dcpmla, workload
+    B, N, H = prob.batch, prob.num_shards, prob.heads
+    q = workload.random_q(B, q_len * H, 9001).to(dev)
+    mq = workload.DecodeProblem(q, prob.kv_cache, prob.kv_dtype, prob.block_tables,
+                                prob.seq_lens, N)
+    streams = [torch.cuda.Stream(device=dev) for _ in range(N)]
+    dec = dcpmla.DcpDecoder(B, H, N, device=dev, impl=args.kernel, streams=streams, q_len=q_len)
+    graph = dec.capture(mq)
+    for _ in range(3):
+        graph.replay()
+    torch.cuda.synchronize(dev)
+    steps = max(10, args.steps // 8)
+    st = replay_stats(graph, steps, torch.cuda.current_stream(dev))
+    assert dec.flags() == 0, "device flags set"
+    st = dict(zip(st, max_over_ranks(list(st.values()))))
+    from long_context_decode_mla_b200.workload import ROW_BYTES
+    lens = prob.seq_lens.long().cpu()
+    read = 0
+    for k in range(q_len):
+        Lk = (lens - (q_len - 1 - k)).clamp(min=0)
+        read += int(Lk.sum()) * ROW_BYTES[prob.kv_dtype]
     kvb = kv_bytes(prob)
-    del graph, dec
-    return {"heads": H, "q_len": q_len, "ms_per_step": round(ms, 4),
-            "value": round(kvb / (ms * 1e-3) / 1e9, 1), "unit": UNIT,
-            "query_tokens_per_s": round(B * q_len * 1e3 / ms, 1)}
+    total = read + N * (B * q_len * H * (576 * 2 + 513 * 4)) + (N + 1) * B * q_len * H * 513 * 4
+    ms = st["mean"]
+    d = leg("agentic", prob, st, world, read, total,
+            extra={"heads": H, "q_len": q_len, "rows": q_len * H,
+                   "cache_GBps": round(world * kvb / (ms * 1e-3) / 1e9, 1),
+                   "query_tokens_per_s": round(world * B * q_len * 1e3 / ms, 1),
+                   "passes_per_shard": q_len if q_len * H > 64 or prob.kv_dtype == "fp8" else 1,
+                   "steps": steps})
+    d["workload"] = (f"agentic cache, {H} heads x q_len {q_len} query tokens per request "
+                     f"(causal), {N} shards + merge")
+    del graph, dec, mq, q
+    torch.cuda.empty_cache()
+    return d
 
 
 def time_merge_heads(dec, dev, steps):
@@ -512,11 +644,16 @@ def time_merge_heads(dec, dev, steps):
         for a in bufs:
             dcpmla.dcp_exchange_free(a)
     per_rank = B * H * 513 * 4                  # its H/N heads from all N shards
-    nvlink_gbs = 770.0                          # measured peer copy, GB/s per direction
+    # an assumed link rate, not measured by this program (one GPU here): the
+    # per-direction peer-copy figure this B200 pool documents for NVLink 5
+    nvlink_gbs = 770.0
     return {"ranks": N, "us_per_rank": round(us, 2), "bytes_per_rank": per_rank,
             "GBps_local": round(per_rank / (us * 1e-6) / 1e9, 1),
             "nvlink_bound_us_per_rank": round((N - 1) / N * per_rank / (nvlink_gbs * 1e9) * 1e6,
-                                              2)}
+                                              2),
+            "nvlink_GBps_assumed": nvlink_gbs,
+            "nvlink_note": "bound at an assumed 770 GB/s per direction (the pool's documented "
+                           "peer copy), not a measurement of this run"}
 
 
 def time_append(prob, dev, steps):
@@ -565,6 +702,16 @@ def time_append(prob, dev, steps):
             "note": "one new token per request, written on its owner shard (N shard calls)"}
 
 
+def dtype_label(kv_dtype, kernel):
+    """The arithmetic of the timed path, by cache format and kernel."""
+    if kernel == "simt":
+        return f"{kv_dtype} cache decoded to f32, f32 arithmetic"
+    if kv_dtype == "fp8":
+        return ("fp8 e4m3 cache codes x e4m3 two-term Q split on the tensor cores (exact "
+                "products), fp32 accumulation; per-128 scales in fp32; P as two e4m3 terms")
+    return "bf16 cache, fp16 MMA operands, fp32 accumulation"
+
+
 def describe(name, prob):
     lens = prob.seq_lens
     return (f"{name}: batch {prob.batch}, {prob.heads} heads, {prob.kv_dtype} rows, "
@@ -591,23 +738,48 @@ def blas_threads() -> int:
         return 1
 
 
-def cpu_sample_problem(workload_name, target_len):
-    """One request of the workload's shape (same heads, row format, shards) on the CPU."""
+def cpu_info():
+    """Host cores this process may run on, the BLAS thread count and the CPU model."""
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    try:
+        cores = len(os.sched_getaffinity(0))
+    except AttributeError:
+        cores = os.cpu_count() or 1
+    return cores, blas_threads(), model
+
+
+def config_slice(workload_name):
+    """A declared slice of the workload for the CPU oracle: request 0 of the
+    seeded configuration at its own length (same heads, row format, shards;
+    for the sparse workload its index-list length), regenerated alone on the
+    host."""
     from long_context_decode_mla_b200 import workload
     cfg = workload.CONFIGS[workload_name]
-    over = dict(batch=1, seq_len=[target_len])
+    if cfg["seq_len"] == "lognormal":
+        L0 = int(workload.lognormal_lengths(cfg["batch"], cfg["seed"])[0])
+    else:
+        L0 = int(cfg["seq_len"])
+    over = dict(batch=1, seq_len=[L0])
     if cfg.get("topk"):
         over["topk"] = cfg["topk"]
-    return workload.make_problem(workload_name, **over)
+    prob = workload.make_problem(workload_name, **over)
+    desc = (f"request 0 of the {workload_name} configuration (L={L0}, {prob.heads} heads, "
+            f"{prob.kv_dtype} rows, {prob.num_shards} shards + merge"
+            + (f", top-{cfg['topk']}" if cfg.get("topk") else "") + ")")
+    return prob, desc
 
 
-def time_oracle(workload_name, seconds_budget, sample_len=None):
-    """Time the oracle on single-request samples until the budget is spent."""
-    from long_context_decode_mla_b200 import workload
-    cfg = workload.CONFIGS[workload_name]
-    if sample_len is None:
-        sample_len = 16384 if cfg["seq_len"] == "lognormal" else min(int(cfg["seq_len"]), 16384)
-    prob = cpu_sample_problem(workload_name, sample_len)
+def time_oracle(workload_name, seconds_budget):
+    """Time the oracle on the workload's declared slice until the budget is spent."""
+    prob, desc = config_slice(workload_name)
     ni = prob.numpy_inputs()
     kvb = kv_bytes(prob)
     n, t0 = 0, time.perf_counter()
@@ -617,20 +789,16 @@ def time_oracle(workload_name, seconds_budget, sample_len=None):
         el = time.perf_counter() - t0
         if el >= seconds_budget:
             break
-    return {"value": round(n * kvb / el / 1e9, 4), "unit": UNIT, "cores": blas_threads(),
-            "kind": "oracle",
-            "sample": (f"{n} x one request of the {workload_name} workload "
-                       f"(L={sample_len}, {prob.heads} heads, {prob.kv_dtype}, "
-                       f"{prob.num_shards} shards + merge), {el:.1f} s of fp64 numpy")}, el / n
+    cores, threads, model = cpu_info()
+    return {"value": round(n * kvb / el / 1e9, 4), "unit": UNIT, "cores": cores,
+            "blas_threads": threads, "cpu_model": model, "kind": "oracle",
+            "sample": f"{n} x {desc}, {el:.1f} s of fp64 numpy"}, el / n
 
 
 def run_reference(args, rank, world):
     if rank != 0:
         return None
-    from long_context_decode_mla_b200 import workload
-    cfg = workload.CONFIGS[args.workload]
-    sample_len = 16384 if cfg["seq_len"] == "lognormal" else min(int(cfg["seq_len"]), 16384)
-    prob = cpu_sample_problem(args.workload, sample_len)
+    prob, desc = config_slice(args.workload)
     ni = prob.numpy_inputs()
     kvb = kv_bytes(prob)
     for _ in range(max(3, args.warmup)):
@@ -640,19 +808,150 @@ def run_reference(args, rank, world):
         oracle_sample_step(ni, 0)
     el = time.perf_counter() - t0
     value = kvb * args.steps / el / 1e9
-    cpu = {"value": round(value, 4), "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
-           "sample": (f"each step: one request of the {args.workload} workload (L={sample_len}, "
-                      f"{prob.heads} heads, {prob.kv_dtype}, {prob.num_shards} shards + merge)")}
+    cores, threads, model = cpu_info()
+    cpu = {"value": round(value, 4), "unit": UNIT, "cores": cores, "blas_threads": threads,
+           "cpu_model": model, "kind": "oracle", "sample": f"each step: {desc}"}
     return {
         "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": UNIT,
         "n_gpus": world, "steps": args.steps, "warmup": max(3, args.warmup),
         "ms_per_step": round(1e3 * el / args.steps, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": describe(args.workload, prob) + " (one-request CPU sample)"},
+        "config": {"workload": desc + " (CPU oracle)"},
         "cpu_baseline": cpu,
         "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
+
+
+# ------------------------------------------------------------- real DCP ----
+
+def run_dcp(args, rank, world, local):
+    """The real DCP step across the GPUs of the job: one shard per rank
+    (tokens t with t mod N == rank, N = the world size), NCCL query
+    all-gather, the partial into the rank's exchange slot, a one-integer
+    all-reduce, and the head-sliced merge that pulls the peers' partials over
+    peer memory (DcpRankDecoder).  The batch is the workload's (the same on
+    every rank), so the work per step is fixed as N grows: strong scaling.
+    Steps are timed eagerly with CUDA events (NCCL is in the step), max over
+    ranks; sampled requests are checked against the oracle at the end."""
+    import datetime
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    from long_context_decode_mla_b200 import dcp_group, dcpmla, workload
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    # a one-process run (no launcher): a one-rank group on this host
+    for k, v in (("RANK", "0"), ("WORLD_SIZE", "1"), ("MASTER_ADDR", "127.0.0.1"),
+                 ("MASTER_PORT", "29511")):
+        os.environ.setdefault(k, v)
+    dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=120))
+    over = {} if args.batch is None else {"batch": args.batch}
+    prob = workload.make_problem(args.workload, num_shards=world, device=dev, kv_device=dev,
+                                 **over)
+    B, H = prob.batch, prob.heads
+    if H % world:
+        raise SystemExit(f"{H} heads do not split over {world} ranks")
+    topk = 0 if prob.sparse_idx is None else prob.sparse_idx.shape[1]
+    dec = dcp_group.DcpRankDecoder(B, H, topk=topk, impl=args.kernel)
+    h0, hn = dec.head_begin, dec.head_count
+    q_local = prob.q[:, h0:h0 + hn].contiguous()
+    table = prob.block_tables[rank].contiguous()
+
+    def step():
+        return dec.step(q_local, prob.kv_cache, prob.kv_dtype, table, prob.seq_lens,
+                        prob.softmax_scale, prob.sparse_idx)
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    try:
+        for _ in range(max(3, args.warmup)):
+            step()
+        torch.cuda.synchronize(dev)
+        dist.barrier()
+        stream = torch.cuda.current_stream(dev)
+        ev = []
+        sampler.mark(True)
+        for _ in range(args.steps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            step()
+            b.record(stream)
+            ev.append((a, b))
+        ev[-1][1].synchronize()
+        sampler.mark(False)
+        t = [a.elapsed_time(b) for a, b in ev]
+        st = {"mean": sum(t) / len(t), "median": statistics.median(t), "min": min(t),
+              "max": max(t)}
+        st = dict(zip(st, max_over_ranks(list(st.values()))))
+        flags = dec.flags()
+        # the merge alone, from the last step's slots (all complete)
+        dist.barrier()
+        parity = (dec.steps - 1) & 1
+        slots = [dec.slot(r, parity) for r in range(world)]
+        m0, m1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = 20
+        m0.record(stream)
+        for _ in range(reps):
+            dcpmla.dcp_merge_heads([x[0] for x in slots], [x[1] for x in slots], B, H, h0, hn,
+                                   dec.out, dec.out_lse)
+        m1.record(stream)
+        m1.synchronize()
+        merge_us = max_over_ranks([m0.elapsed_time(m1) * 1e3 / reps])[0]
+        # results of every rank's heads on rank 0, for the oracle check
+        outs = [torch.empty_like(dec.out) for _ in range(world)]
+        lses = [torch.empty_like(dec.out_lse) for _ in range(world)]
+        dist.all_gather(outs, dec.out)
+        dist.all_gather(lses, dec.out_lse)
+        torch.cuda.synchronize(dev)
+        dist.barrier()
+    finally:
+        sampler.stop()
+        dec.close()
+    result = None
+    if rank == 0:
+        out = torch.cat(outs, dim=1).double().cpu().numpy()
+        lse = torch.cat(lses, dim=1).double().cpu().numpy()
+        import oracle
+        ni = prob.to("cpu").numpy_inputs()
+        ids = sorted({0, B // 2, B - 1})
+        _, _, ro, rl = oracle.dcp_decode(ni["q"], ni["kv_cache"], ni["kv_dtype"],
+                                         ni["block_tables"], ni["seq_lens"], world,
+                                         ni["softmax_scale"], ni["sparse_idx"],
+                                         ni["block_size"], ids)
+        fin = np.isfinite(rl)
+        eo = float(np.abs(out[ids] - ro).max() / max(np.abs(ro).max(), 1e-30))
+        el = float(np.abs(lse[ids][fin] - rl[fin]).max()) if fin.any() else 0.0
+        kvb = kv_bytes(prob)
+        peak, peak_kind = measured_peaks()
+        ms = st["mean"]
+        result = {
+            "metric": METRIC, "value": round(kvb / (ms * 1e-3) / 1e9, 1), "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": max(3, args.warmup),
+            "ms_per_step": round(ms, 4), "ms_step_stats": ms_summary(st),
+            "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
+            "dtype": dtype_label(prob.kv_dtype, args.kernel),
+            "data": "synthetic (seeded; no public trace or checkpoint available)",
+            "config": {"workload": describe(args.workload, prob) + " (the shards on the GPUs)",
+                       "global_batch": B, "heads": H, "kv_dtype": prob.kv_dtype,
+                       "parallelism": f"DCP over {world} GPU(s): NCCL query all-gather, "
+                                      "one shard per rank, all-reduce tick, head-sliced "
+                                      "merge over peer memory",
+                       "l2": "no flush: the KV read per step is larger than 4x the 126 MB L2"},
+            "pct_hbm_peak_kv": round(100 * kvb / (ms * 1e-3) / 1e9 / world / peak, 1),
+            "nccl_ranks": world, "merge_us_per_rank": round(merge_us, 2),
+            "flags": flags,
+            "oracle_check": {"requests": ids, "max_dO_rel": eo, "max_dLSE": el},
+            "gpu_launches": args.steps * 3,
+            "clocks": sampler.summary(),
+            "e2e": None,
+            "note": "eager steps (NCCL collectives inside); e2e not measured in this mode",
+        }
+    dist.barrier()
+    dist.destroy_process_group()
+    return result
 
 
 def main():
@@ -661,6 +960,11 @@ def main():
     if args.impl == "reference":
         res = run_reference(args, rank, world)
         if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+    if args.dcp or (world > 1 and not args.replicas):
+        res = run_dcp(args, rank, world, local)
+        if rank == 0:
             print(json.dumps(res), flush=True)
         return
     res, prob = run_ours(args, rank, world, local)

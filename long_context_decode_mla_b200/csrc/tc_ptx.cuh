@@ -141,7 +141,7 @@ __device__ __forceinline__ void named_bar(int id, int threads) {
 
 // ------------------------------------------------------------------ TMA ----
 
-// 3-D tiled tensor load (no multicast) into shared memory; completion is
+// 3-D tiled tensor load into this CTA's own shared memory; completion is
 // signalled on `bar` as transaction bytes.  x is the innermost coordinate.
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* tmap, int x, int y, int z,
                                             uint64_t* bar) {
