@@ -301,6 +301,49 @@ def id_coded_rows(seq_len: int, kv_dtype: str) -> torch.Tensor:
     return rows
 
 
+def id_coded_problem_device(seq_lens, num_shards: int, kv_dtype: str, heads: int = 64,
+                            seed: int = 0, device="cuda") -> DecodeProblem:
+    """id_coded_problem built directly on a device, for full-size caches.
+
+    Same rows and placement as ``id_coded_problem`` (token t of request b at
+    block tables[t mod N, b, (t div N) div 64], row (t div N) mod 64), made
+    with vectorised tensor operations instead of per-request host copies.
+    """
+    lens = torch.as_tensor([int(x) for x in seq_lens], dtype=torch.int32)
+    tables, num_blocks = shard_block_tables(lens, num_shards, seed + 101)
+    rb = ROW_BYTES[kv_dtype]
+    dev = torch.device(device)
+    cache = torch.zeros(num_blocks, BLOCK_SIZE, rb, dtype=torch.uint8, device=dev)
+    flat = cache.view(-1, rb)
+    tab = tables.to(dev)
+    bits = torch.arange(ID_BITS, device=dev)
+    if kv_dtype == "bf16":
+        one = torch.tensor([1.0], dtype=torch.bfloat16).view(torch.uint8).to(dev)
+    else:
+        one = torch.tensor([1.0]).to(torch.float8_e4m3fn).view(torch.uint8).to(dev)
+        scales = torch.tensor([1.0] * 4, dtype=torch.float32).view(torch.uint8).to(dev)
+    chunk = 1 << 20
+    for b, L in enumerate(lens.tolist()):
+        for t0 in range(0, L, chunk):
+            t = torch.arange(t0, min(L, t0 + chunk), device=dev)
+            s, j = t % num_shards, t // num_shards
+            blk = tab[s, b, j // BLOCK_SIZE].long()
+            dst = blk * BLOCK_SIZE + (j % BLOCK_SIZE)
+            on = ((t[:, None] >> bits[None, :]) & 1).bool()
+            rows = torch.zeros(t.numel(), rb, dtype=torch.uint8, device=dev)
+            if kv_dtype == "bf16":
+                for d in range(ID_BITS):
+                    rows[on[:, d], 2 * d:2 * d + 2] = one
+            else:
+                rows[:, 512:528] = scales
+                for d in range(ID_BITS):
+                    rows[on[:, d], d] = one[0]
+            flat[dst] = rows
+    q = torch.zeros(len(lens), heads, ROW_DIM, dtype=torch.bfloat16, device=dev)
+    return DecodeProblem(q, cache, kv_dtype, tab, lens.to(dev), num_shards,
+                         meta=dict(name="id_coded"))
+
+
 def id_coded_problem(seq_lens, num_shards: int, kv_dtype: str, heads: int = 8, seed: int = 0,
                      sparse_idx=None) -> DecodeProblem:
     """Cache whose row for global token t carries t in binary (exact addressing tests).
