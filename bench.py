@@ -117,10 +117,11 @@ def measured_peaks():
     return 6650.0, "fallback"
 
 
-# the translation unit of the partial kernel (whose DRAM traffic
+# the translation unit of the fp8 partial kernel (whose DRAM traffic
 # profiles/traffic.json records) and the headers it includes; other files are
 # compiled separately and cannot change that kernel
-PARTIAL_KERNEL_SOURCES = ("common.cuh", "kernels.h", "partial_tc.cu", "tc_ptx.cuh")
+PARTIAL_KERNEL_SOURCES = ("common.cuh", "kernels.h", "partial_f8.cu", "schedule.cuh",
+                          "tc_ptx.cuh")
 
 
 def _code_only(text: str) -> str:

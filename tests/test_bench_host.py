@@ -127,7 +127,7 @@ def test_traffic_key_ignores_comments_but_not_code():
     def read(name, edit=None):
         with open(os.path.join(csrc, name), encoding="utf-8") as f:
             text = f.read()
-        return edit(text) if edit and name == "partial_tc.cu" else text
+        return edit(text) if edit and name == "partial_f8.cu" else text
 
     base = bench.kernel_source_hash(read)
     assert base == bench.kernel_source_hash()
