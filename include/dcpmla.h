@@ -379,6 +379,82 @@ int mla_kv_append(const void* latent, const void* rope, int num_tokens, const in
                   int batch, int shard_id, int num_shards, void* kv_cache, int kv_dtype,
                   int64_t num_blocks, int block_size, int32_t* flags, void* stream);
 
+/*
+ * Prefill context parallelism (PCP) over the DCP-sharded cache.
+ *
+ * "How vLLM Serves GLM-5.3 with Million-Token Contexts on 16 H200s",
+ * section "The core design": PCP splits a prompt's query tokens over P
+ * ranks, each computing all heads of its tokens; the prompt is cut into 2P
+ * chunks and rank r takes a front chunk and the matching back chunk (16
+ * chunks for 8 ranks) so that causal work evens out; the cache stays
+ * distributed round-robin over the DCP shards, so prefill gathers the
+ * layer's distributed rows, attends, and drops the gathered copy.
+ * Readings (the page gives no chunk-size rule or attention form): chunks are
+ * contiguous in prompt order, the first T mod 2P one token longer; rank r
+ * owns chunks r and 2P - 1 - r, its queries in that order; attention is the
+ * absorbed form of the decode path (query token i attends to every prompt
+ * token t <= i, scores over 576 values, values the first 512, natural-log
+ * LSE); the prompt's rows are in the cache before its attention.
+ */
+
+/*
+ * The query tokens of PCP rank `rank` of `pcp_size` for a `num_tokens`-token
+ * prompt: chunk rank, then chunk 2 * pcp_size - 1 - rank.  Host only.
+ *   tokens   NULL (only *count is set) or room for `capacity` int32.
+ *   count    receives the number of tokens.
+ * Returns DCPMLA_OK, or DCPMLA_ERR_INVALID_ARGUMENT (bad sizes, rank out of
+ * range, capacity too small).
+ */
+int pcp_rank_tokens(int num_tokens, int pcp_size, int rank, int32_t* tokens, int capacity,
+                    int* count);
+
+/* Bytes of a gathered prompt of `num_tokens` rows: whole 64-row blocks. */
+size_t pcp_gathered_bytes(int num_tokens, int kv_dtype);
+
+/*
+ * Gather one request's prompt rows from the DCP-sharded cache into token
+ * order: row t of `gathered` is token t, read from shard t mod num_shards at
+ * local row t div num_shards through that shard's table row.
+ *   kv_cache      [num_blocks][64][row bytes], 16-byte aligned.
+ *   block_tables  DEVICE [num_shards][block_table_stride] int32: each shard's
+ *                 table row for the request.
+ *   gathered      DEVICE, 16-byte aligned, at least
+ *                 pcp_gathered_bytes(num_tokens, kv_dtype) bytes ([blocks][64]
+ *                 [row bytes]; rows past num_tokens are not written).
+ *   flags         NULL or a DEVICE int32: DCPMLA_FLAG_BAD_BLOCK for a table
+ *                 entry outside the pool, DCPMLA_FLAG_BAD_LENGTH for a local
+ *                 row beyond the table row; such rows are written as zeros.
+ * Returns DCPMLA_OK or a negative code (host checks before any launch).
+ */
+int pcp_gather_rows(const void* kv_cache, int kv_dtype, int64_t num_blocks, int block_size,
+                    const int32_t* block_tables, int block_table_stride, int num_shards,
+                    int num_tokens, void* gathered, size_t gathered_bytes, int32_t* flags,
+                    void* stream);
+
+/*
+ * Causal prefill attention of one rank's query tokens over a gathered
+ * prompt: query b (all num_heads heads) at prompt position positions[b]
+ * attends to gathered rows 0..positions[b].
+ *   q             [num_queries][num_heads][576] bf16, 16-byte aligned.
+ *   positions     DEVICE [num_queries] int32 prompt positions (< the prompt
+ *                 length; a negative one is flagged, DCPMLA_FLAG_BAD_LENGTH).
+ *   gathered      the pcp_gather_rows output, num_gathered_blocks blocks.
+ *   out, out_lse  [num_queries][num_heads][512] and [num_queries][num_heads]
+ *                 fp32.
+ *   workspace     mla_decode_workspace_size(num_queries, num_heads,
+ *                 num_splits, 0) bytes.
+ *   impl          as mla_decode_partial: fp8 rows run on the e4m3-direct
+ *                 kernel (exact scores), bf16 rows on the fp16-operand kernel.
+ * Each query reads its prefix of the gathered rows: the prompt (at most about
+ * 190K fp8 rows fit the 126 MB L2) is read once from HBM and its blocks are
+ * shared by the queries through L2.  Returns as mla_decode_partial.
+ */
+int pcp_prefill_attention(const void* q, const int32_t* positions, int num_queries,
+                          int num_heads, const void* gathered, int kv_dtype,
+                          int64_t num_gathered_blocks, float softmax_scale, float* out,
+                          float* out_lse, void* workspace, size_t workspace_bytes,
+                          int num_splits, int impl, void* stream);
+
 /* Static description of a return code (never NULL). */
 const char* dcpmla_error_string(int code);
 

@@ -30,7 +30,8 @@ struct PartialParams {
                               // multi-query: query-major rows (query i, head h)
   const uint8_t* kv;          // [num_blocks][64][row_bytes]
   long long num_blocks;
-  const int* block_table;     // [B][bt_stride] this shard's table
+  const int* block_table;     // [B][bt_stride] this shard's table; nullptr: the pool's
+                              // blocks in order for every request (a gathered prompt)
   int bt_stride;
   const int* seq_lens;        // [B] global lengths
   int batch;
@@ -47,8 +48,9 @@ struct PartialParams {
   float* out_lse;             // [B][rows_o]
   int rows_q;                 // rows between consecutive requests in q (>= heads)
   int rows_o;                 // rows between consecutive requests in out / out_lse
-  int len_delta;              // subtracted from every valid length (a query pass that
-                              // sits len_delta tokens before the request's end)
+  int len_delta;              // subtracted from every valid length: a multi-query pass
+                              // that ends len_delta tokens before the request's end; -1
+                              // for prefill queries, whose "length" is their position
   int* flags;                 // workspace flag word
   float* ws_o;                // [slots][H][512]
   float* ws_lse;              // [slots][H]
@@ -192,7 +194,7 @@ __device__ __forceinline__ void for_each_dense_segment(const PartialParams& p, i
 // Physical block of local tile `tile` of request b, or -1 (flagged) if the
 // table entry is outside the pool.
 __device__ __forceinline__ int tile_block(const PartialParams& p, int b, int tile) {
-  int blk = __ldg(p.block_table + (size_t)b * p.bt_stride + tile);
+  int blk = p.block_table ? __ldg(p.block_table + (size_t)b * p.bt_stride + tile) : tile;
   if (blk < 0 || (long long)blk >= p.num_blocks) {
     if (p.flags) atomicOr(p.flags, kFlagBadBlock);
     return -1;

@@ -3,6 +3,7 @@
 #include "dcpmla.h"
 
 #include <atomic>
+#include <climits>
 #include <cmath>
 #include <cstdint>
 
@@ -119,7 +120,7 @@ int decode_partial(const void* q, const void* kv_cache, int kv_dtype, int64_t nu
                    int num_shards, const int32_t* sparse_idx, int topk, float softmax_scale,
                    float* out_partial, float* out_lse, void* workspace, size_t workspace_bytes,
                    int num_splits, int impl, void* stream, int rows_q, int rows_o,
-                   int len_delta) {
+                   int len_delta, bool identity_table = false) {
   // ---- scalar checks (fail closed, nothing launched on error) ----
   const bool withhold = (impl & DCPMLA_TEST_WITHHOLD_ARRIVAL) != 0;
   impl &= ~DCPMLA_TEST_WITHHOLD_ARRIVAL;
@@ -135,7 +136,8 @@ int decode_partial(const void* q, const void* kv_cache, int kv_dtype, int64_t nu
     return DCPMLA_ERR_INVALID_ARGUMENT;
   if (num_heads > kMaxHeads || block_size != kBlock) return DCPMLA_ERR_UNSUPPORTED;
   if (batch == 0) return DCPMLA_OK;
-  if (!q || !kv_cache || !block_table || !seq_lens || !out_partial || !out_lse)
+  if (!q || !kv_cache || (!block_table && !identity_table) || !seq_lens || !out_partial ||
+      !out_lse)
     return DCPMLA_ERR_INVALID_ARGUMENT;
   if (!aligned16(q) || !aligned16(kv_cache) || !aligned16(out_partial) ||
       (workspace && !aligned16(workspace)))
@@ -153,7 +155,7 @@ int decode_partial(const void* q, const void* kv_cache, int kv_dtype, int64_t nu
   p.q = static_cast<const __nv_bfloat16*>(q);
   p.kv = static_cast<const uint8_t*>(kv_cache);
   p.num_blocks = num_blocks;
-  p.block_table = block_table;
+  p.block_table = identity_table ? nullptr : block_table;
   p.bt_stride = block_table_stride;
   p.seq_lens = seq_lens;
   p.batch = batch;
@@ -264,6 +266,23 @@ int mla_decode_partial_multi(const void* q, const void* kv_cache, int kv_dtype,
     if (rc != DCPMLA_OK) return rc;
   }
   return DCPMLA_OK;
+}
+
+int pcp_prefill_attention(const void* q, const int32_t* positions, int num_queries,
+                          int num_heads, const void* gathered, int kv_dtype,
+                          int64_t num_gathered_blocks, float softmax_scale, float* out,
+                          float* out_lse, void* workspace, size_t workspace_bytes,
+                          int num_splits, int impl, void* stream) {
+  // Query token b at prompt position positions[b] attends causally to the
+  // gathered rows 0..positions[b]: a decode over the gathered prompt (its
+  // blocks in order, one shard) of length positions[b] + 1.
+  if (num_queries < 0 || num_gathered_blocks < 1 || num_gathered_blocks > INT32_MAX)
+    return DCPMLA_ERR_INVALID_ARGUMENT;
+  if (!positions && num_queries > 0) return DCPMLA_ERR_INVALID_ARGUMENT;
+  return decode_partial(q, gathered, kv_dtype, num_gathered_blocks, kBlock, nullptr,
+                        (int)num_gathered_blocks, positions, num_queries, num_heads, 1, 0, 1,
+                        nullptr, 0, softmax_scale, out, out_lse, workspace, workspace_bytes,
+                        num_splits, impl, stream, num_heads, num_heads, -1, true);
 }
 
 int dcp_merge(const float* partials, const float* lses, int num_shards, int batch,

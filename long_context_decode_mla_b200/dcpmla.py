@@ -73,6 +73,15 @@ def lib() -> ctypes.CDLL:
     L.dcp_exchange_close.restype = i32
     L.dcp_exchange_free.argtypes = [vp]
     L.dcp_exchange_free.restype = i32
+    L.pcp_rank_tokens.argtypes = [i32, i32, i32, vp, i32, ctypes.POINTER(i32)]
+    L.pcp_rank_tokens.restype = i32
+    L.pcp_gathered_bytes.argtypes = [i32, i32]
+    L.pcp_gathered_bytes.restype = sz
+    L.pcp_gather_rows.argtypes = [vp, i32, i64, i32, vp, i32, i32, i32, vp, sz, vp, vp]
+    L.pcp_gather_rows.restype = i32
+    L.pcp_prefill_attention.argtypes = [vp, vp, i32, i32, vp, i32, i64, f32, vp, vp, vp, sz, i32,
+                                        i32, vp]
+    L.pcp_prefill_attention.restype = i32
     _lib = L
     return L
 
@@ -268,6 +277,98 @@ def dcp_exchange_close(address: int) -> None:
 
 def dcp_exchange_free(address: int) -> None:
     _check(lib().dcp_exchange_free(ctypes.c_void_p(address)), "dcp_exchange_free")
+
+
+def pcp_rank_tokens(num_tokens: int, pcp_size: int, rank: int) -> list[int]:
+    """Prompt positions of PCP rank ``rank``'s query tokens (see include/dcpmla.h)."""
+    n = ctypes.c_int(0)
+    _check(lib().pcp_rank_tokens(num_tokens, pcp_size, rank, None, 0, ctypes.byref(n)),
+           "pcp_rank_tokens")
+    buf = (ctypes.c_int32 * max(1, n.value))()
+    _check(lib().pcp_rank_tokens(num_tokens, pcp_size, rank, buf, n.value, ctypes.byref(n)),
+           "pcp_rank_tokens")
+    return list(buf)[:n.value]
+
+
+def pcp_gathered_bytes(num_tokens: int, kv_dtype) -> int:
+    kvd = KV_DTYPES[kv_dtype] if isinstance(kv_dtype, str) else int(kv_dtype)
+    return int(lib().pcp_gathered_bytes(num_tokens, kvd))
+
+
+def pcp_gather_rows(kv_cache, kv_dtype, block_tables, num_tokens, gathered, flags=None,
+                    stream=None, block_size: int = BLOCK_SIZE, num_blocks: int | None = None):
+    """One request's prompt rows in token order: block_tables [N, stride] (each shard's
+    table row for the request) -> gathered (uint8, pcp_gathered_bytes)."""
+    kvd = KV_DTYPES[kv_dtype] if isinstance(kv_dtype, str) else int(kv_dtype)
+    nb = kv_cache.shape[0] if num_blocks is None else num_blocks
+    nbytes = gathered.numel() * gathered.element_size()
+    rc = lib().pcp_gather_rows(_ptr(kv_cache), kvd, nb, block_size, _ptr(block_tables),
+                               block_tables.shape[-1], block_tables.shape[0], num_tokens,
+                               _ptr(gathered), nbytes, None if flags is None else _ptr(flags),
+                               _stream(stream))
+    _check(rc, "pcp_gather_rows")
+
+
+def pcp_prefill_attention(q, positions, gathered, kv_dtype, softmax_scale, out, out_lse,
+                          workspace, num_splits: int = 0, impl: str | int = "auto", stream=None,
+                          num_gathered_blocks: int | None = None):
+    """Causal attention of query tokens q [n, H, 576] at ``positions`` [n] over a
+    gathered prompt (see include/dcpmla.h)."""
+    kvd = KV_DTYPES[kv_dtype] if isinstance(kv_dtype, str) else int(kv_dtype)
+    rb = 656 if kvd == KV_DTYPES["fp8"] else 1152
+    nblk = (gathered.numel() * gathered.element_size() // (BLOCK_SIZE * rb)
+            if num_gathered_blocks is None else num_gathered_blocks)
+    impl_code = IMPLS[impl] if isinstance(impl, str) else int(impl)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    rc = lib().pcp_prefill_attention(_ptr(q), _ptr(positions), q.shape[0], q.shape[1],
+                                     _ptr(gathered), kvd, nblk, float(softmax_scale), _ptr(out),
+                                     _ptr(out_lse), _ptr(workspace), ws_bytes, num_splits,
+                                     impl_code, _stream(stream))
+    _check(rc, "pcp_prefill_attention")
+
+
+class PcpPrefill:
+    """One request's PCP prefill on one GPU: the gathered copy of its prompt
+    rows and each rank's causal attention over it (the ranks of a real PCP
+    group would each hold the gathered copy; here they run in turn)."""
+
+    def __init__(self, num_tokens: int, num_heads: int, pcp_size: int, kv_dtype: str,
+                 device="cuda", num_splits: int = 0, impl: str = "auto"):
+        self.num_tokens, self.num_heads, self.pcp_size = num_tokens, num_heads, pcp_size
+        self.kv_dtype, self.num_splits, self.impl = kv_dtype, num_splits, impl
+        dev = torch.device(device)
+        self.gathered = torch.empty(max(16, pcp_gathered_bytes(num_tokens, kv_dtype)),
+                                    dtype=torch.uint8, device=dev)
+        self.flags = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.tokens = [torch.tensor(pcp_rank_tokens(num_tokens, pcp_size, r), dtype=torch.int32,
+                                    device=dev) for r in range(pcp_size)]
+        most = max(int(t.numel()) for t in self.tokens)
+        self.workspace = torch.zeros(mla_decode_workspace_size(max(1, most), num_heads,
+                                                               num_splits), dtype=torch.uint8,
+                                     device=dev)
+        self.out = [torch.empty(int(t.numel()), num_heads, V_DIM, device=dev)
+                    for t in self.tokens]
+        self.out_lse = [torch.empty(int(t.numel()), num_heads, device=dev) for t in self.tokens]
+        self._q = [None] * pcp_size
+
+    def gather(self, kv_cache, block_tables, stream=None):
+        """block_tables [N, stride]: each DCP shard's table row for the request."""
+        pcp_gather_rows(kv_cache, self.kv_dtype, block_tables, self.num_tokens, self.gathered,
+                        self.flags, stream)
+
+    def attend(self, q_prompt, softmax_scale, stream=None):
+        """q_prompt [T, H, 576] bf16 (every prompt token's query); every rank's
+        share.  Results in ``out[r]`` / ``out_lse[r]``, rows in ``tokens[r]`` order."""
+        for r in range(self.pcp_size):
+            if self.tokens[r].numel() == 0:
+                continue
+            if self._q[r] is None or self._q[r].shape[1] != q_prompt.shape[1]:
+                self._q[r] = torch.empty(self.tokens[r].numel(), q_prompt.shape[1], HEAD_DIM,
+                                         dtype=torch.bfloat16, device=q_prompt.device)
+            torch.index_select(q_prompt, 0, self.tokens[r].long(), out=self._q[r])
+            pcp_prefill_attention(self._q[r], self.tokens[r], self.gathered, self.kv_dtype,
+                                  softmax_scale, self.out[r], self.out_lse[r], self.workspace,
+                                  self.num_splits, self.impl, stream)
 
 
 def check_inputs(block_tables, seq_lens, num_blocks: int, num_shards: int,
