@@ -389,6 +389,7 @@ def run_ours(args, rank, world, local):
                 "million": lambda: time_million_layers(dev, rank, world, args,
                                                        layers=args.million_layers)}
         extras["configs"] = {k: f() for k, f in legs.items()}
+        extras["pcp_prefill"] = time_pcp_prefill(dev, args)
     if prob.sparse_idx is None and not args.no_extras:
         extras["multi_query"] = time_multi_query(prob, dev, args, q_len=4, world=world)
     extras["kv_append"] = time_append(prob, dev, max(20, args.steps // 4))
@@ -592,6 +593,70 @@ def time_multi_query(prob, dev, args, q_len, world=1):
     del graph, dec, mq, q
     torch.cuda.empty_cache()
     return d
+
+
+def time_pcp_prefill(dev, args, num_tokens=16384, pcp_size=8, num_shards=8, heads=64):
+    """PCP prefill of one prompt on one GPU: the gather of its rows from the
+    DCP-sharded cache and every rank's causal attention (the P ranks in turn;
+    on a real PCP group each rank runs its share on its own GPU), graph-
+    replayed.  Roofline: tensor.  Flops per prompt = sum over query tokens i
+    of (i + 1) rows x heads x (576 + 512) x 2; the peak is fp8 dense taken as
+    2x the measured bf16 GEMM rate, else 2x the recipe's 1.59 PFLOP/s."""
+    import torch
+    from long_context_decode_mla_b200 import dcpmla, workload
+    prob = workload.make_problem("agentic", num_shards=num_shards, batch=1, heads=heads,
+                                 seq_len=[num_tokens], device=dev, kv_device=dev, seed=2024)
+    q = workload.random_q(num_tokens, heads, 2025).to(dev)
+    pre = dcpmla.PcpPrefill(num_tokens, heads, pcp_size, "fp8", device=dev, impl=args.kernel)
+    tables = prob.block_tables[:, 0].contiguous()
+
+    def run(stream):
+        pre.gather(prob.kv_cache, tables, stream)
+        pre.attend(q, prob.softmax_scale, stream)
+
+    side = torch.cuda.Stream(device=dev)
+    side.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(side):
+        run(side)
+    torch.cuda.current_stream(dev).wait_stream(side)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=side):
+        run(side)
+    for _ in range(2):
+        graph.replay()
+    torch.cuda.synchronize(dev)
+    steps = max(3, args.steps // 10)
+    st = replay_stats(graph, steps, torch.cuda.current_stream(dev))
+    assert int(pre.flags.item()) == 0 and all(
+        torch.isfinite(x).all() for x in pre.out_lse), "PCP prefill flags or non-finite LSE"
+    flops = sum((i + 1) for i in range(num_tokens)) * heads * (576 + 512) * 2
+    peak_bf16, kind = measured_tensor_peak()
+    peak = 2 * peak_bf16
+    ms = st["mean"]
+    tflops = flops / (ms * 1e-3) / 1e12
+    d = {"workload": f"one {num_tokens}-token prompt, {heads} heads, fp8 rows on {num_shards} "
+                     f"DCP shards, PCP over {pcp_size} ranks (16 chunks for 8), gather + causal "
+                     "attention of every rank", "ms_per_prompt": ms_summary(st),
+         "prefill_tokens_per_s": round(num_tokens * 1e3 / ms, 1),
+         "roofline": {"bound": "tensor", "achieved": round(tflops, 1), "unit": "TFLOP/s",
+                      "peak": round(peak, 1), "frac": round(tflops / peak, 4),
+                      "peak_source": f"fp8 = 2 x bf16 ({kind})"},
+         "gathered_bytes": num_tokens * 656, "steps": steps}
+    del graph, pre, prob, q
+    torch.cuda.empty_cache()
+    return d
+
+
+def measured_tensor_peak():
+    """Dense bf16 tensor peak (TFLOP/s) from MEASURED_PEAKS.json, else the fallback."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        v = d.get("bf16_tflops")
+        if v:
+            return float(v), "measured"
+    return 1590.0, "fallback"
 
 
 def time_merge_heads(dec, dev, steps):
