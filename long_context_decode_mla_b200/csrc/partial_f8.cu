@@ -334,27 +334,38 @@ __device__ __forceinline__ void qk_role(int side, const PartialParams& p, F8Ctl&
   while (true) {
     const uint32_t cs = tau % kCodeStages, rs = tau % kRopeStages;
     if (cur.t == 0 && !wait_or_abort(&c.q_full, sigma & 1, c)) return;
-    // the tile's bytes and scales are staged; and stay at most one tile
-    // ahead of PV: the scores of tile tau are issued once the PV of tile
-    // tau - 2 is done (the release of its code slot, a barrier that cannot
-    // complete its next phase before these scores), so that a PV never
-    // waits behind score MMAs of tiles far ahead
-    const uint32_t tp = tau - 2;
-    uint64_t* thr = tau >= 2 ? &c.code_empty[tp % kCodeStages] : &c.staged[cs];
-    const uint32_t thr_par = tau >= 2 ? (tp / kCodeStages) & 1 : (tau / kCodeStages) & 1;
-    if (!ptx::mbar_wait3(&c.staged[cs], (tau / kCodeStages) & 1, thr, thr_par, thr, thr_par,
-                         &c.abort))
-      return;
+    // One shared-memory round trip tests every barrier the tile's parts
+    // need, then its MMAs issue back to back:
+    //  * the tile's bytes have landed (the scores need neither the staged
+    //    scales nor the clearing of rows past the end: those rows' scores
+    //    are masked, and PV, which does need the clearing, runs after the
+    //    softmax has waited for it);
+    //  * the PV of tile tau - 2 is done (the release of its code slot, a
+    //    barrier that cannot complete its next phase before these scores),
+    //    so that a PV never waits behind score MMAs of tiles far ahead;
+    //  * each part's buffer is free (part number n reuses the buffer of
+    //    part n - 8, released by the softmax).
+    uint64_t* bars[5];
+    uint32_t pars[5];
+    bars[0] = &c.full[cs];
+    pars[0] = (tau / kCodeStages) & 1;
+    bars[1] = tau >= 2 ? &c.code_empty[(tau - 2) % kCodeStages] : bars[0];
+    pars[1] = tau >= 2 ? ((tau - 2) / kCodeStages) & 1 : pars[0];
+#pragma unroll
+    for (int k = 0; k < 3; ++k) {
+      const int part = side + 2 * (k < nparts ? k : nparts - 1);
+      const uint32_t pi = 5 * tau + part;
+      bars[2 + k] = pi >= (uint32_t)kParts ? &c.part_empty[pi % kParts] : bars[0];
+      pars[2 + k] = pi >= (uint32_t)kParts ? ((pi / kParts) + 1) & 1 : pars[0];
+    }
+    if (!ptx::mbar_wait5(bars, pars, &c.abort)) return;
+    ptx::tc_fence_after();
     if (side == 0) F8_TRACE(1, tau);
     const uint64_t dcode = dplus(dc0, cs * kCodeStage), drope = dplus(dr0, rs * kChunk);
 #pragma unroll 1
     for (int k = 0; k < nparts; ++k) {
       const int part = side + 2 * k;
       const uint32_t pi = 5 * tau + part, buf = pi % kParts;
-      if (pi >= (uint32_t)kParts &&
-          !wait_or_abort(&c.part_empty[buf], ((pi / kParts) + 1) & 1, c))
-        return;
-      ptx::tc_fence_after();
       F8_TRACE(12, pi);
       const uint32_t d = c.tmem_base + kColPart + 32 * buf;
       if (part < 4) {
@@ -526,6 +537,7 @@ __device__ __forceinline__ void staging_role(const PartialParams& p, F8Ctl& c, u
       ++sigma;
     }
     if (!wait_or_abort(&c.full[cs], (tau / kCodeStages) & 1, c)) return;
+    if (u == 0) F8_TRACE(20, tau);
     // buffer b was last read by the softmax of tile tau - 2
     if (tau >= 2 && !wait_or_abort(&c.sc_empty[b], ((tau / 2) + 1) & 1, c)) return;
     const int nv = c.nv[cs];
@@ -582,6 +594,7 @@ __device__ __forceinline__ void staging_role(const PartialParams& p, F8Ctl& c, u
       ptx::fence_proxy_async();
     }
     warp_arrive(&c.staged[cs]);
+    if (u == 0) F8_TRACE(21, tau);
     ++tau;
     if (!cur.next(p, c)) break;
   }
