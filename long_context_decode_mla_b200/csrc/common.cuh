@@ -30,9 +30,11 @@ struct PartialParams {
                               // multi-query: query-major rows (query i, head h)
   const uint8_t* kv;          // [num_blocks][64][row_bytes]
   long long num_blocks;
-  const int* block_table;     // [B][bt_stride] this shard's table; nullptr: the pool's
-                              // blocks in order for every request (a gathered prompt)
+  const int* block_table;     // [B][bt_stride] this shard's table; nullptr: request b's
+                              // tile k is block b * id_stride + k of the pool (rows that
+                              // were gathered in order: a prompt, or sparse selections)
   int bt_stride;
+  int id_stride;
   const int* seq_lens;        // [B] global lengths
   int batch;
   int heads;                  // rows per request in this pass: query heads x q_len (<= 64)
@@ -56,6 +58,7 @@ struct PartialParams {
   float* ws_lse;              // [slots][H]
   int* ws_list;               // sparse mode: per-CTA lists of selected local rows
   int num_ctas;               // G: CTAs sharing the dense tile space
+  int per_request_ctas;       // 1: CTA b takes request b whole (grid = batch, no splits)
   int test_withhold;          // test only: converters skip their first arrival (timeout path)
 };
 
@@ -141,6 +144,35 @@ __device__ __forceinline__ int total_tiles(const PartialParams& p, int* warp_sum
   return acc;
 }
 
+// Per-request schedule: the tile range [lo, hi) of request blockIdx.x in the
+// request-major tile order (all threads of the block call it).
+__device__ __forceinline__ void request_tile_range(const PartialParams& p, int* warp_sums,
+                                                   int* lo, int* hi) {
+  int acc = 0, mine_lo = 0, mine_n = 0;
+  for (int base = 0; base < p.batch; base += blockDim.x) {
+    const int b = base + threadIdx.x;
+    int n, nt = 0;
+    if (b < p.batch) nt = request_tiles(p, b, &n);
+    int tot;
+    const int pre = acc + block_exclusive_scan(nt, warp_sums, &tot);
+    if (b == (int)blockIdx.x) {
+      mine_lo = pre;
+      mine_n = nt;
+    }
+    acc += tot;
+  }
+  __syncthreads();
+  // broadcast from the thread that saw request blockIdx.x
+  __shared__ int range[2];
+  if (threadIdx.x == (int)(blockIdx.x % blockDim.x)) {
+    range[0] = mine_lo;
+    range[1] = mine_lo + mine_n;
+  }
+  __syncthreads();
+  *lo = range[0];
+  *hi = range[1];
+}
+
 struct Segment {
   int b;          // request
   int t0, t1;     // tile range within the request
@@ -194,7 +226,8 @@ __device__ __forceinline__ void for_each_dense_segment(const PartialParams& p, i
 // Physical block of local tile `tile` of request b, or -1 (flagged) if the
 // table entry is outside the pool.
 __device__ __forceinline__ int tile_block(const PartialParams& p, int b, int tile) {
-  int blk = p.block_table ? __ldg(p.block_table + (size_t)b * p.bt_stride + tile) : tile;
+  int blk = p.block_table ? __ldg(p.block_table + (size_t)b * p.bt_stride + tile)
+                          : b * p.id_stride + tile;
   if (blk < 0 || (long long)blk >= p.num_blocks) {
     if (p.flags) atomicOr(p.flags, kFlagBadBlock);
     return -1;

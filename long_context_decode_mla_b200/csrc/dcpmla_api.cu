@@ -68,6 +68,26 @@ long long list_ints_for(int batch, int topk, int ctas) {
   return (long long)batch * parts * chunk;
 }
 
+// Sparse decode on the tensor-core kernels runs over gathered rows: room for
+// every request's selections in whole 64-row blocks (rows sized for bf16, so
+// that one size serves both formats) and for the per-request counts.
+long long sparse_maxblk(int topk) { return (topk + kBlock - 1) / kBlock; }
+size_t round256(size_t x) { return (x + 255) & ~(size_t)255; }
+size_t sparse_gather_rows_bytes(int batch, int topk) {
+  return round256((size_t)batch * sparse_maxblk(topk) * kBlock * kRowBytesBf16);
+}
+
+// Workspace of one call: dense decode needs split slots; sparse decode needs
+// either the CUDA-core kernel's layout (a slot and a list chunk per CTA) or the
+// gathered rows with dense split slots, whichever is larger.
+size_t ws_bytes_for(int batch, int heads, int topk, int ctas) {
+  const size_t dense = ws_total((long long)ctas + batch, heads);
+  if (topk <= 0) return dense;
+  const size_t simt = ws_total(slots_for(batch, topk, ctas), heads, list_ints_for(batch, topk, ctas));
+  const size_t gathered = dense + sparse_gather_rows_bytes(batch, topk) + round256((size_t)batch * 4);
+  return simt > gathered ? simt : gathered;
+}
+
 }  // namespace
 }  // namespace dcpmla
 
@@ -101,7 +121,7 @@ int mla_decode_workspace_size(int batch, int num_heads, int num_splits, int topk
   int ctas = 0;
   int rc = resolve_ctas(num_splits, &ctas);
   if (rc != DCPMLA_OK) return rc;
-  *bytes = ws_total(slots_for(batch, topk, ctas), num_heads, list_ints_for(batch, topk, ctas));
+  *bytes = ws_bytes_for(batch, num_heads, topk, ctas);
   return DCPMLA_OK;
 }
 
@@ -148,7 +168,7 @@ int decode_partial(const void* q, const void* kv_cache, int kv_dtype, int64_t nu
   if (rc != DCPMLA_OK) return rc;
   const long long slots = slots_for(batch, eff_topk, ctas);
   const long long list_ints = list_ints_for(batch, eff_topk, ctas);
-  if (!workspace || workspace_bytes < ws_total(slots, num_heads, list_ints))
+  if (!workspace || workspace_bytes < ws_bytes_for(batch, num_heads, eff_topk, ctas))
     return DCPMLA_ERR_WORKSPACE;
 
   PartialParams p{};
@@ -180,8 +200,44 @@ int decode_partial(const void* q, const void* kv_cache, int kv_dtype, int64_t nu
   p.num_ctas = ctas;
   p.test_withhold = withhold ? 1 : 0;
 
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // Sparse decode on the tensor cores: localise and gather the selected rows,
+  // then decode densely over them (one shard of gathered rows, identity
+  // tables), so that fp8 rows reach the exact e4m3 kernel.  The CUDA-core
+  // kernel and the fp16-operand kernel (DCPMLA_IMPL_TC_F16) keep their own
+  // in-kernel selection.
+  const bool gathered_sparse =
+      p.sparse_idx && impl != DCPMLA_IMPL_SIMT && impl != DCPMLA_IMPL_TC_F16;
+  if (gathered_sparse) {
+    const int rb = kv_dtype == DCPMLA_KV_BF16 ? kRowBytesBf16 : kRowBytesFp8;
+    const int maxblk = (int)sparse_maxblk(eff_topk);
+    uint8_t* gathered = ws + ws_total((long long)ctas + batch, num_heads);
+    int* counts = reinterpret_cast<int*>(gathered + sparse_gather_rows_bytes(batch, eff_topk));
+    if (launch_sparse_gather(p, rb, maxblk, gathered, counts, st) != cudaSuccess)
+      return DCPMLA_ERR_CUDA;
+    p.kv = gathered;
+    p.num_blocks = (long long)batch * maxblk;
+    p.block_table = nullptr;
+    p.id_stride = maxblk;
+    p.bt_stride = maxblk;
+    p.seq_lens = counts;
+    p.shard = 0;
+    p.nshards = 1;
+    p.sparse_idx = nullptr;
+    p.topk = 0;
+    p.sparse_parts = 1;
+    p.ws_o = reinterpret_cast<float*>(ws + ws_o_offset());
+    p.ws_lse = reinterpret_cast<float*>(ws + ws_lse_offset((long long)ctas + batch, num_heads));
+    p.ws_list = nullptr;
+  }
   const bool tc_ok = tc_supports(p, kv_dtype);
   const bool f8_ok = f8_supports(p, kv_dtype);
+  if (gathered_sparse && f8_ok) {
+    // a request's selections are a few tiles: one CTA per request keeps each
+    // request whole (one Q image, one epilogue, nothing to combine)
+    p.per_request_ctas = 1;
+    p.num_ctas = batch;
+  }
   enum { kSimt, kTc16, kTc8 } which;
   if (impl == DCPMLA_IMPL_SIMT) {
     which = kSimt;
@@ -199,7 +255,6 @@ int decode_partial(const void* q, const void* kv_cache, int kv_dtype, int64_t nu
   }
   if (q_len > 1 && which == kSimt) return DCPMLA_ERR_UNSUPPORTED;   // causal rows: tensor cores only
 
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e = which == kTc8    ? launch_partial_f8(p, st)
                   : which == kTc16 ? launch_partial_tc(p, kv_dtype, st)
                                    : launch_partial_simt(p, kv_dtype, st);

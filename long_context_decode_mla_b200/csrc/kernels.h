@@ -16,5 +16,7 @@ cudaError_t launch_split_combine(const PartialParams& p, cudaStream_t st);
 cudaError_t launch_dcp_merge(const float* partials, const float* lses, int num_shards, int batch,
                              int heads, float* out, float* out_lse, cudaStream_t st);
 int simt_sparse_chunk_max();
+cudaError_t launch_sparse_gather(const PartialParams& p, int row_bytes, int maxblk,
+                                 uint8_t* gathered, int* counts, cudaStream_t st);
 
 }  // namespace dcpmla

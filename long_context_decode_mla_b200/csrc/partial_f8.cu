@@ -959,7 +959,16 @@ __global__ void __launch_bounds__(kThreads, 1) partial_f8_kernel(const __grid_co
   ptx::tc_fence_after();
 
   int lo = 0, hi = 0;
-  {
+  if (p.per_request_ctas) {
+    request_tile_range(p, c.warp_sums, &lo, &hi);
+    if (lo == hi) {
+      // a request with no row on this shard: the neutral (0, -inf) pair
+      const size_t row0 = (size_t)blockIdx.x * p.rows_o;
+      for (int k = threadIdx.x; k < p.heads * kVDim; k += kThreads)
+        p.out[(row0 + k / kVDim) * kVDim + k % kVDim] = 0.f;
+      if (threadIdx.x < p.heads) p.out_lse[row0 + threadIdx.x] = -CUDART_INF_F;
+    }
+  } else {
     const int T = total_tiles(p, c.warp_sums);
     const int tpc = T > 0 ? (T + p.num_ctas - 1) / p.num_ctas : 0;
     lo = blockIdx.x * tpc;
