@@ -44,7 +44,7 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="agentic",
                     choices=["agentic", "dense", "million", "sparse", "tiny"])
-    ap.add_argument("--kernel", default="auto", choices=["auto", "simt", "tc"])
+    ap.add_argument("--kernel", default="auto", choices=["auto", "simt", "tc", "tc16"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-extras", action="store_true",
@@ -52,6 +52,9 @@ def parse():
     ap.add_argument("--shard-streams", type=int, default=None,
                     help="CUDA streams the N shard launches are spread over "
                          "(default N; 1 = serial)")
+    ap.add_argument("--splits", type=int, default=None,
+                    help="CTAs each shard launch may use (0: all SMs; default: the "
+                         "workload's own choice)")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's batch (smaller cases for profiling)")
     ap.add_argument("--million-layers", type=int, default=83,
@@ -62,6 +65,17 @@ def parse():
     ap.add_argument("--dcp", action="store_true",
                     help="run the real DCP step (one shard per GPU, NCCL) even on one GPU")
     return ap.parse_args()
+
+
+def shard_splits(name, N, args):
+    """CTAs a shard launch may use.  The million-token request splits its one
+    long request over the SM share of its shard; the other workloads let each
+    shard launch size its grid for the whole device (the shards' CTAs then
+    queue on the N streams)."""
+    from long_context_decode_mla_b200 import dcpmla
+    if args.splits is not None:
+        return args.splits
+    return max(1, dcpmla.device_sm_count() // N) if name == "million" else 0
 
 
 def dist_env():
@@ -242,12 +256,11 @@ def run_ours(args, rank, world, local):
                                  seed=cfg["seed"] + 1000 * rank, **over)
     N, B, H = prob.num_shards, prob.batch, prob.heads
     topk = 0 if prob.sparse_idx is None else prob.sparse_idx.shape[1]
-    long_single = args.workload == "million"
     # the N shards are independent: each gets its own stream (a real DCP group
     # runs them on N GPUs), so one shard's ramp-up overlaps another's tail
     n_streams = N if args.shard_streams is None else max(1, min(N, args.shard_streams))
     streams = [torch.cuda.Stream(device=dev) for _ in range(n_streams)] if n_streams > 1 else None
-    splits = max(1, dcpmla.device_sm_count() // N) if long_single else 0
+    splits = shard_splits(args.workload, N, args)
     dec = dcpmla.DcpDecoder(B, H, N, topk=topk, num_splits=splits, device=dev,
                             impl=args.kernel, streams=streams)
     stream = torch.cuda.current_stream(dev)
@@ -278,6 +291,13 @@ def run_ours(args, rank, world, local):
     sampler.mark(True)
     st_step = replay_stats(step_graph, args.steps, stream, flush)
     sampler.mark(False)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    # the partial kernels alone (N shard launches + their split combines),
+    # right after the steps, so that both run at the same clocks (a second of
+    # load first would bring the power cap in)
+    st_part = replay_stats(partial_graph, args.steps, stream, flush)
     # the same steps for about a second more (untimed), so that the clock
     # record under this load has enough samples even when K steps are short
     load = ClockSampler(local)
@@ -290,10 +310,6 @@ def run_ours(args, rank, world, local):
         torch.cuda.synchronize(dev)
     load.mark(False)
     torch.cuda.synchronize(dev)
-    if world > 1:
-        dist.barrier()
-    # the partial kernels alone (N shard launches + their split combines)
-    st_part = replay_stats(partial_graph, args.steps, stream, flush)
     ms_step, ms_partials = st_step["mean"], st_part["mean"]
 
     # end to end through the public API, host buffers in pinned memory
@@ -333,7 +349,25 @@ def run_ours(args, rank, world, local):
     ms_step, e2e_ms, ms_partials = max_over_ranks([ms_step, e2e_ms, ms_partials])
     st_step = dict(zip(st_step, max_over_ranks(list(st_step.values()))))
     st_part = dict(zip(st_part, max_over_ranks(list(st_part.values()))))
-    gpu_launches = args.steps * (N * (1 if (prob.sparse_idx is not None) else 2) + 1)
+    # Launches per shard call.  The e4m3 kernel (fp8 rows, the default) is
+    # preceded by its Q image kernel; dense decode adds the split combine;
+    # sparse decode on the tensor-core path gathers the selected rows first
+    # and keeps whole requests per CTA (no combine).  The fp16-operand and
+    # CUDA-core kernels select sparse rows in-kernel and need the combine only
+    # when a request's list spans several CTAs (lists longer than 2,048, or
+    # fewer requests than SMs).  Plus one merge per step.
+    f8 = prob.kv_dtype == "fp8" and args.kernel in ("auto", "tc")
+    if prob.sparse_idx is not None:
+        if args.kernel in ("tc16", "simt"):
+            sms = torch.cuda.get_device_properties(dev).multi_processor_count
+            parts = max(-(-topk // 2048), sms // max(1, B))
+            per_shard = 2 if parts > 1 else 1
+        else:
+            # gather + image + partial (fp8), gather + partial + combine (bf16)
+            per_shard = 3
+    else:
+        per_shard = 2 + (1 if f8 else 0)
+    gpu_launches = args.steps * (N * per_shard + 1)
     peak, peak_kind = measured_peaks()
     result = None
     if rank == 0:
@@ -365,7 +399,7 @@ def run_ours(args, rank, world, local):
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
                          "unit": "GB/s", "frac": round(achieved / peak, 4),
                          "traffic": traffic, "peak_source": peak_kind,
-                         "kernel": "mla_decode_partial (partial + split combine): the N shard "
+                         "kernel": "mla_decode_partial (Q image + partial + split combine): the N shard "
                                    "launches of a step (one stream each, overlapping), algorithmic "
                                    "bytes / device time of that phase, CUDA-graph replay"},
             "ms_partials_per_step": round(ms_partials, 4),
@@ -477,7 +511,7 @@ def time_other_workload(name, dev, rank, world, args, streams_for=None):
     N = prob.num_shards
     topk = 0 if prob.sparse_idx is None else prob.sparse_idx.shape[1]
     streams = [torch.cuda.Stream(device=dev) for _ in range(N)]
-    splits = max(1, dcpmla.device_sm_count() // N) if name == "million" else 0
+    splits = shard_splits(name, N, args)
     dec = dcpmla.DcpDecoder(prob.batch, prob.heads, N, topk=topk, num_splits=splits, device=dev,
                             impl=args.kernel, streams=streams)
     graph = dec.capture(prob)

@@ -15,9 +15,15 @@ constexpr int kVDim = 512;
 constexpr int kRopeDim = 64;
 constexpr int kBlock = 64;        // rows per cache block
 constexpr int kMaxHeads = 64;
+constexpr int kMaxRequestsPerCta = 32;   // request-aligned schedule: requests a CTA takes
 constexpr int kMaxQueryLen = 64;   // query tokens per request of a multi-query call
 constexpr int kRowBytesBf16 = 1152;
 constexpr int kRowBytesFp8 = 656;
+// Q operand image of one request for the e4m3 kernel: the e4m3 hi and lo
+// codes of the latent (2 x 4 chunks of 64 rows x 128 B), the bf16 rope
+// (64 rows x 128 B), each in the kernel's 128-byte-swizzled shared-memory
+// order, then the 64 per-head frame factors 2^-a (fp32).
+constexpr int kQImageBytes = 2 * 4 * 8192 + 8192 + 64 * 4;
 constexpr int kWsHeader = 256;    // workspace header: flag word + reserved
 constexpr int kMaxDevicesConfigured = 64;   // device ordinals the per-device caches cover
 
@@ -58,7 +64,8 @@ struct PartialParams {
   float* ws_lse;              // [slots][H]
   int* ws_list;               // sparse mode: per-CTA lists of selected local rows
   int num_ctas;               // G: CTAs sharing the dense tile space
-  int per_request_ctas;       // 1: CTA b takes request b whole (grid = batch, no splits)
+  uint8_t* q_image;           // e4m3 kernel: per-request Q operand images (workspace)
+  int request_aligned;        // 1: CTA c takes requests [c B / G, (c+1) B / G) whole (no splits)
   int test_withhold;          // test only: converters skip their first arrival (timeout path)
 };
 
@@ -144,33 +151,37 @@ __device__ __forceinline__ int total_tiles(const PartialParams& p, int* warp_sum
   return acc;
 }
 
-// Per-request schedule: the tile range [lo, hi) of request blockIdx.x in the
-// request-major tile order (all threads of the block call it).
-__device__ __forceinline__ void request_tile_range(const PartialParams& p, int* warp_sums,
-                                                   int* lo, int* hi) {
-  int acc = 0, mine_lo = 0, mine_n = 0;
+// Request-aligned schedule: CTA c of G = num_ctas takes the whole requests
+// [c B / G, (c+1) B / G) and covers their tiles [lo, hi) of the request-major
+// tile order (all threads of the block call it).  Requests of the range with
+// no tile on this shard are marked in *empty_mask (bit r - r0; at most 32
+// requests a CTA).
+__device__ __forceinline__ void request_range_tiles(const PartialParams& p, int* warp_sums,
+                                                    int* r0_out, int* lo, int* hi,
+                                                    uint32_t* empty_mask) {
+  const int r0 = (int)(((long long)blockIdx.x * p.batch) / p.num_ctas);
+  const int r1 = (int)(((long long)(blockIdx.x + 1) * p.batch) / p.num_ctas);
+  __shared__ int range[2];
+  __shared__ uint32_t empties;
+  if (threadIdx.x == 0) empties = 0u;
+  __syncthreads();
+  int acc = 0;
   for (int base = 0; base < p.batch; base += blockDim.x) {
     const int b = base + threadIdx.x;
     int n, nt = 0;
     if (b < p.batch) nt = request_tiles(p, b, &n);
     int tot;
     const int pre = acc + block_exclusive_scan(nt, warp_sums, &tot);
-    if (b == (int)blockIdx.x) {
-      mine_lo = pre;
-      mine_n = nt;
-    }
+    if (b == r0) range[0] = pre;
+    if (b == r1 - 1) range[1] = pre + nt;
+    if (b >= r0 && b < r1 && nt == 0) atomicOr(&empties, 1u << (b - r0));
     acc += tot;
   }
   __syncthreads();
-  // broadcast from the thread that saw request blockIdx.x
-  __shared__ int range[2];
-  if (threadIdx.x == (int)(blockIdx.x % blockDim.x)) {
-    range[0] = mine_lo;
-    range[1] = mine_lo + mine_n;
-  }
-  __syncthreads();
-  *lo = range[0];
-  *hi = range[1];
+  *r0_out = r0;
+  *lo = r1 > r0 ? range[0] : 0;
+  *hi = r1 > r0 ? range[1] : 0;
+  *empty_mask = empties;
 }
 
 struct Segment {

@@ -2,6 +2,7 @@
 // The entry points are declared (and their contracts stated) in dcpmla.h.
 #include "dcpmla.h"
 
+#include <algorithm>
 #include <atomic>
 #include <climits>
 #include <cmath>
@@ -77,14 +78,17 @@ size_t sparse_gather_rows_bytes(int batch, int topk) {
   return round256((size_t)batch * sparse_maxblk(topk) * kBlock * kRowBytesBf16);
 }
 
-// Workspace of one call: dense decode needs split slots; sparse decode needs
-// either the CUDA-core kernel's layout (a slot and a list chunk per CTA) or the
-// gathered rows with dense split slots, whichever is larger.
+// Workspace of one call: dense decode needs split slots and the e4m3
+// kernel's Q images; sparse decode needs either the CUDA-core kernel's layout
+// (a slot and a list chunk per CTA) or the gathered rows with dense split
+// slots and the Q images, whichever is larger.
+size_t q_image_bytes(int batch) { return round256((size_t)batch * kQImageBytes); }
 size_t ws_bytes_for(int batch, int heads, int topk, int ctas) {
   const size_t dense = ws_total((long long)ctas + batch, heads);
-  if (topk <= 0) return dense;
+  if (topk <= 0) return dense + q_image_bytes(batch);
   const size_t simt = ws_total(slots_for(batch, topk, ctas), heads, list_ints_for(batch, topk, ctas));
-  const size_t gathered = dense + sparse_gather_rows_bytes(batch, topk) + round256((size_t)batch * 4);
+  const size_t gathered = dense + sparse_gather_rows_bytes(batch, topk) + round256((size_t)batch * 4) +
+                          q_image_bytes(batch);
   return simt > gathered ? simt : gathered;
 }
 
@@ -199,6 +203,7 @@ int decode_partial(const void* q, const void* kv_cache, int kv_dtype, int64_t nu
   p.ws_list = list_ints ? reinterpret_cast<int*>(ws + ws_list_offset(slots, num_heads)) : nullptr;
   p.num_ctas = ctas;
   p.test_withhold = withhold ? 1 : 0;
+  p.q_image = ws + ws_total((long long)ctas + batch, num_heads);
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   // Sparse decode on the tensor cores: localise and gather the selected rows,
@@ -215,6 +220,7 @@ int decode_partial(const void* q, const void* kv_cache, int kv_dtype, int64_t nu
     int* counts = reinterpret_cast<int*>(gathered + sparse_gather_rows_bytes(batch, eff_topk));
     if (launch_sparse_gather(p, rb, maxblk, gathered, counts, st) != cudaSuccess)
       return DCPMLA_ERR_CUDA;
+    p.q_image = reinterpret_cast<uint8_t*>(counts) + round256((size_t)batch * 4);
     p.kv = gathered;
     p.num_blocks = (long long)batch * maxblk;
     p.block_table = nullptr;
@@ -233,10 +239,12 @@ int decode_partial(const void* q, const void* kv_cache, int kv_dtype, int64_t nu
   const bool tc_ok = tc_supports(p, kv_dtype);
   const bool f8_ok = f8_supports(p, kv_dtype);
   if (gathered_sparse && f8_ok) {
-    // a request's selections are a few tiles: one CTA per request keeps each
-    // request whole (one Q image, one epilogue, nothing to combine)
-    p.per_request_ctas = 1;
-    p.num_ctas = batch;
+    // a request's selections are a few tiles: whole requests per CTA (one Q
+    // image and one epilogue each, nothing to combine), at least
+    // ceil(batch / 32) CTAs, at most one per request
+    const int min_ctas = (batch + kMaxRequestsPerCta - 1) / kMaxRequestsPerCta;
+    p.request_aligned = 1;
+    p.num_ctas = std::max(min_ctas, std::min(batch, ctas));
   }
   enum { kSimt, kTc16, kTc8 } which;
   if (impl == DCPMLA_IMPL_SIMT) {

@@ -83,7 +83,7 @@ cudaError_t launch_dcp_merge(const float* partials, const float* lses, int num_s
 }
 
 cudaError_t launch_split_combine(const PartialParams& p, cudaStream_t st) {
-  if ((p.sparse_idx && p.sparse_parts == 1) || p.per_request_ctas) return cudaSuccess;
+  if ((p.sparse_idx && p.sparse_parts == 1) || p.request_aligned) return cudaSuccess;
   const int hgroups = (p.heads + 7) / 8;
   split_combine_kernel<<<p.batch * hgroups, 256, 0, st>>>(p);
   return cudaGetLastError();

@@ -98,6 +98,8 @@ constexpr uint32_t kOffQh = 0;                    // Q hi: 4 chunks of 64 rows x
 constexpr uint32_t kOffQl = kOffQh + 4 * kChunk;  // Q lo
 constexpr uint32_t kOffQr = kOffQl + 4 * kChunk;  // Q rope: 64 rows x 64 bf16
 constexpr uint32_t kOffCode = kOffQr + kChunk;
+constexpr uint32_t kQOperandBytes = kOffCode - kOffQh;   // hi, lo and rope, contiguous
+static_assert(kQOperandBytes + 64 * 4 == (uint32_t)kQImageBytes, "Q image = operands + frame");
 constexpr uint32_t kOffRope = kOffCode + kCodeStages * kCodeStage;
 constexpr uint32_t kOffP = kOffRope + kRopeStages * kChunk;
 constexpr uint32_t kOffCtl = kOffP + 8 * kPVar;
@@ -136,7 +138,7 @@ struct F8Ctl {
   alignas(16) float sc_r[2][4];     // per group: O rescale factor S_old / S_new at this tile
   alignas(16) float sc_ref[2][4];   // per group: S_g in force for this tile
   alignas(16) float gw[2][4][4];    // staging: per-warp group maxima of |scale|
-  float qexp[64];                   // 2^-a per head (Q frame)
+  alignas(16) float qexp[64];       // 2^-a per head (Q frame)
   float mred[2][4][64];             // [tile parity] per-thread-column maxima of the scores; in
                                     // the epilogue (other parity) the per-thread-column sums
   uint64_t full[kCodeStages];       // TMA bytes of a tile landed
@@ -441,76 +443,26 @@ __device__ __forceinline__ void pv_role(const PartialParams& p, F8Ctl& c, uint8_
   }
 }
 
-// Q of request b (the 128 staging threads): thread u handles head u / 2 and
-// half the latent (256 values) and rope (32 values).  Writes the hi and lo A
-// operands (64 rows each), the rope A operand and 2^-a per head, once the
-// previous request's score MMAs are done and its softmax read its Q frame.
-__device__ __forceinline__ bool prepare_q(const PartialParams& p, F8Ctl& c, uint8_t* base, int b,
-                          uint32_t sigma) {
+// Q of request b: one bulk copy of its operand image (hi and lo codes and
+// rope, in shared-memory order) and one of its frame factors, issued once the
+// previous request's score MMAs are done and its softmax read its frame.
+// Staging warp 0 arms q_full with the bytes; the other three arrive.
+__device__ __forceinline__ bool load_q(const PartialParams& p, F8Ctl& c, uint8_t* base, int b,
+                                       uint32_t sigma) {
   const int u = threadIdx.x - kStageWarp0 * 32;   // 0..127
-  const int hq = u >> 1, part = u & 1;
-  uint8_t* qh = base + kOffQh;
-  uint8_t* ql = base + kOffQl;
-  uint8_t* qr = base + kOffQr;
   if (sigma > 0 && !wait_or_abort(&c.q_empty, (sigma - 1) & 1, c)) return false;
-  const bool live = hq < p.heads;
-  const uint4* src =
-      reinterpret_cast<const uint4*>(p.q + ((size_t)b * p.rows_q + (live ? hq : 0)) * kHeadDim);
-  float amax = 0.f;
-#pragma unroll 4
-  for (int k = 0; k < 32; ++k) {
-    const uint4 v = live ? __ldg(src + part * 32 + k) : make_uint4(0, 0, 0, 0);
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int e = 0; e < 4; ++e)
-      amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(w[e] << 16)),
-                               fabsf(__uint_as_float(w[e] & 0xFFFF0000u))));
+  if (u == 0) {
+    F8_TRACE(22, sigma);
+    // the softmax read the old frame through the generic proxy
+    ptx::fence_proxy_async();
+    const uint8_t* img = p.q_image + (size_t)b * kQImageBytes;
+    ptx::mbar_arrive_expect_tx(&c.q_full, kQImageBytes);
+    ptx::bulk_g2s(ptx::smem_addr(base + kOffQh), img, kQOperandBytes, &c.q_full);
+    ptx::bulk_g2s(ptx::smem_addr(c.qexp), img + kQOperandBytes, kQImageBytes - kQOperandBytes,
+                  &c.q_full);
+  } else if (u >= 32) {
+    warp_arrive(&c.q_full);
   }
-  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-  // frame: q * 2^a with max |q * 2^a| in [128, 256)
-  int a = 0;
-  if (amax > 0.f) {
-    const int e = (int)((__float_as_uint(amax) >> 23) & 0xFF) - 127;
-    a = min(120, max(-120, 7 - e));
-  }
-  const float fa = __uint_as_float((uint32_t)(127 + a) << 23);
-  if (part == 0) c.qexp[hq] = __uint_as_float((uint32_t)(127 - a) << 23);
-  // latent: 16 output units of 16 codes (two groups of 128 values) per term
-  // (not unrolled: these warps keep a small register budget)
-#pragma unroll 1
-  for (int uo = 0; uo < 16; ++uo) {
-    const int g = 2 * part + (uo >> 3), un = uo & 7;
-    uint32_t hw[4], lw[4];
-#pragma unroll
-    for (int k = 0; k < 2; ++k) {
-      const uint4 v = live ? __ldg(src + part * 32 + 2 * uo + k) : make_uint4(0, 0, 0, 0);
-      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-      for (int e = 0; e < 4; e += 2) {
-        // four bf16 values -> one word of hi codes and one of lo codes
-        const float f0 = __uint_as_float(w[e] << 16) * fa;
-        const float f1 = __uint_as_float(w[e] & 0xFFFF0000u) * fa;
-        const float f2 = __uint_as_float(w[e + 1] << 16) * fa;
-        const float f3 = __uint_as_float(w[e + 1] & 0xFFFF0000u) * fa;
-        const uint32_t h01 = e4m3x2_f32(f0, f1), h23 = e4m3x2_f32(f2, f3);
-        const float2 b01 = e4m3x2_to_f32(h01), b23 = e4m3x2_to_f32(h23);
-        const uint32_t l01 = e4m3x2_f32(f0 - b01.x, f1 - b01.y);
-        const uint32_t l23 = e4m3x2_f32(f2 - b23.x, f3 - b23.y);
-        hw[2 * k + e / 2] = h01 | (h23 << 16);
-        lw[2 * k + e / 2] = l01 | (l23 << 16);
-      }
-    }
-    *reinterpret_cast<uint4*>(qh + g * kChunk + sw128(hq, un)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-    *reinterpret_cast<uint4*>(ql + g * kChunk + sw128(hq, un)) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
-  }
-  // rope: 32 bf16 values = 4 units
-#pragma unroll
-  for (int un = 0; un < 4; ++un) {
-    const uint4 v = live ? __ldg(src + 64 + part * 4 + un) : make_uint4(0, 0, 0, 0);
-    *reinterpret_cast<uint4*>(qr + sw128(hq, part * 4 + un)) = v;
-  }
-  ptx::fence_proxy_async();
-  warp_arrive(&c.q_full);
   return true;
 }
 
@@ -533,7 +485,7 @@ __device__ __forceinline__ void staging_role(const PartialParams& p, F8Ctl& c, u
     const int b = tau & 1;
     const bool first = cur.t == 0;
     if (first) {
-      if (!prepare_q(p, c, base, cur.v.b, sigma)) return;
+      if (!load_q(p, c, base, cur.v.b, sigma)) return;
       ++sigma;
     }
     if (!wait_or_abort(&c.full[cs], (tau / kCodeStages) & 1, c)) return;
@@ -812,6 +764,7 @@ __device__ __forceinline__ void softmax_role(const PartialParams& p, F8Ctl& c, u
       ls[col][h] = l;
       // o_full completes once per request, after its last PV
       if (!wait_or_abort(&c.o_full, sigma & 1, c)) return;
+      if (T == 0) F8_TRACE(17, sigma);
       ptx::named_bar(kBarSoft, kSoftThreads);
       __syncwarp();
       ptx::tc_fence_after();
@@ -820,8 +773,14 @@ __device__ __forceinline__ void softmax_role(const PartialParams& p, F8Ctl& c, u
         (v.whole ? p.out_lse : p.ws_lse)[slot * (v.whole ? p.rows_o : p.heads) + h] =
             ltot > 0.f ? (m_used + log2f(ltot)) * kLn2 : -CUDART_INF_F;
       const float il = ltot > 0.f ? 1.f / ltot : 0.f;
-      float* o_base = (v.whole ? p.out : p.ws_o) +
-                      (slot * (v.whole ? p.rows_o : p.heads) + h) * kVDim + odh;
+      // O leaves through this warp's 4 KB of the P buffer (free: the last PV
+      // is done): lane i writes its head's 32 values (128 bytes) as row i,
+      // 16-byte units xor-swizzled by i % 8; then 8 lanes take one row, so
+      // that each store writes four whole 128-byte lines of O.
+      float* o_rows = (v.whole ? p.out : p.ws_o) + slot * (v.whole ? p.rows_o : p.heads) * kVDim;
+      uint8_t* scr = pbuf + w * 4096;
+      const int h_w = (32 * q) & 63;         // head of lane 0 of this warp
+      const int rq = i >> 3, un = i & 7;     // read side: row 4 k + rq, unit un
 #pragma unroll 1
       for (int g = 0; g < 4; ++g) {
         const float sg = g == 0 ? sref.x : g == 1 ? sref.y : g == 2 ? sref.z : sref.w;
@@ -829,17 +788,24 @@ __device__ __forceinline__ void softmax_role(const PartialParams& p, F8Ctl& c, u
         uint32_t v32[32];
         ptx::tmem_ld32(lane_base + 64 * g + 32 * th, v32);
         ptx::tmem_wait_ld();
-        if (h < p.heads) {
-          float4* dst = reinterpret_cast<float4*>(o_base + g * 128);
 #pragma unroll
-          for (int e = 0; e < 8; ++e)
-            dst[e] = make_float4(__uint_as_float(v32[4 * e]) * f, __uint_as_float(v32[4 * e + 1]) * f,
-                                 __uint_as_float(v32[4 * e + 2]) * f,
-                                 __uint_as_float(v32[4 * e + 3]) * f);
+        for (int e = 0; e < 8; ++e)
+          *reinterpret_cast<float4*>(scr + i * 128 + ((e ^ (i & 7)) << 4)) =
+              make_float4(__uint_as_float(v32[4 * e]) * f, __uint_as_float(v32[4 * e + 1]) * f,
+                          __uint_as_float(v32[4 * e + 2]) * f, __uint_as_float(v32[4 * e + 3]) * f);
+        __syncwarp();
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const int r = 4 * k + rq;
+          const float4 val = *reinterpret_cast<const float4*>(scr + r * 128 + ((un ^ (r & 7)) << 4));
+          if (h_w + r < p.heads)
+            *reinterpret_cast<float4*>(o_rows + (size_t)(h_w + r) * kVDim + g * 128 + odh + 4 * un) = val;
         }
+        __syncwarp();
       }
       ptx::tc_fence_before();
       ptx::named_bar(kBarSoft, kSoftThreads);
+      if (T == 0) F8_TRACE(18, sigma);
       ++sigma;
     }
     ++tau;
@@ -917,6 +883,8 @@ __device__ __forceinline__ void run_roles(const F8Params& P, const PartialParams
     if (threadIdx.x == kProdWarp * 32)
       for (int s = 0; s < kCodeStages; ++s)
         if (fills[s] > 0) wait_or_abort(&c.full[s], (fills[s] - 1) & 1, c);
+    // the last Q image copy (the staging warps count their requests in sigma)
+    if (threadIdx.x == kStageWarp0 * 32 && sigma > 0) wait_or_abort(&c.q_full, (sigma - 1) & 1, c);
   }
 }
 
@@ -959,11 +927,15 @@ __global__ void __launch_bounds__(kThreads, 1) partial_f8_kernel(const __grid_co
   ptx::tc_fence_after();
 
   int lo = 0, hi = 0;
-  if (p.per_request_ctas) {
-    request_tile_range(p, c.warp_sums, &lo, &hi);
-    if (lo == hi) {
-      // a request with no row on this shard: the neutral (0, -inf) pair
-      const size_t row0 = (size_t)blockIdx.x * p.rows_o;
+  if (p.request_aligned) {
+    int r0;
+    uint32_t empties;
+    request_range_tiles(p, c.warp_sums, &r0, &lo, &hi, &empties);
+    // requests of the range with no row on this shard: the neutral (0, -inf)
+    while (empties) {
+      const int b = r0 + __ffs(empties) - 1;
+      empties &= empties - 1;
+      const size_t row0 = (size_t)b * p.rows_o;
       for (int k = threadIdx.x; k < p.heads * kVDim; k += kThreads)
         p.out[(row0 + k / kVDim) * kVDim + k % kVDim] = 0.f;
       if (threadIdx.x < p.heads) p.out_lse[row0 + threadIdx.x] = -CUDART_INF_F;
@@ -993,6 +965,77 @@ __global__ void __launch_bounds__(kThreads, 1) partial_f8_kernel(const __grid_co
   block_bar();
   ptx::tc_fence_after();
   if (warp == 0) ptx::tmem_dealloc(c.tmem_base, kTmemCols);
+}
+
+// ------------------------------------------------------------- Q image ----
+
+// Two words of bf16 pairs (four values) times the frame 2^a -> the e4m3 codes
+// of the four values (hi) and the e4m3 codes of what hi leaves of them (lo),
+// first value in the low byte.  The product is exact (a power of two within
+// range) and so is the remainder.
+__device__ __forceinline__ void split_q4(uint32_t w0, uint32_t w1, float fa, uint32_t& hi,
+                                         uint32_t& lo) {
+  const float f0 = __uint_as_float(w0 << 16) * fa;
+  const float f1 = __uint_as_float(w0 & 0xFFFF0000u) * fa;
+  const float f2 = __uint_as_float(w1 << 16) * fa;
+  const float f3 = __uint_as_float(w1 & 0xFFFF0000u) * fa;
+  const uint32_t h01 = e4m3x2_f32(f0, f1), h23 = e4m3x2_f32(f2, f3);
+  const float2 b01 = e4m3x2_to_f32(h01), b23 = e4m3x2_to_f32(h23);
+  hi = h01 | (h23 << 16);
+  lo = e4m3x2_f32(f0 - b01.x, f1 - b01.y) | (e4m3x2_f32(f2 - b23.x, f3 - b23.y) << 16);
+}
+
+// Q operand images, one per request: the frame 2^a of a head puts the largest
+// |q| of its latent in [128, 256); the latent times 2^a is split into two
+// e4m3 terms, and the rope is copied as it is (the softmax scales its score
+// by 2^a).  Head rows past p.heads are zero.  Grid (batch, 2): each CTA covers
+// 32 head rows with 8 threads per head; thread t holds latent values
+// [64 t, 64 t + 64) (four 16-value units of group t / 2) and rope unit t, and
+// issues all its loads before any use.
+__global__ void __launch_bounds__(256) f8_q_image_kernel(const PartialParams p, uint8_t* image) {
+  const int b = blockIdx.x;
+  const int h = blockIdx.y * 32 + (threadIdx.x >> 3), t = threadIdx.x & 7;
+  const bool live = h < p.heads;
+  const uint4* src =
+      reinterpret_cast<const uint4*>(p.q + ((size_t)b * p.rows_q + (live ? h : 0)) * kHeadDim);
+  const uint4 zero = make_uint4(0, 0, 0, 0);
+  uint4 v[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) v[k] = live ? __ldg(src + 8 * t + k) : zero;
+  const uint4 rope = live ? __ldg(src + 64 + t) : zero;
+  float amax = 0.f;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const uint32_t w[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(w[e] << 16)),
+                               fabsf(__uint_as_float(w[e] & 0xFFFF0000u))));
+  }
+#pragma unroll
+  for (int o = 1; o < 8; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  int a = 0;
+  if (amax > 0.f) {
+    const int e = (int)((__float_as_uint(amax) >> 23) & 0xFF) - 127;
+    a = min(120, max(-120, 7 - e));
+  }
+  const float fa = __uint_as_float((uint32_t)(127 + a) << 23);
+  uint8_t* img = image + (size_t)b * kQImageBytes;
+  if (t == 0) reinterpret_cast<float*>(img + kQOperandBytes)[h] = __uint_as_float((uint32_t)(127 - a) << 23);
+  const int g = t >> 1;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int un = (t & 1) * 4 + j;
+    const uint4 x0 = v[2 * j], x1 = v[2 * j + 1];
+    uint4 hi, lo;
+    split_q4(x0.x, x0.y, fa, hi.x, lo.x);
+    split_q4(x0.z, x0.w, fa, hi.y, lo.y);
+    split_q4(x1.x, x1.y, fa, hi.z, lo.z);
+    split_q4(x1.z, x1.w, fa, hi.w, lo.w);
+    *reinterpret_cast<uint4*>(img + kOffQh + g * kChunk + sw128(h, un)) = hi;
+    *reinterpret_cast<uint4*>(img + kOffQl + g * kChunk + sw128(h, un)) = lo;
+  }
+  *reinterpret_cast<uint4*>(img + kOffQr + sw128(h, t)) = rope;
 }
 
 // ---------------------------------------------------------------- host -----
@@ -1047,6 +1090,7 @@ bool f8_supports(const PartialParams& p, int kv_dtype) {
 }
 
 cudaError_t launch_partial_f8(const PartialParams& p, cudaStream_t st) {
+  if (!p.q_image) return cudaErrorInvalidValue;
   F8Params fp;
   fp.p = p;
   if (!encode_maps(p, &fp.rows, &fp.scales)) return cudaErrorInvalidValue;
@@ -1074,6 +1118,7 @@ cudaError_t launch_partial_f8(const PartialParams& p, cudaStream_t st) {
       g_attr_done[dev] = true;
     }
   }
+  f8_q_image_kernel<<<dim3(p.batch, 2), 256, 0, st>>>(p, p.q_image);
   partial_f8_kernel<<<p.num_ctas, kThreads, smem, st>>>(fp);
   return cudaGetLastError();
 }

@@ -123,15 +123,18 @@ def test_split_counts_agree(impl, splits):
     _check_problem(prob, impl, num_splits=splits)
 
 
+# splits: 0 gives every request its own CTA; 2 puts three whole requests,
+# empty ones among them, on each CTA of the request-aligned schedule
 @pytest.mark.parametrize("impl", IMPLS)
 @pytest.mark.parametrize("N", [1, 2, 8])
-def test_sparse_small(impl, N):
+@pytest.mark.parametrize("splits", [0, 2])
+def test_sparse_small(impl, N, splits):
     prob = wl.make_problem("sparse", num_shards=N, batch=6, seq_len=3000, topk=300, seed=4)
     idx = prob.sparse_idx
     idx[1] = -1                                   # empty list
     idx[2, :] = (torch.arange(300) * N) % 3000    # everything on shard 0
     idx[3, :150] = torch.arange(150) + 3000       # half out of range
-    _check_problem(prob, impl)
+    _check_problem(prob, impl, num_splits=splits)
 
 
 # --------------------------------------------------------------- addressing -
@@ -163,7 +166,8 @@ def test_block_table_addressing_is_exact(impl, kv_dtype, N):
 
 @pytest.mark.parametrize("impl", IMPLS)
 @pytest.mark.parametrize("N", [1, 2, 4, 8])
-def test_sparse_selection_is_exact(impl, N):
+@pytest.mark.parametrize("splits", [0, 2])
+def test_sparse_selection_is_exact(impl, N, splits):
     L = 6000
     rng = np.random.default_rng(N)
     idx = np.full((5, 512), -1, dtype=np.int32)
@@ -173,7 +177,7 @@ def test_sparse_selection_is_exact(impl, N):
     idx[3, :300] = rng.choice(L, 300, replace=False)
     idx[4, :] = rng.choice(L, 512, replace=False)
     prob = wl.id_coded_problem([L] * 5, N, "fp8", heads=8, seed=N, sparse_idx=idx)
-    parts, lses, out, lse = _run(prob, impl)
+    parts, lses, out, lse = _run(prob, impl, num_splits=splits)
     for b in range(5):
         for s in range(N):
             ids = [int(t) for t in idx[b] if 0 <= t < L and t % N == s]
@@ -263,6 +267,13 @@ def test_million_config_full_size(N):
 def test_sparse_config_full_size(N):
     prob = wl.make_problem("sparse", num_shards=N, kv_device="cuda")
     _check_problem(prob, "auto", batch_ids=[0, 64, 127])
+
+
+def test_sparse_config_full_size_sm_share():
+    # the bench's launch: 8 shards, each given 148 / 8 CTAs (seven or eight
+    # whole requests each)
+    prob = wl.make_problem("sparse", num_shards=8, kv_device="cuda")
+    _check_problem(prob, "auto", batch_ids=[0, 6, 7, 127], num_splits=18)
 
 
 @pytest.mark.parametrize("impl", IMPLS)
