@@ -65,6 +65,10 @@ struct PartialParams {
   int* ws_list;               // sparse mode: per-CTA lists of selected local rows
   int num_ctas;               // G: CTAs sharing the dense tile space
   uint8_t* q_image;           // e4m3 kernel: per-request Q operand images (workspace)
+  const int* row_ids;         // e4m3 kernel, sparse: per-request flat cache rows (padded
+                              // to whole tiles); tile k of request b is rows
+                              // [b * row_stride + 64 k, + 64) of the list
+  int row_stride;
   int request_aligned;        // 1: CTA c takes requests [c B / G, (c+1) B / G) whole (no splits)
   int test_withhold;          // test only: converters skip their first arrival (timeout path)
 };

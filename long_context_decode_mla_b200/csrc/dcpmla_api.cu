@@ -218,11 +218,25 @@ int decode_partial(const void* q, const void* kv_cache, int kv_dtype, int64_t nu
     const int maxblk = (int)sparse_maxblk(eff_topk);
     uint8_t* gathered = ws + ws_total((long long)ctas + batch, num_heads);
     int* counts = reinterpret_cast<int*>(gathered + sparse_gather_rows_bytes(batch, eff_topk));
-    if (launch_sparse_gather(p, rb, maxblk, gathered, counts, st) != cudaSuccess)
-      return DCPMLA_ERR_CUDA;
     p.q_image = reinterpret_cast<uint8_t*>(counts) + round256((size_t)batch * 4);
-    p.kv = gathered;
-    p.num_blocks = (long long)batch * maxblk;
+    // The e4m3 kernel fetches the selected rows from the cache itself, given
+    // their flat row numbers (int32); the other kernels read the rows copied
+    // into whole blocks.
+    PartialParams dense_view = p;
+    dense_view.sparse_idx = nullptr;
+    const bool listed = impl != DCPMLA_IMPL_TC_F16 && f8_supports(dense_view, kv_dtype) &&
+                        num_blocks <= (int64_t)(INT32_MAX / kBlock);
+    if (listed) {
+      int* rows = reinterpret_cast<int*>(gathered);
+      if (launch_sparse_rows(p, maxblk, rows, counts, st) != cudaSuccess) return DCPMLA_ERR_CUDA;
+      p.row_ids = rows;
+      p.row_stride = maxblk * kBlock;
+    } else {
+      if (launch_sparse_gather(p, rb, maxblk, gathered, counts, st) != cudaSuccess)
+        return DCPMLA_ERR_CUDA;
+      p.kv = gathered;
+      p.num_blocks = (long long)batch * maxblk;
+    }
     p.block_table = nullptr;
     p.id_stride = maxblk;
     p.bt_stride = maxblk;

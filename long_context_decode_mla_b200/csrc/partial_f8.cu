@@ -107,6 +107,7 @@ static_assert(kOffCode % 1024 == 0 && kCodeStage % 1024 == 0 && kOffRope % 1024 
                   kOffP % 1024 == 0,
               "swizzled operands need 1024-byte alignment");
 static_assert(kTileBytes == 4 * kChunk + 1024 + kChunk, "a tile is codes, scales and rope");
+constexpr uint32_t kListedTileBytes = kTileBytes - 1024;   // gathered: codes and rope
 
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColPart = 256;      // 8 score part buffers of 32 columns; O: [0, 256)
@@ -257,52 +258,86 @@ __device__ __forceinline__ void split_hilo4(uint32_t x0, uint32_t x1, uint32_t& 
 
 // ---------------------------------------------------------------- roles ----
 
-// TMA producer (one thread): tile tau goes to code slot tau % 3 and rope
-// slot tau % 2.  A tile whose table entry is out of range (flagged) loads
-// block 0 instead; it then has no valid rows.
+// TMA producer (one warp): tile tau goes to code slot tau % 3 and rope slot
+// tau % 2.  Lane 0 waits for the slots and arms the tile's barrier.  A block
+// tile is six box loads by lane 0; a tile whose table entry is out of range
+// (flagged) loads block 0 instead and has no valid rows.  A listed tile
+// (sparse rows, p.row_ids) is fetched by lanes 0..15, four rows each: five
+// gathers of four rows (the four code chunks and the rope); its scales are
+// read by the staging warps (four rows of 16 bytes would not land on the
+// 128-byte boundary a tensor copy needs).
+template <bool kListed>
 __device__ __forceinline__ void producer_role(const F8Params& P, const PartialParams& p, F8Ctl& c,
                               uint8_t* base, int nseg, uint32_t& tau,
                               uint32_t (&fills)[kCodeStages]) {
+  const int lane = threadIdx.x & 31;
+  const bool lead = lane == 0;
   TileCursor cur, pf;
   if (!cur.start(p, c, nseg)) return;
   pf = cur;
-  bool pf_ok = true;
+  bool pf_ok = !kListed;
   for (int i = 0; i < kPrefetchTiles && pf_ok; ++i) {
     const int blk = tile_block(p, pf.v.b, (pf.v.row_begin >> 6) + pf.t);
-    if (blk >= 0) ptx::prefetch_l2(p.kv + (size_t)blk * kTileBytes, kTileBytes);
+    if (lead && blk >= 0) ptx::prefetch_l2(p.kv + (size_t)blk * kTileBytes, kTileBytes);
     pf_ok = pf.next(p, c);
   }
   while (true) {
     const uint32_t cs = tau % kCodeStages, rs = tau % kRopeStages;
     // slot reuse: the PV of tile tau - 3 and the rope part of tile tau - 2
-    if (tau >= (uint32_t)kCodeStages &&
-        !wait_or_abort(&c.code_empty[cs], ((tau / kCodeStages) + 1) & 1, c))
-      return;
-    if (tau >= (uint32_t)kRopeStages &&
-        !wait_or_abort(&c.rope_empty[rs], ((tau / kRopeStages) + 1) & 1, c))
-      return;
-    const int blk = tile_block(p, cur.v.b, (cur.v.row_begin >> 6) + cur.t);
-    const int z = blk >= 0 ? blk : 0;
-    // read after the bytes land (the arrival below releases this write)
-    c.nv[cs] = blk >= 0 ? cur.tile_valid_rows() : 0;
-    F8_TRACE(0, tau);
+    bool ok = true;
+    if (lead) {
+      if (tau >= (uint32_t)kCodeStages)
+        ok = wait_or_abort(&c.code_empty[cs], ((tau / kCodeStages) + 1) & 1, c);
+      if (ok && tau >= (uint32_t)kRopeStages)
+        ok = wait_or_abort(&c.rope_empty[rs], ((tau / kRopeStages) + 1) & 1, c);
+    }
+    if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) return;
     // test only: withholding the very first tile makes every pipeline wait
     // of the CTA run out, which exercises the timeout path
-    if (!(p.test_withhold && tau == 0)) {
-      uint64_t* bar = &c.full[cs];
-      ptx::mbar_arrive_expect_tx(bar, kTileBytes);
-      const uint32_t dst = ptx::smem_addr(base + kOffCode + cs * kCodeStage);
+    const bool issue = !(p.test_withhold && tau == 0);
+    uint64_t* bar = &c.full[cs];
+    const uint32_t dst = ptx::smem_addr(base + kOffCode + cs * kCodeStage);
+    const uint32_t dst_rope = ptx::smem_addr(base + kOffRope + rs * kChunk);
+    if constexpr (!kListed) {
+      if (lead) {
+        const int blk = tile_block(p, cur.v.b, (cur.v.row_begin >> 6) + cur.t);
+        const int z = blk >= 0 ? blk : 0;
+        // read after the bytes land (the arrival below releases this write)
+        c.nv[cs] = blk >= 0 ? cur.tile_valid_rows() : 0;
+        F8_TRACE(0, tau);
+        if (issue) {
+          ptx::mbar_arrive_expect_tx(bar, kTileBytes);
 #pragma unroll
-      for (int k = 0; k < 4; ++k) ptx::tma_load_3d(dst + k * kChunk, &P.rows, box_x(k), 0, z, bar);
-      ptx::tma_load_3d(dst + kScalesOff, &P.scales, 512, 0, z, bar);
-      ptx::tma_load_3d(ptx::smem_addr(base + kOffRope + rs * kChunk), &P.rows, box_x(4), 0, z, bar);
-      ++fills[cs];
+          for (int k = 0; k < 4; ++k) ptx::tma_load_3d(dst + k * kChunk, &P.rows, box_x(k), 0, z, bar);
+          ptx::tma_load_3d(dst + kScalesOff, &P.scales, 512, 0, z, bar);
+          ptx::tma_load_3d(dst_rope, &P.rows, box_x(4), 0, z, bar);
+          ++fills[cs];
+        }
+      }
+    } else {
+      if (lead) {
+        c.nv[cs] = cur.tile_valid_rows();
+        F8_TRACE(0, tau);
+        if (issue) {
+          ptx::mbar_arrive_expect_tx(bar, kListedTileBytes);
+          ++fills[cs];
+        }
+      }
+      __syncwarp();
+      if (issue && lane < 16) {
+        const int4 r = __ldg(reinterpret_cast<const int4*>(
+                                 p.row_ids + (size_t)cur.v.b * p.row_stride + cur.v.row_begin +
+                                 cur.t * kTileRows) + lane);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) ptx::tma_gather4(dst + k * kChunk + lane * 512, &P.rows, box_x(k), r, bar);
+        ptx::tma_gather4(dst_rope + lane * 512, &P.rows, box_x(4), r, bar);
+      }
     }
     ++tau;
     if (!cur.next(p, c)) break;
     if (pf_ok) {
       const int pb = tile_block(p, pf.v.b, (pf.v.row_begin >> 6) + pf.t);
-      if (pb >= 0) ptx::prefetch_l2(p.kv + (size_t)pb * kTileBytes, kTileBytes);
+      if (lead && pb >= 0) ptx::prefetch_l2(p.kv + (size_t)pb * kTileBytes, kTileBytes);
       pf_ok = pf.next(p, c);
     }
   }
@@ -342,25 +377,21 @@ __device__ __forceinline__ void qk_role(int side, const PartialParams& p, F8Ctl&
     //    scales nor the clearing of rows past the end: those rows' scores
     //    are masked, and PV, which does need the clearing, runs after the
     //    softmax has waited for it);
-    //  * the PV of tile tau - 2 is done (the release of its code slot, a
-    //    barrier that cannot complete its next phase before these scores),
-    //    so that a PV never waits behind score MMAs of tiles far ahead;
     //  * each part's buffer is free (part number n reuses the buffer of
-    //    part n - 8, released by the softmax).
-    uint64_t* bars[5];
-    uint32_t pars[5];
+    //    part n - 8, released by the softmax), which keeps the scores at
+    //    most 1.6 tiles ahead of the softmax.
+    uint64_t* bars[4];
+    uint32_t pars[4];
     bars[0] = &c.full[cs];
     pars[0] = (tau / kCodeStages) & 1;
-    bars[1] = tau >= 2 ? &c.code_empty[(tau - 2) % kCodeStages] : bars[0];
-    pars[1] = tau >= 2 ? ((tau - 2) / kCodeStages) & 1 : pars[0];
 #pragma unroll
     for (int k = 0; k < 3; ++k) {
       const int part = side + 2 * (k < nparts ? k : nparts - 1);
       const uint32_t pi = 5 * tau + part;
-      bars[2 + k] = pi >= (uint32_t)kParts ? &c.part_empty[pi % kParts] : bars[0];
-      pars[2 + k] = pi >= (uint32_t)kParts ? ((pi / kParts) + 1) & 1 : pars[0];
+      bars[1 + k] = pi >= (uint32_t)kParts ? &c.part_empty[pi % kParts] : bars[0];
+      pars[1 + k] = pi >= (uint32_t)kParts ? ((pi / kParts) + 1) & 1 : pars[0];
     }
-    if (!ptx::mbar_wait5(bars, pars, &c.abort)) return;
+    if (!ptx::mbar_wait4(bars, pars, &c.abort)) return;
     ptx::tc_fence_after();
     if (side == 0) F8_TRACE(1, tau);
     const uint64_t dcode = dplus(dc0, cs * kCodeStage), drope = dplus(dr0, rs * kChunk);
@@ -472,6 +503,7 @@ __device__ __forceinline__ bool load_q(const PartialParams& p, F8Ctl& c, uint8_t
 // implies, and zeros over the codes of rows past the request's end (their
 // bytes are whatever the block holds and must not reach PV).  Thread u
 // handles row u / 2, groups 2 (u % 2) and 2 (u % 2) + 1.
+template <bool kListed>
 __device__ __forceinline__ void staging_role(const PartialParams& p, F8Ctl& c, uint8_t* base, int nseg,
                              uint32_t& tau, uint32_t& sigma) {
   const int u = threadIdx.x - kStageWarp0 * 32;   // 0..127
@@ -484,6 +516,15 @@ __device__ __forceinline__ void staging_role(const PartialParams& p, F8Ctl& c, u
     const uint32_t cs = tau % kCodeStages;
     const int b = tau & 1;
     const bool first = cur.t == 0;
+    // a listed tile's scales come from the cache rows themselves, loaded
+    // before the wait for the tile's bytes
+    float2 sv_listed = make_float2(0.f, 0.f);
+    if constexpr (kListed) {
+      const int rid = __ldg(p.row_ids + (size_t)cur.v.b * p.row_stride + cur.v.row_begin +
+                            cur.t * kTileRows + row);
+      sv_listed = __ldg(reinterpret_cast<const float2*>(p.kv + (size_t)rid * kRowBytesFp8 + 512 +
+                                                         gp * 4));
+    }
     if (first) {
       if (!load_q(p, c, base, cur.v.b, sigma)) return;
       ++sigma;
@@ -494,7 +535,8 @@ __device__ __forceinline__ void staging_role(const PartialParams& p, F8Ctl& c, u
     if (tau >= 2 && !wait_or_abort(&c.sc_empty[b], ((tau / 2) + 1) & 1, c)) return;
     const int nv = c.nv[cs];
     uint8_t* code = base + kOffCode + cs * kCodeStage;
-    const float2 sv = *reinterpret_cast<const float2*>(code + kScalesOff + row * 16 + gp * 4);
+    const float2 sv = kListed ? sv_listed
+                                : *reinterpret_cast<const float2*>(code + kScalesOff + row * 16 + gp * 4);
     const bool valid = row < nv;
     float m0 = valid ? fabsf(sv.x) : 0.f, m1 = valid ? fabsf(sv.y) : 0.f;
 #pragma unroll
@@ -820,7 +862,7 @@ __device__ __forceinline__ void block_bar() { ptx::named_bar(kBarBlock, kThreads
 // The batch loop of one side of the register split: kSoft runs the softmax
 // warps, !kSoft every other role and, at the end, the drains of the
 // asynchronous arrivals.  Both sides take the same block barriers.
-template <bool kSoft>
+template <bool kSoft, bool kListed>
 __device__ __forceinline__ void run_roles(const F8Params& P, const PartialParams& p, F8Ctl& c,
                                           uint8_t* base, int lo, int hi) {
   const int warp = threadIdx.x >> 5;
@@ -836,13 +878,13 @@ __device__ __forceinline__ void run_roles(const F8Params& P, const PartialParams
       softmax_role(p, c, base, nseg, tau, sigma, pi);
     } else {
       if (warp == kProdWarp) {
-        if ((threadIdx.x & 31) == 0) producer_role(P, p, c, base, nseg, tau, fills);
+        producer_role<kListed>(P, p, c, base, nseg, tau, fills);
       } else if (warp == kQkWarp || warp == kQkWarp2) {
         if ((threadIdx.x & 31) == 0) qk_role(warp == kQkWarp ? 0 : 1, p, c, base, nseg, tau, sigma);
       } else if (warp == kPvWarp) {
         if ((threadIdx.x & 31) == 0) pv_role(p, c, base, nseg, tau, uses, o_commits);
       } else {
-        staging_role(p, c, base, nseg, tau, sigma);
+        staging_role<kListed>(p, c, base, nseg, tau, sigma);
       }
     }
     block_bar();
@@ -888,6 +930,7 @@ __device__ __forceinline__ void run_roles(const F8Params& P, const PartialParams
   }
 }
 
+template <bool kListed>
 __global__ void __launch_bounds__(kThreads, 1) partial_f8_kernel(const __grid_constant__ F8Params P) {
   // dense only: a known-null index list lets the compiler drop the sparse
   // branches of the shared schedule
@@ -955,10 +998,10 @@ __global__ void __launch_bounds__(kThreads, 1) partial_f8_kernel(const __grid_co
   // end so that each is compiled within its own budget.
   if (warp < kSoftWarps) {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftRegs));
-    run_roles<true>(P, p, c, base, lo, hi);
+    run_roles<true, kListed>(P, p, c, base, lo, hi);
   } else {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kOtherRegs));
-    run_roles<false>(P, p, c, base, lo, hi);
+    run_roles<false, kListed>(P, p, c, base, lo, hi);
   }
   if (c.abort && threadIdx.x == 0 && p.flags) atomicOr(p.flags, kFlagTimeout);
   ptx::tc_fence_before();
@@ -1063,6 +1106,19 @@ EncodeTiledFn encode_fn() {
 bool encode_maps(const PartialParams& p, CUtensorMap* rows, CUtensorMap* scales) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
+  if (p.row_ids) {
+    // listed rows: the cache as [blocks * 64][656] bytes, boxes one row high
+    // (128-byte code and rope chunks for the four-row gathers)
+    const cuuint64_t dims2[2] = {(cuuint64_t)kRowBytesFp8, (cuuint64_t)p.num_blocks * kBlock};
+    const cuuint64_t strides2[1] = {(cuuint64_t)kRowBytesFp8};
+    const cuuint32_t box2[2] = {128, 1};
+    const cuuint32_t es2[2] = {1, 1};
+    void* g2 = const_cast<uint8_t*>(p.kv);
+    *scales = CUtensorMap{};
+    return enc(rows, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, g2, dims2, strides2, box2, es2,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  }
   const cuuint64_t dims[3] = {(cuuint64_t)kRowBytesFp8, (cuuint64_t)kBlock,
                               (cuuint64_t)p.num_blocks};
   const cuuint64_t strides[2] = {(cuuint64_t)kRowBytesFp8, (cuuint64_t)kRowBytesFp8 * kBlock};
@@ -1080,7 +1136,7 @@ bool encode_maps(const PartialParams& p, CUtensorMap* rows, CUtensorMap* scales)
 }
 
 std::mutex g_attr_mutex;
-bool g_attr_done[kMaxDevicesConfigured] = {};
+bool g_attr_done[2][kMaxDevicesConfigured] = {};   // [listed rows][device]
 
 }  // namespace
 
@@ -1099,27 +1155,29 @@ cudaError_t launch_partial_f8(const PartialParams& p, cudaStream_t st) {
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevicesConfigured) return cudaErrorInvalidDevice;
   const int smem = (int)kSmemBytes;
+  const bool listed = p.row_ids != nullptr;
+  auto kernel = listed ? partial_f8_kernel<true> : partial_f8_kernel<false>;
   {
-    // raise the shared-memory limit once per device, so that later launches
-    // (including ones captured into a CUDA graph) are plain launches
+    // raise the shared-memory limit once per device and instantiation, so
+    // that later launches (including ones captured into a CUDA graph) are
+    // plain launches
     std::lock_guard<std::mutex> lock(g_attr_mutex);
-    if (!g_attr_done[dev]) {
+    if (!g_attr_done[listed][dev]) {
       // the in-kernel register split assumes exactly kLaunchRegs registers
       // per thread at launch; with fewer, the softmax warpgroups' increase
       // could never be granted
       cudaFuncAttributes fa;
-      e = cudaFuncGetAttributes(&fa, partial_f8_kernel);
+      e = cudaFuncGetAttributes(&fa, kernel);
       if (e != cudaSuccess) return e;
       if (fa.numRegs != kLaunchRegs || fa.maxThreadsPerBlock < kThreads)
         return cudaErrorInvalidDeviceFunction;
-      e = cudaFuncSetAttribute(partial_f8_kernel,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
       if (e != cudaSuccess) return e;
-      g_attr_done[dev] = true;
+      g_attr_done[listed][dev] = true;
     }
   }
   f8_q_image_kernel<<<dim3(p.batch, 2), 256, 0, st>>>(p, p.q_image);
-  partial_f8_kernel<<<p.num_ctas, kThreads, smem, st>>>(fp);
+  kernel<<<p.num_ctas, kThreads, smem, st>>>(fp);
   return cudaGetLastError();
 }
 

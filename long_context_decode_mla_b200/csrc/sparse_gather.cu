@@ -1,7 +1,12 @@
 // Sparse decode on the tensor-core kernels: each request's index list is
-// localised to this shard and its selected rows are gathered, in list order,
-// into a contiguous run of the workspace; the dense kernels then attend over
-// the gathered rows (tile k of request b is gathered block b * maxblk + k).
+// localised to this shard and compacted, in list order, into the selected
+// rows of the cache.  Two outputs:
+//  * rows: the flat cache row (block * 64 + row) of every selection, the
+//    list padded to whole 64-row tiles with its last entry; the e4m3 kernel
+//    fetches these rows itself (four rows per TMA gather);
+//  * gathered: the selected rows copied into a contiguous run of the
+//    workspace (tile k of request b is gathered block b * maxblk + k), for
+//    the kernels that read whole blocks.
 //
 // "GLM-5.2 vLLM Decode Context Parallelism", section "Separate the backend
 // merge from stable": the global top-K indices are localised to the rank
@@ -24,12 +29,14 @@ constexpr int kPass = kGatherThreads * kPerThread;
 // One CTA per request.  Each pass takes 2,048 indices, 8 consecutive ones per
 // thread: their loads, then their table entries, are independent, so a pass
 // costs two global round trips; a block scan of the per-thread counts places
-// the selections in list order, and the CTA's warps copy the selected rows,
-// four rows in flight per warp.
+// the selections in list order.  kCopy: the CTA's warps copy the selected
+// rows, four rows in flight per warp; else the rows' flat indices are
+// written to rows[b * maxblk * 64 + slot].
+template <bool kCopy>
 __global__ void __launch_bounds__(kGatherThreads) sparse_gather_kernel(
     const uint8_t* kv, long long num_blocks, int row_bytes, const int* block_table, int bt_stride,
     const int* seq_lens, const int* idx, int topk, int shard, int nshards, int maxblk,
-    uint8_t* gathered, int* counts, int* flags) {
+    uint8_t* gathered, int* rows, int* counts, int* flags) {
   __shared__ int warp_sums[kGatherThreads / 32];
   __shared__ long long sel_row[kPass];
   const int b = blockIdx.x;
@@ -73,6 +80,14 @@ __global__ void __launch_bounds__(kGatherThreads) sparse_gather_kernel(
     }
     int tot;
     int pos = block_exclusive_scan(n, warp_sums, &tot);
+    if constexpr (!kCopy) {
+      int* out = rows + (size_t)b * maxblk * kBlock + count;
+#pragma unroll
+      for (int k = 0; k < kPerThread; ++k)
+        if (own[k]) out[pos++] = blk[k] * kBlock + ((t[k] / nshards) & 63);
+      count += tot;
+      continue;                     // the scan's barriers order the passes
+    }
 #pragma unroll
     for (int k = 0; k < kPerThread; ++k)
       if (own[k]) sel_row[pos++] = (long long)blk[k] * kBlock + ((t[k] / nshards) & 63);
@@ -105,6 +120,14 @@ __global__ void __launch_bounds__(kGatherThreads) sparse_gather_kernel(
     count += tot;
     __syncthreads();
   }
+  if constexpr (!kCopy) {
+    // pad the last tile with the last selection (its rows past the count are
+    // cleared and masked by the kernel)
+    __syncthreads();
+    int* out = rows + (size_t)b * maxblk * kBlock;
+    const int pad = (kBlock - count % kBlock) % kBlock;
+    if (count > 0 && (int)threadIdx.x < pad) out[count + threadIdx.x] = out[count - 1];
+  }
   if (threadIdx.x == 0) counts[b] = count;
 }
 
@@ -112,9 +135,17 @@ __global__ void __launch_bounds__(kGatherThreads) sparse_gather_kernel(
 
 cudaError_t launch_sparse_gather(const PartialParams& p, int row_bytes, int maxblk,
                                  uint8_t* gathered, int* counts, cudaStream_t st) {
-  sparse_gather_kernel<<<p.batch, kGatherThreads, 0, st>>>(
+  sparse_gather_kernel<true><<<p.batch, kGatherThreads, 0, st>>>(
       p.kv, p.num_blocks, row_bytes, p.block_table, p.bt_stride, p.seq_lens, p.sparse_idx,
-      p.topk, p.shard, p.nshards, maxblk, gathered, counts, p.flags);
+      p.topk, p.shard, p.nshards, maxblk, gathered, nullptr, counts, p.flags);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_sparse_rows(const PartialParams& p, int maxblk, int* rows, int* counts,
+                               cudaStream_t st) {
+  sparse_gather_kernel<false><<<p.batch, kGatherThreads, 0, st>>>(
+      p.kv, p.num_blocks, 0, p.block_table, p.bt_stride, p.seq_lens, p.sparse_idx, p.topk,
+      p.shard, p.nshards, maxblk, nullptr, rows, counts, p.flags);
   return cudaGetLastError();
 }
 

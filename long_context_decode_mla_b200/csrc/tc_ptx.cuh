@@ -104,28 +104,27 @@ __device__ __forceinline__ bool mbar_wait3(uint64_t* b0, uint32_t p0, uint64_t* 
   return true;
 }
 
-// mbar_wait for five phases at once, one shared-memory round trip for the
-// first test of all five (any of them may repeat a barrier).
-__device__ __forceinline__ bool mbar_wait5(uint64_t* const (&b)[5], const uint32_t (&p)[5],
+// mbar_wait for four phases at once, one shared-memory round trip for the
+// first test of all four (any of them may repeat a barrier).
+__device__ __forceinline__ bool mbar_wait4(uint64_t* const (&b)[4], const uint32_t (&p)[4],
                                            volatile int* abort) {
   uint32_t m;
   asm volatile(
-      "{\n .reg .pred q0, q1, q2, q3, q4;\n .reg .b32 t0, t1, t2, t3, t4;\n"
+      "{\n .reg .pred q0, q1, q2, q3;\n .reg .b32 t0, t1, t2, t3;\n"
       " mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 q0, [%1], %2;\n"
       " mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 q1, [%3], %4;\n"
       " mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 q2, [%5], %6;\n"
       " mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 q3, [%7], %8;\n"
-      " mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 q4, [%9], %10;\n"
       " selp.b32 t0, 1, 0, q0;\n selp.b32 t1, 2, 0, q1;\n selp.b32 t2, 4, 0, q2;\n"
-      " selp.b32 t3, 8, 0, q3;\n selp.b32 t4, 16, 0, q4;\n"
-      " or.b32 t0, t0, t1;\n or.b32 t2, t2, t3;\n or.b32 t0, t0, t4;\n or.b32 %0, t0, t2;\n}\n"
+      " selp.b32 t3, 8, 0, q3;\n"
+      " or.b32 t0, t0, t1;\n or.b32 t2, t2, t3;\n or.b32 %0, t0, t2;\n}\n"
       : "=r"(m)
       : "r"(smem_addr(b[0])), "r"(p[0]), "r"(smem_addr(b[1])), "r"(p[1]), "r"(smem_addr(b[2])),
-        "r"(p[2]), "r"(smem_addr(b[3])), "r"(p[3]), "r"(smem_addr(b[4])), "r"(p[4])
+        "r"(p[2]), "r"(smem_addr(b[3])), "r"(p[3])
       : "memory");
-  if (m == 31u) return true;
+  if (m == 15u) return true;
 #pragma unroll
-  for (int k = 0; k < 5; ++k)
+  for (int k = 0; k < 4; ++k)
     if (!(m & (1u << k)) && !mbar_wait(b[k], p[k], abort)) return false;
   return true;
 }
@@ -186,6 +185,19 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* tmap, int 
       "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
       "l"(tmap), "r"(x), "r"(y), "r"(z), "r"(smem_addr(bar))
+      : "memory");
+}
+
+// Four rows of a 2-D tensor map whose box is one row high: rows r.x .. r.w
+// (any order, repeats allowed), inner coordinate x (x times the element size
+// a multiple of 16 bytes), landing as four consecutive box rows at dst (128-
+// byte aligned; with a swizzled map the pattern follows dst's address bits).
+__device__ __forceinline__ void tma_gather4(uint32_t dst, const void* tmap, int x, int4 r,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(dst),
+      "l"(tmap), "r"(x), "r"(r.x), "r"(r.y), "r"(r.z), "r"(r.w), "r"(smem_addr(bar))
       : "memory");
 }
 
