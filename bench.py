@@ -68,14 +68,15 @@ def parse():
 
 
 def shard_splits(name, N, args):
-    """CTAs a shard launch may use.  The million-token request splits its one
-    long request over the SM share of its shard; the other workloads let each
-    shard launch size its grid for the whole device (the shards' CTAs then
-    queue on the N streams)."""
+    """CTAs a shard launch may use.  The emulated step runs the N shard
+    launches of a DCP group on one GPU at once, so each is sized for its
+    share of the SMs (148 // N: one wave of about one CTA per SM for all N
+    launches together), as each shard would own a whole GPU in the group.
+    The real-DCP mode (one shard per GPU) uses every SM (splits 0)."""
     from long_context_decode_mla_b200 import dcpmla
     if args.splits is not None:
         return args.splits
-    return max(1, dcpmla.device_sm_count() // N) if name == "million" else 0
+    return max(1, dcpmla.device_sm_count() // N)
 
 
 def dist_env():
@@ -389,7 +390,8 @@ def run_ours(args, rank, world, local):
                 "seq_len_median": int(prob.seq_lens.float().median()),
                 "kv_bytes_per_step_per_gpu": kvb, "kernel": args.kernel,
                 "parallelism": f"{world} independent replicas, {N} DCP shards emulated per GPU "
-                               f"on {n_streams} CUDA stream(s)",
+                               f"on {n_streams} CUDA stream(s), each shard launch given "
+                               f"{splits} CTAs (its share of the SMs)",
                 "l2": ("no flush: the KV read per step is larger than 4x the 126 MB L2"
                        if flush is None else
                        "256 MB written before every timed step (outside the timed events)"),
@@ -526,7 +528,7 @@ def time_other_workload(name, dev, rank, world, args, streams_for=None):
     assert dec.flags() == 0, "device flags set"
     st = dict(zip(st, max_over_ranks(list(st.values()))))
     d = leg(name, prob, st, world, kvb,
-            extra={"steps": steps,
+            extra={"steps": steps, "ctas_per_shard_launch": splits,
                    "l2": "256 MB written before every step" if flush is not None else "no flush"})
     if prob.sparse_idx is not None:
         d["note"] = ("kv_GBps counts the selected rows read (each once); total_GBps adds the "

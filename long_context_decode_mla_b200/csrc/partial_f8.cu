@@ -107,7 +107,8 @@ static_assert(kOffCode % 1024 == 0 && kCodeStage % 1024 == 0 && kOffRope % 1024 
                   kOffP % 1024 == 0,
               "swizzled operands need 1024-byte alignment");
 static_assert(kTileBytes == 4 * kChunk + 1024 + kChunk, "a tile is codes, scales and rope");
-constexpr uint32_t kListedTileBytes = kTileBytes - 1024;   // gathered: codes and rope
+constexpr uint32_t kListedTmaBytes = 4 * kChunk;   // listed tile: the gathered code chunks
+constexpr int kListedCopyArrivals = 32;             // listed tile: one per producer lane
 
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColPart = 256;      // 8 score part buffers of 32 columns; O: [0, 256)
@@ -262,10 +263,12 @@ __device__ __forceinline__ void split_hilo4(uint32_t x0, uint32_t x1, uint32_t& 
 // tau % 2.  Lane 0 waits for the slots and arms the tile's barrier.  A block
 // tile is six box loads by lane 0; a tile whose table entry is out of range
 // (flagged) loads block 0 instead and has no valid rows.  A listed tile
-// (sparse rows, p.row_ids) is fetched by lanes 0..15, four rows each: five
-// gathers of four rows (the four code chunks and the rope); its scales are
-// read by the staging warps (four rows of 16 bytes would not land on the
-// 128-byte boundary a tensor copy needs).
+// (sparse rows, p.row_ids) takes the whole warp: lanes 0..15 fetch the code
+// chunks of four rows each by TMA gathers (64 gathers a tile: the tensor
+// unit takes one about every 50 cycles, so the smaller pieces go another
+// way), and every lane copies rope and scales with 16-byte cp.async (eight
+// lanes a 128-byte rope row, swizzled like the tensor copies, and the scales
+// of two rows), then arrives on the tile's barrier when its copies land.
 template <bool kListed>
 __device__ __forceinline__ void producer_role(const F8Params& P, const PartialParams& p, F8Ctl& c,
                               uint8_t* base, int nseg, uint32_t& tau,
@@ -319,18 +322,42 @@ __device__ __forceinline__ void producer_role(const F8Params& P, const PartialPa
         c.nv[cs] = cur.tile_valid_rows();
         F8_TRACE(0, tau);
         if (issue) {
-          ptx::mbar_arrive_expect_tx(bar, kListedTileBytes);
+          ptx::mbar_arrive_expect_tx(bar, kListedTmaBytes);
           ++fills[cs];
         }
       }
       __syncwarp();
-      if (issue && lane < 16) {
-        const int4 r = __ldg(reinterpret_cast<const int4*>(
-                                 p.row_ids + (size_t)cur.v.b * p.row_stride + cur.v.row_begin +
-                                 cur.t * kTileRows) + lane);
+      if (issue) {
+        // lane l holds the flat rows of tile rows 2 l and 2 l + 1
+        const int2 my = __ldg(reinterpret_cast<const int2*>(
+                                  p.row_ids + (size_t)cur.v.b * p.row_stride + cur.v.row_begin +
+                                  cur.t * kTileRows) + lane);
+        const int src4 = 2 * (lane & 15);
+        const int4 r = make_int4(__shfl_sync(0xffffffffu, my.x, src4),
+                                 __shfl_sync(0xffffffffu, my.y, src4),
+                                 __shfl_sync(0xffffffffu, my.x, src4 + 1),
+                                 __shfl_sync(0xffffffffu, my.y, src4 + 1));
+        if (lead) F8_TRACE(9, tau);
+        if (lane < 16) {
 #pragma unroll
-        for (int k = 0; k < 4; ++k) ptx::tma_gather4(dst + k * kChunk + lane * 512, &P.rows, box_x(k), r, bar);
-        ptx::tma_gather4(dst_rope + lane * 512, &P.rows, box_x(4), r, bar);
+          for (int k = 0; k < 4; ++k)
+            ptx::tma_gather4(dst + k * kChunk + lane * 512, &P.rows, box_x(k), r, bar);
+        }
+        if (lead) F8_TRACE(15, tau);
+        const int un = lane & 7;
+#pragma unroll 4
+        for (int k = 0; k < 16; ++k) {
+          const int rr = 4 * k + (lane >> 3);
+          const int ix = __shfl_sync(0xffffffffu, my.x, rr >> 1);
+          const int iy = __shfl_sync(0xffffffffu, my.y, rr >> 1);
+          const uint8_t* src = p.kv + (size_t)((rr & 1) ? iy : ix) * kRowBytesFp8 + 528 + 16 * un;
+          ptx::cp_async16(dst_rope + sw128(rr, un), src, 16);
+        }
+        ptx::cp_async16(dst + kScalesOff + (2 * lane) * 16,
+                        p.kv + (size_t)my.x * kRowBytesFp8 + 512, 16);
+        ptx::cp_async16(dst + kScalesOff + (2 * lane + 1) * 16,
+                        p.kv + (size_t)my.y * kRowBytesFp8 + 512, 16);
+        ptx::cp_async_arrive(bar);
       }
     }
     ++tau;
@@ -356,6 +383,7 @@ __device__ __forceinline__ uint64_t dplus(uint64_t d, uint32_t byte_off) {
 // K-steps of 32, each a hi and a lo MMA into one accumulator; the rope part
 // is four bf16 K-steps of 16.  One loop serves both sides (a small
 // instruction footprint matters more here than constant offsets).
+template <bool kListed>
 __device__ __forceinline__ void qk_role(int side, const PartialParams& p, F8Ctl& c, uint8_t* base,
                                         int nseg, uint32_t& tau, uint32_t& sigma) {
   constexpr uint32_t kIdF8 = ptx::idesc_make(64, 64, 0, false, false);
@@ -393,6 +421,9 @@ __device__ __forceinline__ void qk_role(int side, const PartialParams& p, F8Ctl&
     }
     if (!ptx::mbar_wait4(bars, pars, &c.abort)) return;
     ptx::tc_fence_after();
+    // a listed tile's rope arrived by cp.async (the generic proxy): order it
+    // before the score MMAs, which read through the async proxy
+    if constexpr (kListed) ptx::fence_proxy_async();
     if (side == 0) F8_TRACE(1, tau);
     const uint64_t dcode = dplus(dc0, cs * kCodeStage), drope = dplus(dr0, rs * kChunk);
 #pragma unroll 1
@@ -503,7 +534,6 @@ __device__ __forceinline__ bool load_q(const PartialParams& p, F8Ctl& c, uint8_t
 // implies, and zeros over the codes of rows past the request's end (their
 // bytes are whatever the block holds and must not reach PV).  Thread u
 // handles row u / 2, groups 2 (u % 2) and 2 (u % 2) + 1.
-template <bool kListed>
 __device__ __forceinline__ void staging_role(const PartialParams& p, F8Ctl& c, uint8_t* base, int nseg,
                              uint32_t& tau, uint32_t& sigma) {
   const int u = threadIdx.x - kStageWarp0 * 32;   // 0..127
@@ -516,15 +546,6 @@ __device__ __forceinline__ void staging_role(const PartialParams& p, F8Ctl& c, u
     const uint32_t cs = tau % kCodeStages;
     const int b = tau & 1;
     const bool first = cur.t == 0;
-    // a listed tile's scales come from the cache rows themselves, loaded
-    // before the wait for the tile's bytes
-    float2 sv_listed = make_float2(0.f, 0.f);
-    if constexpr (kListed) {
-      const int rid = __ldg(p.row_ids + (size_t)cur.v.b * p.row_stride + cur.v.row_begin +
-                            cur.t * kTileRows + row);
-      sv_listed = __ldg(reinterpret_cast<const float2*>(p.kv + (size_t)rid * kRowBytesFp8 + 512 +
-                                                         gp * 4));
-    }
     if (first) {
       if (!load_q(p, c, base, cur.v.b, sigma)) return;
       ++sigma;
@@ -535,8 +556,7 @@ __device__ __forceinline__ void staging_role(const PartialParams& p, F8Ctl& c, u
     if (tau >= 2 && !wait_or_abort(&c.sc_empty[b], ((tau / 2) + 1) & 1, c)) return;
     const int nv = c.nv[cs];
     uint8_t* code = base + kOffCode + cs * kCodeStage;
-    const float2 sv = kListed ? sv_listed
-                                : *reinterpret_cast<const float2*>(code + kScalesOff + row * 16 + gp * 4);
+    const float2 sv = *reinterpret_cast<const float2*>(code + kScalesOff + row * 16 + gp * 4);
     const bool valid = row < nv;
     float m0 = valid ? fabsf(sv.x) : 0.f, m1 = valid ? fabsf(sv.y) : 0.f;
 #pragma unroll
@@ -880,11 +900,12 @@ __device__ __forceinline__ void run_roles(const F8Params& P, const PartialParams
       if (warp == kProdWarp) {
         producer_role<kListed>(P, p, c, base, nseg, tau, fills);
       } else if (warp == kQkWarp || warp == kQkWarp2) {
-        if ((threadIdx.x & 31) == 0) qk_role(warp == kQkWarp ? 0 : 1, p, c, base, nseg, tau, sigma);
+        if ((threadIdx.x & 31) == 0)
+          qk_role<kListed>(warp == kQkWarp ? 0 : 1, p, c, base, nseg, tau, sigma);
       } else if (warp == kPvWarp) {
         if ((threadIdx.x & 31) == 0) pv_role(p, c, base, nseg, tau, uses, o_commits);
       } else {
-        staging_role<kListed>(p, c, base, nseg, tau, sigma);
+        staging_role(p, c, base, nseg, tau, sigma);
       }
     }
     block_bar();
@@ -944,7 +965,7 @@ __global__ void __launch_bounds__(kThreads, 1) partial_f8_kernel(const __grid_co
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kCodeStages; ++s) {
-      ptx::mbar_init(&c.full[s], 1);
+      ptx::mbar_init(&c.full[s], kListed ? 1 + kListedCopyArrivals : 1);
       ptx::mbar_init(&c.staged[s], kStageThreads / 32);
       ptx::mbar_init(&c.code_empty[s], 1);
     }

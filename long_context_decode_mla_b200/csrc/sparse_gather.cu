@@ -85,40 +85,40 @@ __global__ void __launch_bounds__(kGatherThreads) sparse_gather_kernel(
 #pragma unroll
       for (int k = 0; k < kPerThread; ++k)
         if (own[k]) out[pos++] = blk[k] * kBlock + ((t[k] / nshards) & 63);
-      count += tot;
-      continue;                     // the scan's barriers order the passes
-    }
+      count += tot;                 // the scan's barriers order the passes
+    } else {
 #pragma unroll
-    for (int k = 0; k < kPerThread; ++k)
-      if (own[k]) sel_row[pos++] = (long long)blk[k] * kBlock + ((t[k] / nshards) & 63);
-    __syncthreads();
-    for (int k0 = warp * 4; k0 < tot; k0 += kWarps * 4) {
-      uint4 v[4][2];
-      const int nr = min(4, tot - k0);
-      // a row is at most 72 units: each lane moves units lane and lane + 32
-      // (and lane + 64 for bf16 rows, below)
+      for (int k = 0; k < kPerThread; ++k)
+        if (own[k]) sel_row[pos++] = (long long)blk[k] * kBlock + ((t[k] / nshards) & 63);
+      __syncthreads();
+      for (int k0 = warp * 4; k0 < tot; k0 += kWarps * 4) {
+        uint4 v[4][2];
+        const int nr = min(4, tot - k0);
+        // a row is at most 72 units: each lane moves units lane and lane + 32
+        // (and lane + 64 for bf16 rows, below)
 #pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const uint4* src = reinterpret_cast<const uint4*>(kv + (size_t)sel_row[k0 + min(r, nr - 1)] * row_bytes);
-        v[r][0] = lane < units ? __ldg(src + lane) : make_uint4(0, 0, 0, 0);
-        v[r][1] = lane + 32 < units ? __ldg(src + lane + 32) : make_uint4(0, 0, 0, 0);
-      }
+        for (int r = 0; r < 4; ++r) {
+          const uint4* src = reinterpret_cast<const uint4*>(kv + (size_t)sel_row[k0 + min(r, nr - 1)] * row_bytes);
+          v[r][0] = lane < units ? __ldg(src + lane) : make_uint4(0, 0, 0, 0);
+          v[r][1] = lane + 32 < units ? __ldg(src + lane + 32) : make_uint4(0, 0, 0, 0);
+        }
 #pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        if (r >= nr) break;
-        const int slot = count + k0 + r;
-        uint4* dst = reinterpret_cast<uint4*>(
-            gathered + (((size_t)b * maxblk + slot / kBlock) * kBlock + slot % kBlock) * row_bytes);
-        if (lane < units) dst[lane] = v[r][0];
-        if (lane + 32 < units) dst[lane + 32] = v[r][1];
-        if (lane + 64 < units) {
-          const uint4* src = reinterpret_cast<const uint4*>(kv + (size_t)sel_row[k0 + r] * row_bytes);
-          dst[lane + 64] = __ldg(src + lane + 64);
+        for (int r = 0; r < 4; ++r) {
+          if (r >= nr) break;
+          const int slot = count + k0 + r;
+          uint4* dst = reinterpret_cast<uint4*>(
+              gathered + (((size_t)b * maxblk + slot / kBlock) * kBlock + slot % kBlock) * row_bytes);
+          if (lane < units) dst[lane] = v[r][0];
+          if (lane + 32 < units) dst[lane + 32] = v[r][1];
+          if (lane + 64 < units) {
+            const uint4* src = reinterpret_cast<const uint4*>(kv + (size_t)sel_row[k0 + r] * row_bytes);
+            dst[lane + 64] = __ldg(src + lane + 64);
+          }
         }
       }
+      count += tot;
+      __syncthreads();
     }
-    count += tot;
-    __syncthreads();
   }
   if constexpr (!kCopy) {
     // pad the last tile with the last selection (its rows past the count are

@@ -137,6 +137,21 @@ def test_sparse_small(impl, N, splits):
     _check_problem(prob, impl, num_splits=splits)
 
 
+# bf16 rows: the auto path copies the selected rows into whole blocks for the
+# fp16-operand kernel; the others select in-kernel
+@pytest.mark.parametrize("impl", IMPLS + ["tc16"])
+@pytest.mark.parametrize("N", [1, 4])
+@pytest.mark.parametrize("splits", [0, 3])
+def test_sparse_bf16_rows(impl, N, splits):
+    prob = wl.make_problem("sparse", num_shards=N, batch=5, seq_len=2500, topk=260,
+                           kv_dtype="bf16", seed=41)
+    idx = prob.sparse_idx
+    idx[0, 100:] = -1                             # a short list
+    idx[2, :] = -1                                # empty list
+    idx[4, :50] = torch.arange(50) + 2500         # some out of range
+    _check_problem(prob, impl, num_splits=splits)
+
+
 # --------------------------------------------------------------- addressing -
 
 def _id_expect(ids):
