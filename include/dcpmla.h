@@ -66,10 +66,10 @@ extern "C" {
 /* Kernel selection for mla_decode_partial. */
 #define DCPMLA_IMPL_AUTO 0   /* fastest available for the arguments */
 #define DCPMLA_IMPL_SIMT 1   /* plain CUDA-core kernel (any H <= 64) */
-#define DCPMLA_IMPL_TC 2     /* tcgen05 / TMEM tensor-core kernel: fp8 rows (dense,
-                                one query token) go to the kernel that multiplies
-                                the e4m3 codes directly; everything else to the
-                                fp16-operand kernel */
+#define DCPMLA_IMPL_TC 2     /* tcgen05 / TMEM tensor-core kernel: fp8 rows (dense
+                                or sparse, one query token per pass) go to the
+                                kernel that multiplies the e4m3 codes directly;
+                                bf16 rows to the fp16-operand kernel */
 #define DCPMLA_IMPL_TC_F16 3 /* the fp16-operand tensor-core kernel for every
                                 argument combination it supports (bf16 rows, fp8
                                 rows converted to fp16; kept for comparison) */
@@ -112,7 +112,10 @@ extern "C" {
  *   bytes: receives the size.
  *
  * Layout: a 256-byte header (int32 flag word at byte 0, the rest reserved),
- * then per-split partial results.  The flag word is OR-ed by the kernels and
+ * then per-split partial results, the sparse selections of a call with
+ * topk > 0 (flat cache rows, or the selected rows copied into whole blocks,
+ * sized for bf16 rows) and the per-request Q operand images of the fp8
+ * kernel (73,984 bytes each).  The flag word is OR-ed by the kernels and
  * never cleared by the library: zero it before the first call if you read it.
  * Returns DCPMLA_OK or a negative code.
  */
@@ -140,6 +143,10 @@ int mla_decode_workspace_size(int batch, int num_heads, int num_splits, int topk
  *   out_lse      [batch][num_heads] fp32: natural-log LSE (-inf if none).
  *   workspace, workspace_bytes: at least mla_decode_workspace_size(...).
  *   num_splits   CTAs to spread the work over (0 = automatic: the SM count).
+ *                Dense decode splits the shard's tiles evenly over them;
+ *                sparse decode on the tensor-core path gives each CTA a
+ *                contiguous range of whole requests (at most 32 each, so the
+ *                grid is at least ceil(batch / 32) CTAs).
  *   impl         DCPMLA_IMPL_* (AUTO picks the tensor-core kernel when it
  *                supports the arguments).
  *   stream       cudaStream_t to enqueue on.
@@ -195,9 +202,10 @@ int mla_decode_partial_multi(const void* q, const void* kv_cache, int kv_dtype,
 /*
  * Bytes of the scratch array built into the library for
  * mla_decode_partial_noalloc: 32 MiB per device, enough for batch 64 x 64
- * heads x 148 splits (about 27.8 MB).  Of the five workloads the tiny,
- * dense, agentic and million-token ones fit; the sparse one (batch 128 with
- * several index-list parts per request) does not and is refused with
+ * heads x 148 splits (about 32.6 MB, 4.7 MB of it the Q operand images of
+ * the fp8 kernel).  Of the five workloads the tiny, dense, agentic and
+ * million-token ones fit; the sparse one (batch 128, whose selections take
+ * about 330 MB of workspace) does not and is refused with
  * DCPMLA_ERR_WORKSPACE.  The array is part of the library's device module:
  * with CUDA's lazy module loading (the default) it takes device memory only
  * on devices where the module is loaded, i.e. that call into the library;
