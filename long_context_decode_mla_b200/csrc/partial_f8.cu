@@ -107,7 +107,13 @@ static_assert(kOffCode % 1024 == 0 && kCodeStage % 1024 == 0 && kOffRope % 1024 
                   kOffP % 1024 == 0,
               "swizzled operands need 1024-byte alignment");
 static_assert(kTileBytes == 4 * kChunk + 1024 + kChunk, "a tile is codes, scales and rope");
-constexpr uint32_t kListedTmaBytes = 4 * kChunk;   // listed tile: the gathered code chunks
+// Listed tile: code chunks 0 and 1 arrive by TMA gathers, 2 and 3 (with the
+// rope and scales) by cp.async.  The tensor unit takes a four-row gather about
+// every 65 cycles and the load/store unit a warp's copy instruction about every
+// 60: splitting the bytes between them was measured best at two chunks each
+// (sparse step 722 GB/s, against 670 with all four gathered and 648 with none).
+constexpr int kGatheredChunks = 2;
+constexpr uint32_t kListedTmaBytes = kGatheredChunks * kChunk;
 constexpr int kListedCopyArrivals = 32;             // listed tile: one per producer lane
 
 constexpr uint32_t kTmemCols = 512;
@@ -263,12 +269,11 @@ __device__ __forceinline__ void split_hilo4(uint32_t x0, uint32_t x1, uint32_t& 
 // tau % 2.  Lane 0 waits for the slots and arms the tile's barrier.  A block
 // tile is six box loads by lane 0; a tile whose table entry is out of range
 // (flagged) loads block 0 instead and has no valid rows.  A listed tile
-// (sparse rows, p.row_ids) takes the whole warp: lanes 0..15 fetch the code
-// chunks of four rows each by TMA gathers (64 gathers a tile: the tensor
-// unit takes one about every 50 cycles, so the smaller pieces go another
-// way), and every lane copies rope and scales with 16-byte cp.async (eight
-// lanes a 128-byte rope row, swizzled like the tensor copies, and the scales
-// of two rows), then arrives on the tile's barrier when its copies land.
+// (sparse rows, p.row_ids) takes the whole warp: lanes 0..15 fetch code
+// chunks of four rows each by TMA gathers, and every lane copies the other
+// chunks, the rope and the scales with 16-byte cp.async (eight lanes a
+// 128-byte row piece, swizzled like the tensor copies, and the scales of two
+// rows), then arrives on the tile's barrier when its copies land.
 template <bool kListed>
 __device__ __forceinline__ void producer_role(const F8Params& P, const PartialParams& p, F8Ctl& c,
                               uint8_t* base, int nseg, uint32_t& tau,
@@ -338,20 +343,22 @@ __device__ __forceinline__ void producer_role(const F8Params& P, const PartialPa
                                  __shfl_sync(0xffffffffu, my.x, src4 + 1),
                                  __shfl_sync(0xffffffffu, my.y, src4 + 1));
         if (lead) F8_TRACE(9, tau);
-        if (lane < 16) {
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-            ptx::tma_gather4(dst + k * kChunk + lane * 512, &P.rows, box_x(k), r, bar);
-        }
-        if (lead) F8_TRACE(15, tau);
         const int un = lane & 7;
+        // code chunks [0, kGatheredChunks) by TMA gathers, the others and the
+        // rope by cp.async, interleaved so that the tensor copy unit and the
+        // load/store unit drain their queues together
 #pragma unroll 4
         for (int k = 0; k < 16; ++k) {
+          if ((k & 3) == 0 && (k >> 2) < kGatheredChunks && lane < 16)
+            ptx::tma_gather4(dst + (k >> 2) * kChunk + lane * 512, &P.rows, box_x(k >> 2), r, bar);
           const int rr = 4 * k + (lane >> 3);
           const int ix = __shfl_sync(0xffffffffu, my.x, rr >> 1);
           const int iy = __shfl_sync(0xffffffffu, my.y, rr >> 1);
-          const uint8_t* src = p.kv + (size_t)((rr & 1) ? iy : ix) * kRowBytesFp8 + 528 + 16 * un;
-          ptx::cp_async16(dst_rope + sw128(rr, un), src, 16);
+          const uint8_t* row = p.kv + (size_t)((rr & 1) ? iy : ix) * kRowBytesFp8 + 16 * un;
+          ptx::cp_async16(dst_rope + sw128(rr, un), row + 528, 16);
+#pragma unroll
+          for (int g = kGatheredChunks; g < 4; ++g)
+            ptx::cp_async16(dst + g * kChunk + sw128(rr, un), row + 128 * g, 16);
         }
         ptx::cp_async16(dst + kScalesOff + (2 * lane) * 16,
                         p.kv + (size_t)my.x * kRowBytesFp8 + 512, 16);
@@ -421,7 +428,7 @@ __device__ __forceinline__ void qk_role(int side, const PartialParams& p, F8Ctl&
     }
     if (!ptx::mbar_wait4(bars, pars, &c.abort)) return;
     ptx::tc_fence_after();
-    // a listed tile's rope arrived by cp.async (the generic proxy): order it
+    // part of a listed tile arrived by cp.async (the generic proxy): order it
     // before the score MMAs, which read through the async proxy
     if constexpr (kListed) ptx::fence_proxy_async();
     if (side == 0) F8_TRACE(1, tau);
@@ -465,6 +472,7 @@ __device__ __forceinline__ void qk_role(int side, const PartialParams& p, F8Ctl&
 // stationary M = 64 heads, N = 128 values, K = 32 tokens; V_g is the code
 // chunk g of the tile's slot read MN-major, kept in a collector buffer
 // between the hi and lo MMAs.
+template <bool kListed>
 __device__ __forceinline__ void pv_role(const PartialParams& p, F8Ctl& c, uint8_t* base, int nseg, uint32_t& tau,
                         uint32_t (&uses)[kCodeStages], uint32_t& o_commits) {
   constexpr uint32_t kIdPv = ptx::idesc_make(64, 128, 0, false, true);
@@ -476,6 +484,8 @@ __device__ __forceinline__ void pv_role(const PartialParams& p, F8Ctl& c, uint8_
     const uint32_t cs = tau % kCodeStages;
     if (!wait_or_abort(&c.p_full, tau & 1, c)) return;
     ptx::tc_fence_after();
+    // a listed tile's V chunks 2 and 3 arrived by cp.async (the generic proxy)
+    if constexpr (kListed) ptx::fence_proxy_async();
     F8_TRACE(3, tau);
     const uint64_t dv = dplus(dv0, cs * kCodeStage);
     const uint32_t acc0 = cur.t == 0 ? 0u : 1u;
@@ -903,7 +913,7 @@ __device__ __forceinline__ void run_roles(const F8Params& P, const PartialParams
         if ((threadIdx.x & 31) == 0)
           qk_role<kListed>(warp == kQkWarp ? 0 : 1, p, c, base, nseg, tau, sigma);
       } else if (warp == kPvWarp) {
-        if ((threadIdx.x & 31) == 0) pv_role(p, c, base, nseg, tau, uses, o_commits);
+        if ((threadIdx.x & 31) == 0) pv_role<kListed>(p, c, base, nseg, tau, uses, o_commits);
       } else {
         staging_role(p, c, base, nseg, tau, sigma);
       }
