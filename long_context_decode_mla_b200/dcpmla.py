@@ -497,3 +497,126 @@ class DcpDecoder:
         with torch.cuda.graph(g, stream=side):
             self.step(prob, side, merge)
         return g
+
+
+class _StepInputs:
+    """Device copies of one step's inputs, in the attribute form DcpDecoder
+    reads; the cache is shared resident state."""
+
+    def __init__(self, prob):
+        self.q = prob.q.clone()
+        self.kv_cache = prob.kv_cache
+        self.kv_dtype = prob.kv_dtype
+        self.block_tables = prob.block_tables.clone()
+        self.seq_lens = prob.seq_lens.clone()
+        self.sparse_idx = None if prob.sparse_idx is None else prob.sparse_idx.clone()
+        self.softmax_scale = prob.softmax_scale
+        self.block_size = prob.block_size
+        self.num_shards = prob.num_shards
+
+
+class HostPipeline:
+    """Whole decode steps fed from host memory, host copies overlapped with
+    the compute of the neighbouring steps.
+
+    Two slots, each a DcpDecoder with its own device inputs (q, lengths,
+    block tables, sparse lists), outputs and captured step graph; the KV cache
+    (``prob.kv_cache``) is shared, resident state.  Step k runs in slot k % 2:
+
+    * its inputs are copied in on the copy-in stream, once the slot's previous
+      graph has finished reading them;
+    * its graph runs on the compute stream, after that copy and after the
+      slot's previous results have been copied out;
+    * its merged O and LSE are copied out on the copy-out stream.
+
+    So step k + 1's inputs and step k − 1's results cross PCIe while step k
+    computes.  Host buffers should be pinned (``tensor.pin_memory()``) for
+    the copies to be asynchronous.  A step's host results are ready once
+    ``done_event(k)`` has completed; the host input buffers of step k may be
+    reused once ``inputs_copied_event(k)`` has.
+    """
+
+    def __init__(self, prob, num_shards=None, topk=0, num_splits=0, impl="auto", streams=None,
+                 compute_stream=None):
+        n = prob.num_shards if num_shards is None else num_shards
+        dev = prob.q.device
+        self.compute = compute_stream or torch.cuda.current_stream(dev)
+        self.copy_in = torch.cuda.Stream(device=dev)
+        self.copy_out = torch.cuda.Stream(device=dev)
+        self.slots = []
+        for _ in range(2):
+            inputs = _StepInputs(prob)
+            dec = DcpDecoder(prob.q.shape[0], prob.q.shape[1], n, topk=topk,
+                             num_splits=num_splits, device=dev, impl=impl, streams=streams)
+            with torch.cuda.stream(self.compute):
+                graph = dec.capture(inputs)
+            self.slots.append((inputs, dec, graph))
+        torch.cuda.synchronize(dev)
+        self._in_copied = [None, None]      # per slot: inputs landed (copy-in stream)
+        self._computed = [None, None]       # per slot: graph done (compute stream)
+        self._out_copied = [None, None]     # per slot: results copied out
+        self.k = 0
+
+    def decoder(self, slot: int) -> DcpDecoder:
+        return self.slots[slot][1]
+
+    def submit(self, h_q, h_lens, h_tables, h_idx, h_out, h_lse) -> int:
+        """Enqueue one step; returns its index k.  ``h_out`` [B, H, 512] and
+        ``h_lse`` [B, H] receive the merged results."""
+        x = self.k % 2
+        inputs, dec, graph = self.slots[x]
+        if self._computed[x] is not None:
+            self.copy_in.wait_event(self._computed[x])
+        with torch.cuda.stream(self.copy_in):
+            inputs.q.copy_(h_q, non_blocking=True)
+            inputs.seq_lens.copy_(h_lens, non_blocking=True)
+            inputs.block_tables.copy_(h_tables, non_blocking=True)
+            if h_idx is not None:
+                inputs.sparse_idx.copy_(h_idx, non_blocking=True)
+        e_in = torch.cuda.Event()
+        e_in.record(self.copy_in)
+        self._in_copied[x] = e_in
+        self.compute.wait_event(e_in)
+        if self._out_copied[x] is not None:
+            self.compute.wait_event(self._out_copied[x])
+        with torch.cuda.stream(self.compute):
+            graph.replay()
+        e_c = torch.cuda.Event()
+        e_c.record(self.compute)
+        self._computed[x] = e_c
+        self.copy_out.wait_event(e_c)
+        with torch.cuda.stream(self.copy_out):
+            h_out.copy_(dec.out, non_blocking=True)
+            h_lse.copy_(dec.out_lse, non_blocking=True)
+        e_o = torch.cuda.Event()
+        e_o.record(self.copy_out)
+        self._out_copied[x] = e_o
+        self.k += 1
+        return self.k - 1
+
+    def done_event(self, k: int):
+        """Event completing when step k's results are on the host (valid
+        until step k + 2 is submitted)."""
+        assert k in (self.k - 1, self.k - 2), "only the last two steps are tracked"
+        return self._out_copied[k % 2]
+
+    def inputs_copied_event(self, k: int):
+        assert k in (self.k - 1, self.k - 2), "only the last two steps are tracked"
+        return self._in_copied[k % 2]
+
+    def start_after(self, event) -> None:
+        """Make the pipeline's next work (on all three streams) wait for
+        ``event`` (e.g. the start event of a timed region)."""
+        for s in (self.copy_in, self.compute, self.copy_out):
+            s.wait_event(event)
+
+    def join(self, stream=None) -> None:
+        """Make ``stream`` (default: the compute stream) wait for every
+        submitted step's copies."""
+        s = self.compute if stream is None else stream
+        for e in self._out_copied + self._in_copied:
+            if e is not None:
+                s.wait_event(e)
+
+    def flags(self) -> int:
+        return self.slots[0][1].flags() | self.slots[1][1].flags()
