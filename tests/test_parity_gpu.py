@@ -242,6 +242,35 @@ def test_bad_block_entry_is_flagged_not_read():
     assert dec.flags() & dcpmla.FLAG_BAD_BLOCK
 
 
+@pytest.mark.parametrize("impl", IMPLS)
+@pytest.mark.parametrize("splits", [0, 2])
+def test_sparse_bad_block_entry_is_flagged_and_skipped(impl, splits):
+    # one table entry of shard 1 points outside the pool: the selections in
+    # that block are flagged and left out, the rest decode as usual
+    N, bad_b, bad_k = 2, 1, 2
+    prob = wl.make_problem("sparse", num_shards=N, batch=4, seq_len=3000, topk=300, seed=21)
+    expect = wl.DecodeProblem(prob.q, prob.kv_cache, prob.kv_dtype, prob.block_tables.clone(),
+                              prob.seq_lens, N, prob.softmax_scale, prob.sparse_idx.clone(),
+                              prob.block_size)
+    idx = expect.sparse_idx[bad_b]
+    hit = (idx >= 0) & (idx % N == 1) & ((idx // N) // prob.block_size == bad_k)
+    assert hit.any()
+    idx[hit] = -1
+    prob.block_tables[1, bad_b, bad_k] = 10 ** 6
+    dp = prob.to("cuda")
+    dec = dcpmla.DcpDecoder(prob.batch, prob.heads, N, topk=prob.sparse_idx.shape[1],
+                            num_splits=splits, impl=impl)
+    dec.step(dp)
+    torch.cuda.synchronize()
+    assert dec.flags() & dcpmla.FLAG_BAD_BLOCK
+    rp, rl, ro, rlse = _oracle(expect)
+    parts, lses = dec.partials.double().cpu().numpy(), dec.lses.double().cpu().numpy()
+    for s in range(N):
+        _compare(parts[s], lses[s], rp[s], rl[s], prob.kv_dtype, f"shard {s}")
+    _compare(dec.out.double().cpu().numpy(), dec.out_lse.double().cpu().numpy(), ro, rlse,
+             prob.kv_dtype, "merged")
+
+
 def test_length_beyond_table_is_flagged():
     prob = wl.make_problem("tiny", num_shards=2).to("cuda")
     prob.seq_lens[0] = 10 ** 6                       # needs more blocks than the row has
