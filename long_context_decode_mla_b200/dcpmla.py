@@ -539,6 +539,8 @@ class HostPipeline:
     def __init__(self, prob, num_shards=None, topk=0, num_splits=0, impl="auto", streams=None,
                  compute_stream=None):
         n = prob.num_shards if num_shards is None else num_shards
+        if prob.q.dim() != 3 or prob.q.shape[1] > MAX_HEADS:
+            raise ValueError("HostPipeline runs single-query steps: q must be [B, H <= 64, 576]")
         dev = prob.q.device
         self.compute = compute_stream or torch.cuda.current_stream(dev)
         self.copy_in = torch.cuda.Stream(device=dev)

@@ -137,6 +137,18 @@ def test_sparse_small(impl, N, splits):
     _check_problem(prob, impl, num_splits=splits)
 
 
+# more requests than one CTA of the request-aligned schedule takes (32): a
+# single requested CTA becomes ceil(70 / 32) = 3, each with empty lists
+@pytest.mark.parametrize("impl", IMPLS)
+def test_sparse_many_requests_per_cta(impl):
+    prob = wl.make_problem("sparse", num_shards=2, batch=70, seq_len=1500, topk=100, seed=33)
+    idx = prob.sparse_idx
+    idx[5] = -1
+    idx[40] = -1
+    idx[69, 1:] = -1
+    _check_problem(prob, impl, num_splits=1)
+
+
 # bf16 rows: the auto path copies the selected rows into whole blocks for the
 # fp16-operand kernel; the others select in-kernel
 @pytest.mark.parametrize("impl", IMPLS + ["tc16"])
