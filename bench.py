@@ -135,8 +135,8 @@ def measured_peaks():
 # the translation unit of the fp8 partial kernel (whose DRAM traffic
 # profiles/traffic.json records) and the headers it includes; other files are
 # compiled separately and cannot change that kernel
-PARTIAL_KERNEL_SOURCES = ("common.cuh", "kernels.h", "partial_f8.cu", "schedule.cuh",
-                          "tc_ptx.cuh")
+PARTIAL_KERNEL_SOURCES = ("common.cuh", "kernels.h", "partial_f8.cu", "q_image.cuh",
+                          "schedule.cuh", "tc_ptx.cuh")
 
 
 def _code_only(text: str) -> str:
@@ -375,13 +375,14 @@ def run_ours(args, rank, world, local):
         [ms_step, e2e_ms, ms_partials, e2e_serial_ms])
     st_step = dict(zip(st_step, max_over_ranks(list(st_step.values()))))
     st_part = dict(zip(st_part, max_over_ranks(list(st_part.values()))))
-    # Launches per shard call.  The e4m3 kernel (fp8 rows, the default) is
-    # preceded by its Q image kernel; dense decode adds the split combine;
-    # sparse decode on the tensor-core path gathers the selected rows first
-    # and keeps whole requests per CTA (no combine).  The fp16-operand and
-    # CUDA-core kernels select sparse rows in-kernel and need the combine only
-    # when a request's list spans several CTAs (lists longer than 2,048, or
-    # fewer requests than SMs).  Plus one merge per step.
+    # Launches per shard call.  Dense: the e4m3 kernel (fp8 rows, the default)
+    # is preceded by its Q image kernel and followed by the split combine.
+    # Sparse on the tensor-core path: a pre-kernel localises the lists, then
+    # the Q image and the partial with whole requests per CTA (fp8), or the
+    # partial and the combine (bf16).  The fp16-operand
+    # and CUDA-core kernels select sparse rows in-kernel and need the combine
+    # only when a request's list spans several CTAs (lists longer than 2,048,
+    # or fewer requests than SMs).  Plus one merge per step.
     f8 = prob.kv_dtype == "fp8" and args.kernel in ("auto", "tc")
     if prob.sparse_idx is not None:
         if args.kernel in ("tc16", "simt"):
@@ -389,7 +390,6 @@ def run_ours(args, rank, world, local):
             parts = max(-(-topk // 2048), sms // max(1, B))
             per_shard = 2 if parts > 1 else 1
         else:
-            # gather + image + partial (fp8), gather + partial + combine (bf16)
             per_shard = 3
     else:
         per_shard = 2 + (1 if f8 else 0)

@@ -57,6 +57,7 @@
 #include "common.cuh"
 #include "kernels.h"
 #include "schedule.cuh"
+#include "q_image.cuh"
 #include "tc_ptx.cuh"
 
 namespace dcpmla {
@@ -100,6 +101,9 @@ constexpr uint32_t kOffQr = kOffQl + 4 * kChunk;  // Q rope: 64 rows x 64 bf16
 constexpr uint32_t kOffCode = kOffQr + kChunk;
 constexpr uint32_t kQOperandBytes = kOffCode - kOffQh;   // hi, lo and rope, contiguous
 static_assert(kQOperandBytes + 64 * 4 == (uint32_t)kQImageBytes, "Q image = operands + frame");
+static_assert(kOffQl - kOffQh == qimg::kLo && kOffQr - kOffQh == qimg::kRope &&
+                  kQOperandBytes == qimg::kFrame,
+              "the image's operand part is the Q region of shared memory, byte for byte");
 constexpr uint32_t kOffRope = kOffCode + kCodeStages * kCodeStage;
 constexpr uint32_t kOffP = kOffRope + kRopeStages * kChunk;
 constexpr uint32_t kOffCtl = kOffP + 8 * kPVar;
@@ -173,9 +177,7 @@ struct F8Ctl {
 constexpr size_t kSmemBytes = kOffCtl + sizeof(F8Ctl) + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
-__device__ __forceinline__ uint32_t sw128(int r, int u) {
-  return (uint32_t)((r >> 3) * 1024 + (r & 7) * 128 + ((u ^ (r & 7)) << 4));
-}
+using qimg::sw128;   // 128-byte swizzle of unit u in row r
 __device__ __forceinline__ uint32_t sw64(int r, int u) {
   return (uint32_t)((r >> 3) * 512 + (r & 7) * 64 + (((u ^ ((r & 7) >> 1)) & 3) << 4));
 }
@@ -196,23 +198,6 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
-}
-
-// two fp32 -> two e4m3 (lo -> low byte), round to nearest even, saturated
-__device__ __forceinline__ uint32_t e4m3x2_f32(float lo, float hi) {
-  uint16_t r;
-  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
-  return r;
-}
-// two e4m3 (low byte first) -> two fp32, exact
-__device__ __forceinline__ float2 e4m3x2_to_f32(uint32_t pair) {
-  uint32_t h;
-  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"((uint16_t)pair));
-  float lo, hi;
-  asm("{\n .reg .f16 a, b;\n mov.b32 {a, b}, %2;\n cvt.f32.f16 %0, a;\n cvt.f32.f16 %1, b;\n}\n"
-      : "=f"(lo), "=f"(hi)
-      : "r"(h));
-  return make_float2(lo, hi);
 }
 
 // fp16 pairs as 32-bit words, round-to-nearest arithmetic that the compiler
@@ -1043,73 +1028,11 @@ __global__ void __launch_bounds__(kThreads, 1) partial_f8_kernel(const __grid_co
 
 // ------------------------------------------------------------- Q image ----
 
-// Two words of bf16 pairs (four values) times the frame 2^a -> the e4m3 codes
-// of the four values (hi) and the e4m3 codes of what hi leaves of them (lo),
-// first value in the low byte.  The product is exact (a power of two within
-// range) and so is the remainder.
-__device__ __forceinline__ void split_q4(uint32_t w0, uint32_t w1, float fa, uint32_t& hi,
-                                         uint32_t& lo) {
-  const float f0 = __uint_as_float(w0 << 16) * fa;
-  const float f1 = __uint_as_float(w0 & 0xFFFF0000u) * fa;
-  const float f2 = __uint_as_float(w1 << 16) * fa;
-  const float f3 = __uint_as_float(w1 & 0xFFFF0000u) * fa;
-  const uint32_t h01 = e4m3x2_f32(f0, f1), h23 = e4m3x2_f32(f2, f3);
-  const float2 b01 = e4m3x2_to_f32(h01), b23 = e4m3x2_to_f32(h23);
-  hi = h01 | (h23 << 16);
-  lo = e4m3x2_f32(f0 - b01.x, f1 - b01.y) | (e4m3x2_f32(f2 - b23.x, f3 - b23.y) << 16);
-}
-
-// Q operand images, one per request: the frame 2^a of a head puts the largest
-// |q| of its latent in [128, 256); the latent times 2^a is split into two
-// e4m3 terms, and the rope is copied as it is (the softmax scales its score
-// by 2^a).  Head rows past p.heads are zero.  Grid (batch, 2): each CTA covers
-// 32 head rows with 8 threads per head; thread t holds latent values
-// [64 t, 64 t + 64) (four 16-value units of group t / 2) and rope unit t, and
-// issues all its loads before any use.
+// Q operand images of every request (q_image.cuh).  Grid (batch, 2): each CTA
+// covers 32 head rows with 8 threads per head.
 __global__ void __launch_bounds__(256) f8_q_image_kernel(const PartialParams p, uint8_t* image) {
-  const int b = blockIdx.x;
-  const int h = blockIdx.y * 32 + (threadIdx.x >> 3), t = threadIdx.x & 7;
-  const bool live = h < p.heads;
-  const uint4* src =
-      reinterpret_cast<const uint4*>(p.q + ((size_t)b * p.rows_q + (live ? h : 0)) * kHeadDim);
-  const uint4 zero = make_uint4(0, 0, 0, 0);
-  uint4 v[8];
-#pragma unroll
-  for (int k = 0; k < 8; ++k) v[k] = live ? __ldg(src + 8 * t + k) : zero;
-  const uint4 rope = live ? __ldg(src + 64 + t) : zero;
-  float amax = 0.f;
-#pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    const uint32_t w[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
-#pragma unroll
-    for (int e = 0; e < 4; ++e)
-      amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(w[e] << 16)),
-                               fabsf(__uint_as_float(w[e] & 0xFFFF0000u))));
-  }
-#pragma unroll
-  for (int o = 1; o < 8; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-  int a = 0;
-  if (amax > 0.f) {
-    const int e = (int)((__float_as_uint(amax) >> 23) & 0xFF) - 127;
-    a = min(120, max(-120, 7 - e));
-  }
-  const float fa = __uint_as_float((uint32_t)(127 + a) << 23);
-  uint8_t* img = image + (size_t)b * kQImageBytes;
-  if (t == 0) reinterpret_cast<float*>(img + kQOperandBytes)[h] = __uint_as_float((uint32_t)(127 - a) << 23);
-  const int g = t >> 1;
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const int un = (t & 1) * 4 + j;
-    const uint4 x0 = v[2 * j], x1 = v[2 * j + 1];
-    uint4 hi, lo;
-    split_q4(x0.x, x0.y, fa, hi.x, lo.x);
-    split_q4(x0.z, x0.w, fa, hi.y, lo.y);
-    split_q4(x1.x, x1.y, fa, hi.z, lo.z);
-    split_q4(x1.z, x1.w, fa, hi.w, lo.w);
-    *reinterpret_cast<uint4*>(img + kOffQh + g * kChunk + sw128(h, un)) = hi;
-    *reinterpret_cast<uint4*>(img + kOffQl + g * kChunk + sw128(h, un)) = lo;
-  }
-  *reinterpret_cast<uint4*>(img + kOffQr + sw128(h, t)) = rope;
+  qimg::build_q_image_row(p.q, p.rows_q, p.heads, blockIdx.x,
+                          blockIdx.y * 32 + (threadIdx.x >> 3), threadIdx.x & 7, image);
 }
 
 // ---------------------------------------------------------------- host -----

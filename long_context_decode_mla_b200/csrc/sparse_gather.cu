@@ -3,7 +3,7 @@
 // rows of the cache.  Two outputs:
 //  * rows: the flat cache row (block * 64 + row) of every selection, the
 //    list padded to whole 64-row tiles with its last entry; the e4m3 kernel
-//    fetches these rows itself (four rows per TMA gather);
+//    fetches these rows itself (TMA gathers and cp.async);
 //  * gathered: the selected rows copied into a contiguous run of the
 //    workspace (tile k of request b is gathered block b * maxblk + k), for
 //    the kernels that read whole blocks.
