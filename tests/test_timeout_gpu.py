@@ -93,3 +93,39 @@ def test_withhold_needs_the_tensor_core_kernel():
                                       prob.seq_lens, 0, 2, None, prob.softmax_scale, o, l, ws, 8,
                                       impl)
         assert e.value.code == -1
+
+
+def test_withheld_tile_times_out_on_the_listed_e4m3_kernel():
+    # sparse fp8 decode runs on the listed instantiation of the e4m3 kernel
+    # (row lists, TMA gathers and cp.async): its producer withholds every
+    # CTA's first tile, the waits run out, the copies of the tiles it did
+    # issue are drained, and the next call is correct
+    prob = wl.make_problem("sparse", num_shards=2, batch=4, seq_len=3000, topk=300,
+                           seed=43).to("cuda")
+    B, H = prob.batch, prob.heads
+    topk = prob.sparse_idx.shape[1]
+    o = torch.empty(B, H, 512, device="cuda")
+    l = torch.empty(B, H, device="cuda")
+    ws = torch.zeros(dcpmla.mla_decode_workspace_size(B, H, 2, topk), dtype=torch.uint8,
+                     device="cuda")
+    dcpmla.mla_decode_partial(prob.q, prob.kv_cache, "fp8", prob.block_tables[0], prob.seq_lens,
+                              0, 2, prob.sparse_idx, prob.softmax_scale, o, l, ws, 2,
+                              dcpmla.IMPLS["tc"] | WITHHOLD)
+    torch.cuda.synchronize()
+    assert int(ws[:4].view(torch.int32).item()) & dcpmla.FLAG_TIMEOUT
+
+    dec = dcpmla.DcpDecoder(B, H, 2, topk=topk, impl="tc")
+    dec.step(prob)
+    torch.cuda.synchronize()
+    assert dec.flags() == 0
+    ni = wl.make_problem("sparse", num_shards=2, batch=4, seq_len=3000, topk=300,
+                         seed=43).numpy_inputs()
+    _, _, ref, ref_lse = oracle.dcp_decode(ni["q"], ni["kv_cache"], "fp8", ni["block_tables"],
+                                           ni["seq_lens"], 2, ni["softmax_scale"],
+                                           ni["sparse_idx"], ni["block_size"])
+    out = dec.out.double().cpu().numpy()
+    lse = dec.out_lse.double().cpu().numpy()
+    assert np.abs(out - ref).max() <= 2e-2 * np.abs(ref).max()
+    fin = np.isfinite(ref_lse)
+    assert np.array_equal(fin, np.isfinite(lse))
+    assert np.abs(lse[fin] - ref_lse[fin]).max() <= 1e-3
