@@ -528,20 +528,44 @@ __device__ __forceinline__ void softmax_role(const PartialParams& p, TcCtl& c, u
       ptx::named_bar(1, 128);
       const float ltot = l + c.lred[half ^ 1][h];
       const float inv = ltot > 0.f ? 1.f / ltot : 0.f;
-#pragma unroll
+      // Each lane holds 32 values of its head's row per TMEM load; eight
+      // lanes exchange them (an 8 x 8 transpose of 16-byte pieces in three
+      // butterfly steps) so that the eight pieces of one row leave together
+      // as a whole 128-byte line, instead of every store touching 32 lines.
+      const int i8 = L & 7, row8 = L & 24;   // place in, and first lane of, the group of 8
+      float* o_rows = (v.whole ? p.out : p.ws_o) + (row - h + (h & ~31) + row8) * kVDim;
+#pragma unroll 1
       for (int q = 0; q < 8; ++q) {
         uint32_t r[32];
         ptx::tmem_ld32(lane_base + (q >> 2) * 128 + (q & 3) * 32, r);
         ptx::tmem_wait_ld();
-        if (h < p.heads) {
-          float4* dst =
-              reinterpret_cast<float4*>(o_base + (q >> 2) * 256 + half * 128 + (q & 3) * 32);
+        float4 piece[8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e)
-            dst[e] = make_float4(__uint_as_float(r[4 * e]) * inv, __uint_as_float(r[4 * e + 1]) * inv,
+        for (int e = 0; e < 8; ++e)
+          piece[e] = make_float4(__uint_as_float(r[4 * e]) * inv, __uint_as_float(r[4 * e + 1]) * inv,
                                  __uint_as_float(r[4 * e + 2]) * inv,
                                  __uint_as_float(r[4 * e + 3]) * inv);
+#pragma unroll
+        for (int m = 4; m >= 1; m >>= 1) {
+          const bool upper = (i8 & m) != 0;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            if (e & m) continue;
+            const float4 send = upper ? piece[e] : piece[e | m];
+            float4 got;
+            got.x = __shfl_xor_sync(0xffffffffu, send.x, m);
+            got.y = __shfl_xor_sync(0xffffffffu, send.y, m);
+            got.z = __shfl_xor_sync(0xffffffffu, send.z, m);
+            got.w = __shfl_xor_sync(0xffffffffu, send.w, m);
+            if (upper) piece[e] = got; else piece[e | m] = got;
+          }
         }
+        // piece[k] is now piece i8 of the row of lane row8 + k
+        const int col = (q >> 2) * 256 + half * 128 + (q & 3) * 32 + 4 * i8;
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          if ((h & ~31) + row8 + k < p.heads)
+            *reinterpret_cast<float4*>(o_rows + (size_t)k * kVDim + col) = piece[k];
       }
       if (h < p.heads && half == 0)
         *l_base = ltot > 0.f ? (m_used + log2f(ltot)) * kLn2 : -CUDART_INF_F;
