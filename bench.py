@@ -79,6 +79,24 @@ def shard_splits(name, N, args):
     return max(1, dcpmla.device_sm_count() // N)
 
 
+def launches_per_shard(kv_dtype, kernel, sparse, topk, batch, sms):
+    """Kernel launches of one mla_decode_partial call.  Dense: the e4m3
+    kernel (fp8 rows under the auto and tc choices) is preceded by its Q image
+    kernel; the split combine follows.  Sparse on the tensor-core path: a
+    pre-kernel localises the lists, then the Q image and the partial with
+    whole requests per CTA (fp8), or the partial and the combine (bf16).  The
+    fp16-operand and CUDA-core kernels select sparse rows in-kernel and need
+    the combine only when a request's list spans several CTAs (lists longer
+    than 2,048, or fewer requests than SMs)."""
+    f8 = kv_dtype == "fp8" and kernel in ("auto", "tc")
+    if sparse:
+        if kernel in ("tc16", "simt"):
+            parts = max(-(-topk // 2048), sms // max(1, batch))
+            return 2 if parts > 1 else 1
+        return 3
+    return 3 if f8 else 2
+
+
 def dist_env():
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -375,24 +393,9 @@ def run_ours(args, rank, world, local):
         [ms_step, e2e_ms, ms_partials, e2e_serial_ms])
     st_step = dict(zip(st_step, max_over_ranks(list(st_step.values()))))
     st_part = dict(zip(st_part, max_over_ranks(list(st_part.values()))))
-    # Launches per shard call.  Dense: the e4m3 kernel (fp8 rows, the default)
-    # is preceded by its Q image kernel and followed by the split combine.
-    # Sparse on the tensor-core path: a pre-kernel localises the lists, then
-    # the Q image and the partial with whole requests per CTA (fp8), or the
-    # partial and the combine (bf16).  The fp16-operand
-    # and CUDA-core kernels select sparse rows in-kernel and need the combine
-    # only when a request's list spans several CTAs (lists longer than 2,048,
-    # or fewer requests than SMs).  Plus one merge per step.
-    f8 = prob.kv_dtype == "fp8" and args.kernel in ("auto", "tc")
-    if prob.sparse_idx is not None:
-        if args.kernel in ("tc16", "simt"):
-            sms = torch.cuda.get_device_properties(dev).multi_processor_count
-            parts = max(-(-topk // 2048), sms // max(1, B))
-            per_shard = 2 if parts > 1 else 1
-        else:
-            per_shard = 3
-    else:
-        per_shard = 2 + (1 if f8 else 0)
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    per_shard = launches_per_shard(prob.kv_dtype, args.kernel, prob.sparse_idx is not None,
+                                   topk, B, sms)
     gpu_launches = args.steps * (N * per_shard + 1)
     peak, peak_kind = measured_peaks()
     result = None

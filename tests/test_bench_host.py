@@ -159,3 +159,36 @@ def test_shard_kv_bytes_add_up_to_the_step():
         for N in (1, 3, 8):
             p = workload.make_problem(name, num_shards=N, **over)
             assert sum(bench.shard_kv_bytes(p, s) for s in range(N)) == bench.kv_bytes(p)
+
+
+def test_launches_per_shard_call():
+    import bench
+    sms = 148
+    # dense: Q image + e4m3 partial + split combine for fp8 under auto/tc
+    assert bench.launches_per_shard("fp8", "auto", False, 0, 64, sms) == 3
+    assert bench.launches_per_shard("fp8", "tc", False, 0, 64, sms) == 3
+    # dense bf16 rows, or the fp16-operand / CUDA-core kernels: partial + combine
+    assert bench.launches_per_shard("bf16", "auto", False, 0, 32, sms) == 2
+    assert bench.launches_per_shard("fp8", "tc16", False, 0, 64, sms) == 2
+    assert bench.launches_per_shard("fp8", "simt", False, 0, 64, sms) == 2
+    # sparse on the tensor-core path: lists + image + partial (fp8), or
+    # lists + partial + combine (bf16)
+    assert bench.launches_per_shard("fp8", "auto", True, 2048, 128, sms) == 3
+    assert bench.launches_per_shard("bf16", "auto", True, 2048, 128, sms) == 3
+    # in-kernel selection: a combine only when a list spans several CTAs
+    assert bench.launches_per_shard("fp8", "tc16", True, 2048, 128, sms) == 1
+    assert bench.launches_per_shard("fp8", "simt", True, 4096, 128, sms) == 2
+    assert bench.launches_per_shard("fp8", "tc16", True, 256, 16, sms) == 2
+
+
+def test_shard_splits_is_the_sm_share(monkeypatch):
+    import argparse
+    import bench
+    from long_context_decode_mla_b200 import dcpmla
+    monkeypatch.setattr(dcpmla, "device_sm_count", lambda: 148)
+    args = argparse.Namespace(splits=None)
+    assert bench.shard_splits("agentic", 8, args) == 18
+    assert bench.shard_splits("tiny", 2, args) == 74
+    assert bench.shard_splits("million", 1, args) == 148
+    args.splits = 37
+    assert bench.shard_splits("sparse", 8, args) == 37
