@@ -111,14 +111,15 @@ static_assert(kOffCode % 1024 == 0 && kCodeStage % 1024 == 0 && kOffRope % 1024 
                   kOffP % 1024 == 0,
               "swizzled operands need 1024-byte alignment");
 static_assert(kTileBytes == 4 * kChunk + 1024 + kChunk, "a tile is codes, scales and rope");
-// Listed tile: code chunks 0 and 1 arrive by TMA gathers, 2 and 3 (with the
-// rope and scales) by cp.async.  The tensor unit takes a four-row gather about
-// every 65 cycles and the load/store unit a warp's copy instruction about every
-// 60: splitting the bytes between them was measured best at two chunks each
-// (sparse step 722 GB/s, against 670 with all four gathered and 648 with none).
+// Listed tile: code chunks 0 and 1 arrive by TMA gathers from the producer
+// warp, 2 and 3 (with the rope and scales) by cp.async from the staging warps.
+// The tensor unit takes a four-row gather about every 65 cycles and a warp's
+// copy instruction costs about as much: splitting the bytes between the two
+// units was measured best at two chunks each, and spreading the copies over
+// the four staging warps (one per scheduler) takes them off the producer.
 constexpr int kGatheredChunks = 2;
 constexpr uint32_t kListedTmaBytes = kGatheredChunks * kChunk;
-constexpr int kListedCopyArrivals = 32;             // listed tile: one per producer lane
+constexpr int kListedCopyArrivals = 128;            // listed tile: one per staging thread
 
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColPart = 256;      // 8 score part buffers of 32 columns; O: [0, 256)
@@ -254,11 +255,8 @@ __device__ __forceinline__ void split_hilo4(uint32_t x0, uint32_t x1, uint32_t& 
 // tau % 2.  Lane 0 waits for the slots and arms the tile's barrier.  A block
 // tile is six box loads by lane 0; a tile whose table entry is out of range
 // (flagged) loads block 0 instead and has no valid rows.  A listed tile
-// (sparse rows, p.row_ids) takes the whole warp: lanes 0..15 fetch code
-// chunks of four rows each by TMA gathers, and every lane copies the other
-// chunks, the rope and the scales with 16-byte cp.async (eight lanes a
-// 128-byte row piece, swizzled like the tensor copies, and the scales of two
-// rows), then arrives on the tile's barrier when its copies land.
+// (sparse rows, p.row_ids): lanes 0..15 fetch code chunks 0 and 1 of four
+// rows each by TMA gathers; the staging warps copy the rest (listed_fetch).
 template <bool kListed>
 __device__ __forceinline__ void producer_role(const F8Params& P, const PartialParams& p, F8Ctl& c,
                               uint8_t* base, int nseg, uint32_t& tau,
@@ -317,39 +315,15 @@ __device__ __forceinline__ void producer_role(const F8Params& P, const PartialPa
         }
       }
       __syncwarp();
-      if (issue) {
-        // lane l holds the flat rows of tile rows 2 l and 2 l + 1
-        const int2 my = __ldg(reinterpret_cast<const int2*>(
-                                  p.row_ids + (size_t)cur.v.b * p.row_stride + cur.v.row_begin +
-                                  cur.t * kTileRows) + lane);
-        const int src4 = 2 * (lane & 15);
-        const int4 r = make_int4(__shfl_sync(0xffffffffu, my.x, src4),
-                                 __shfl_sync(0xffffffffu, my.y, src4),
-                                 __shfl_sync(0xffffffffu, my.x, src4 + 1),
-                                 __shfl_sync(0xffffffffu, my.y, src4 + 1));
+      if (issue && lane < 16) {
+        // rows 4 l .. 4 l + 3 of the tile
+        const int4 r = __ldg(reinterpret_cast<const int4*>(
+                                 p.row_ids + (size_t)cur.v.b * p.row_stride + cur.v.row_begin +
+                                 cur.t * kTileRows) + lane);
         if (lead) F8_TRACE(9, tau);
-        const int un = lane & 7;
-        // code chunks [0, kGatheredChunks) by TMA gathers, the others and the
-        // rope by cp.async, interleaved so that the tensor copy unit and the
-        // load/store unit drain their queues together
-#pragma unroll 4
-        for (int k = 0; k < 16; ++k) {
-          if ((k & 3) == 0 && (k >> 2) < kGatheredChunks && lane < 16)
-            ptx::tma_gather4(dst + (k >> 2) * kChunk + lane * 512, &P.rows, box_x(k >> 2), r, bar);
-          const int rr = 4 * k + (lane >> 3);
-          const int ix = __shfl_sync(0xffffffffu, my.x, rr >> 1);
-          const int iy = __shfl_sync(0xffffffffu, my.y, rr >> 1);
-          const uint8_t* row = p.kv + (size_t)((rr & 1) ? iy : ix) * kRowBytesFp8 + 16 * un;
-          ptx::cp_async16(dst_rope + sw128(rr, un), row + 528, 16);
 #pragma unroll
-          for (int g = kGatheredChunks; g < 4; ++g)
-            ptx::cp_async16(dst + g * kChunk + sw128(rr, un), row + 128 * g, 16);
-        }
-        ptx::cp_async16(dst + kScalesOff + (2 * lane) * 16,
-                        p.kv + (size_t)my.x * kRowBytesFp8 + 512, 16);
-        ptx::cp_async16(dst + kScalesOff + (2 * lane + 1) * 16,
-                        p.kv + (size_t)my.y * kRowBytesFp8 + 512, 16);
-        ptx::cp_async_arrive(bar);
+        for (int k = 0; k < kGatheredChunks; ++k)
+          ptx::tma_gather4(dst + k * kChunk + lane * 512, &P.rows, box_x(k), r, bar);
       }
     }
     ++tau;
@@ -523,12 +497,51 @@ __device__ __forceinline__ bool load_q(const PartialParams& p, F8Ctl& c, uint8_t
   return true;
 }
 
+// Listed tile tau (cursor t): the parts the producer's gathers leave (code
+// chunks kGatheredChunks.., the rope and the scales), copied by the 128
+// staging threads with 16-byte cp.async into the tile's slots, once the
+// slots are free (the PV of tile tau - 3, the score MMAs of tile tau - 2);
+// eight threads take one 128-byte piece of a row, swizzled like the tensor
+// copies.  Each thread arrives on the tile's barrier when its copies land.
+__device__ __forceinline__ bool listed_fetch(const PartialParams& p, F8Ctl& c, uint8_t* base,
+                                             const TileCursor& t, uint32_t tau, int u) {
+  const uint32_t cs = tau % kCodeStages, rs = tau % kRopeStages;
+  if (tau >= (uint32_t)kCodeStages &&
+      !wait_or_abort(&c.code_empty[cs], ((tau / kCodeStages) + 1) & 1, c))
+    return false;
+  if (tau >= (uint32_t)kRopeStages &&
+      !wait_or_abort(&c.rope_empty[rs], ((tau / kRopeStages) + 1) & 1, c))
+    return false;
+  const int* ids = p.row_ids + (size_t)t.v.b * p.row_stride + t.v.row_begin + t.t * kTileRows;
+  const int un = u & 7, r0 = u >> 3;         // rows r0 + 16 k, 16-byte unit un
+  int id[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) id[k] = __ldg(ids + r0 + 16 * k);
+  const int sid = u < kTileRows ? __ldg(ids + u) : 0;
+  const uint32_t dst = ptx::smem_addr(base + kOffCode + cs * kCodeStage);
+  const uint32_t dst_rope = ptx::smem_addr(base + kOffRope + rs * kChunk);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int rr = r0 + 16 * k;
+    const uint8_t* row = p.kv + (size_t)id[k] * kRowBytesFp8 + 16 * un;
+    ptx::cp_async16(dst_rope + sw128(rr, un), row + 528, 16);
+#pragma unroll
+    for (int g = kGatheredChunks; g < 4; ++g)
+      ptx::cp_async16(dst + g * kChunk + sw128(rr, un), row + 128 * g, 16);
+  }
+  if (u < kTileRows)
+    ptx::cp_async16(dst + kScalesOff + u * 16, p.kv + (size_t)sid * kRowBytesFp8 + 512, 16);
+  ptx::cp_async_arrive(&c.full[cs]);
+  return true;
+}
+
 // Staging (4 warps): per request, its Q; per tile, once its bytes landed,
 // the scales as [group][row] copies (raw, and times kPNorm / S_g as fp16),
 // the reference scales S_g with the O rescale factor a raised reference
 // implies, and zeros over the codes of rows past the request's end (their
 // bytes are whatever the block holds and must not reach PV).  Thread u
 // handles row u / 2, groups 2 (u % 2) and 2 (u % 2) + 1.
+template <bool kListed>
 __device__ __forceinline__ void staging_role(const PartialParams& p, F8Ctl& c, uint8_t* base, int nseg,
                              uint32_t& tau, uint32_t& sigma) {
   const int u = threadIdx.x - kStageWarp0 * 32;   // 0..127
@@ -536,6 +549,11 @@ __device__ __forceinline__ void staging_role(const PartialParams& p, F8Ctl& c, u
   const int row = u >> 1, gp = (u & 1) * 2;
   TileCursor cur;
   if (!cur.start(p, c, nseg)) return;
+  // listed tiles: the copies of a tile are issued one tile ahead of its
+  // staging (the first here)
+  if constexpr (kListed) {
+    if (!listed_fetch(p, c, base, cur, tau, u)) return;
+  }
   float sref[4] = {1.f, 1.f, 1.f, 1.f};
   while (true) {
     const uint32_t cs = tau % kCodeStages;
@@ -604,6 +622,10 @@ __device__ __forceinline__ void staging_role(const PartialParams& p, F8Ctl& c, u
     }
     warp_arrive(&c.staged[cs]);
     if (u == 0) F8_TRACE(21, tau);
+    if constexpr (kListed) {
+      TileCursor nx = cur;
+      if (nx.next(p, c) && !listed_fetch(p, c, base, nx, tau + 1, u)) return;
+    }
     ++tau;
     if (!cur.next(p, c)) break;
   }
@@ -900,7 +922,7 @@ __device__ __forceinline__ void run_roles(const F8Params& P, const PartialParams
       } else if (warp == kPvWarp) {
         if ((threadIdx.x & 31) == 0) pv_role<kListed>(p, c, base, nseg, tau, uses, o_commits);
       } else {
-        staging_role(p, c, base, nseg, tau, sigma);
+        staging_role<kListed>(p, c, base, nseg, tau, sigma);
       }
     }
     block_bar();
@@ -943,6 +965,9 @@ __device__ __forceinline__ void run_roles(const F8Params& P, const PartialParams
         if (fills[s] > 0) wait_or_abort(&c.full[s], (fills[s] - 1) & 1, c);
     // the last Q image copy (the staging warps count their requests in sigma)
     if (threadIdx.x == kStageWarp0 * 32 && sigma > 0) wait_or_abort(&c.q_full, (sigma - 1) & 1, c);
+    // listed tiles: the staging threads' own row copies
+    if (kListed && warp >= kStageWarp0 && warp < kStageWarp0 + kStageThreads / 32)
+      ptx::cp_async_wait_all();
   }
 }
 
