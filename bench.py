@@ -83,8 +83,9 @@ def launches_per_shard(kv_dtype, kernel, sparse, topk, batch, sms):
     """Kernel launches of one mla_decode_partial call.  Dense: the e4m3
     kernel (fp8 rows under the auto and tc choices) is preceded by its Q image
     kernel; the split combine follows.  Sparse on the tensor-core path: a
-    pre-kernel localises the lists, then the Q image and the partial with
-    whole requests per CTA (fp8), or the partial and the combine (bf16).  The
+    pre-kernel localises the lists (and, for fp8 rows, builds the Q images in
+    CTAs of its own), then the partial with whole requests per CTA (fp8), or
+    the partial and the combine (bf16).  The
     fp16-operand and CUDA-core kernels select sparse rows in-kernel and need
     the combine only when a request's list spans several CTAs (lists longer
     than 2,048, or fewer requests than SMs)."""
@@ -93,7 +94,7 @@ def launches_per_shard(kv_dtype, kernel, sparse, topk, batch, sms):
         if kernel in ("tc16", "simt"):
             parts = max(-(-topk // 2048), sms // max(1, batch))
             return 2 if parts > 1 else 1
-        return 3
+        return 2 if f8 else 3
     return 3 if f8 else 2
 
 

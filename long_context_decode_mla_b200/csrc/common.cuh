@@ -65,6 +65,7 @@ struct PartialParams {
   int* ws_list;               // sparse mode: per-CTA lists of selected local rows
   int num_ctas;               // G: CTAs sharing the dense tile space
   uint8_t* q_image;           // e4m3 kernel: per-request Q operand images (workspace)
+  int q_image_ready;          // 1: an earlier launch of the call built them
   const int* row_ids;         // e4m3 kernel, sparse: per-request flat cache rows (padded
                               // to whole tiles); tile k of request b is rows
                               // [b * row_stride + 64 k, + 64) of the list

@@ -228,9 +228,11 @@ int decode_partial(const void* q, const void* kv_cache, int kv_dtype, int64_t nu
                         num_blocks <= (int64_t)(INT32_MAX / kBlock);
     if (listed) {
       int* rows = reinterpret_cast<int*>(gathered);
-      if (launch_sparse_rows(p, maxblk, rows, counts, st) != cudaSuccess) return DCPMLA_ERR_CUDA;
+      if (launch_sparse_rows(p, maxblk, rows, counts, p.q_image, st) != cudaSuccess)
+        return DCPMLA_ERR_CUDA;
       p.row_ids = rows;
       p.row_stride = maxblk * kBlock;
+      p.q_image_ready = 1;
     } else {
       if (launch_sparse_gather(p, rb, maxblk, gathered, counts, st) != cudaSuccess)
         return DCPMLA_ERR_CUDA;

@@ -19,6 +19,6 @@ int simt_sparse_chunk_max();
 cudaError_t launch_sparse_gather(const PartialParams& p, int row_bytes, int maxblk,
                                  uint8_t* gathered, int* counts, cudaStream_t st);
 cudaError_t launch_sparse_rows(const PartialParams& p, int maxblk, int* rows, int* counts,
-                               cudaStream_t st);
+                               uint8_t* q_image, cudaStream_t st);
 
 }  // namespace dcpmla

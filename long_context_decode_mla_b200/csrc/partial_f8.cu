@@ -1155,7 +1155,7 @@ cudaError_t launch_partial_f8(const PartialParams& p, cudaStream_t st) {
       g_attr_done[listed][dev] = true;
     }
   }
-  f8_q_image_kernel<<<dim3(p.batch, 2), 256, 0, st>>>(p, p.q_image);
+  if (!p.q_image_ready) f8_q_image_kernel<<<dim3(p.batch, 2), 256, 0, st>>>(p, p.q_image);
   kernel<<<p.num_ctas, kThreads, smem, st>>>(fp);
   return cudaGetLastError();
 }

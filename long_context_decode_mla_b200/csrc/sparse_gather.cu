@@ -3,7 +3,8 @@
 // rows of the cache.  Two outputs:
 //  * rows: the flat cache row (block * 64 + row) of every selection, the
 //    list padded to whole 64-row tiles with its last entry; the e4m3 kernel
-//    fetches these rows itself (TMA gathers and cp.async);
+//    fetches these rows itself (TMA gathers and cp.async).  The same launch
+//    builds that kernel's Q operand images in CTAs of their own;
 //  * gathered: the selected rows copied into a contiguous run of the
 //    workspace (tile k of request b is gathered block b * maxblk + k), for
 //    the kernels that read whole blocks.
@@ -18,6 +19,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "q_image.cuh"
 
 namespace dcpmla {
 namespace {
@@ -36,9 +38,18 @@ template <bool kCopy>
 __global__ void __launch_bounds__(kGatherThreads) sparse_gather_kernel(
     const uint8_t* kv, long long num_blocks, int row_bytes, const int* block_table, int bt_stride,
     const int* seq_lens, const int* idx, int topk, int shard, int nshards, int maxblk,
-    uint8_t* gathered, int* rows, int* counts, int* flags) {
+    uint8_t* gathered, int* rows, int* counts, int* flags, const __nv_bfloat16* q, int rows_q,
+    int heads, uint8_t* q_image) {
   __shared__ int warp_sums[kGatherThreads / 32];
-  __shared__ long long sel_row[kPass];
+  __shared__ long long sel_row[kCopy ? kPass : 1];
+  // CTAs past the batch build the e4m3 kernel's Q operand images (two per
+  // request, 32 head rows each) alongside the lists, in the same launch
+  if (!kCopy && (int)blockIdx.x >= gridDim.x / 3) {
+    const int k = blockIdx.x - gridDim.x / 3;
+    qimg::build_q_image_row(q, rows_q, heads, k >> 1, (k & 1) * 32 + (threadIdx.x >> 3),
+                            threadIdx.x & 7, q_image);
+    return;
+  }
   const int b = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr int kWarps = kGatherThreads / 32;
@@ -137,15 +148,18 @@ cudaError_t launch_sparse_gather(const PartialParams& p, int row_bytes, int maxb
                                  uint8_t* gathered, int* counts, cudaStream_t st) {
   sparse_gather_kernel<true><<<p.batch, kGatherThreads, 0, st>>>(
       p.kv, p.num_blocks, row_bytes, p.block_table, p.bt_stride, p.seq_lens, p.sparse_idx,
-      p.topk, p.shard, p.nshards, maxblk, gathered, nullptr, counts, p.flags);
+      p.topk, p.shard, p.nshards, maxblk, gathered, nullptr, counts, p.flags, nullptr, 0, 0,
+      nullptr);
   return cudaGetLastError();
 }
 
 cudaError_t launch_sparse_rows(const PartialParams& p, int maxblk, int* rows, int* counts,
-                               cudaStream_t st) {
-  sparse_gather_kernel<false><<<p.batch, kGatherThreads, 0, st>>>(
+                               uint8_t* q_image, cudaStream_t st) {
+  // grid: batch list CTAs, then 2 x batch Q image CTAs
+  sparse_gather_kernel<false><<<3 * p.batch, kGatherThreads, 0, st>>>(
       p.kv, p.num_blocks, 0, p.block_table, p.bt_stride, p.seq_lens, p.sparse_idx, p.topk,
-      p.shard, p.nshards, maxblk, nullptr, rows, counts, p.flags);
+      p.shard, p.nshards, maxblk, nullptr, rows, counts, p.flags, p.q, p.rows_q, p.heads,
+      q_image);
   return cudaGetLastError();
 }
 

@@ -171,9 +171,9 @@ def test_launches_per_shard_call():
     assert bench.launches_per_shard("bf16", "auto", False, 0, 32, sms) == 2
     assert bench.launches_per_shard("fp8", "tc16", False, 0, 64, sms) == 2
     assert bench.launches_per_shard("fp8", "simt", False, 0, 64, sms) == 2
-    # sparse on the tensor-core path: lists + image + partial (fp8), or
-    # lists + partial + combine (bf16)
-    assert bench.launches_per_shard("fp8", "auto", True, 2048, 128, sms) == 3
+    # sparse on the tensor-core path: lists with the Q images + partial (fp8),
+    # or lists + partial + combine (bf16)
+    assert bench.launches_per_shard("fp8", "auto", True, 2048, 128, sms) == 2
     assert bench.launches_per_shard("bf16", "auto", True, 2048, 128, sms) == 3
     # in-kernel selection: a combine only when a list spans several CTAs
     assert bench.launches_per_shard("fp8", "tc16", True, 2048, 128, sms) == 1
