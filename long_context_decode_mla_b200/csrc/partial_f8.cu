@@ -9,15 +9,16 @@
 // round-robin ownership from "How vLLM Serves GLM-5.3 with Million-Token
 // Contexts on 16 H200s", "The core design").
 //
-// How.  The cache rows are read by TMA straight into shared memory and the
-// tensor cores consume the e4m3 codes as they are (kind::f8f6f4); no thread
-// converts cache values.  Scores are exact up to fp32 accumulation order:
+// How.  The cache rows are read straight into shared memory (whole 64-row
+// blocks by TMA; for sparse lists, the listed rows by TMA gathers and
+// cp.async) and the tensor cores consume the e4m3 codes as they are
+// (kind::f8f6f4); no thread converts cache values.  Scores are exact up to
+// fp32 accumulation order:
 //  * Q (bf16, 8 significant bits) is split per head into two e4m3 terms in
-//    one power-of-two frame, q * 2^a = hi + lo.  That is exact for every
-//    element above 2^-9 of the head's largest (smaller ones lose low bits and
-//    weigh at most 2^-9 of it).  hi and lo are two MMAs into one accumulator
-//    that share the key operand through a tensor-core collector buffer, so
-//    the codes are read from shared memory once.
+//    one power-of-two frame, q * 2^a = hi + lo (q_image.cuh, built once per
+//    request by a small kernel).  That is exact for every element of at
+//    least 2^-9 of the head's largest (smaller ones lose low bits and weigh
+//    at most 2^-9 of it).  hi and lo are two MMAs into one accumulator.
 //  * Each 128-value scale group of the latent row has its own accumulator
 //    (weight-stationary M = 64 heads, N = 64 tokens): codes . (hi + lo) for
 //    that group.  The softmax threads multiply it by the token's fp32 group
@@ -31,7 +32,8 @@
 //  * O += P V reads V as the same e4m3 codes.  The group scale multiplies P:
 //    for group g, P_g = p * s_tg * (8 / S_g), stored as two e4m3 terms (hi:
 //    the 4 leading bits of the fp16 value, lo: the rest rounded to 4 bits;
-//    within 2^-7 of P_g together) in a 64 x 64 K-major tile per term; the two
+//    together within max(2^-7 P_g, 2^-9) of P_g) in a 64 x 64 K-major tile
+//    per term; the two
 //    PV MMAs of a term pair share V through a collector buffer.  S_g is a
 //    per-request reference scale (the group's largest scale in the request's
 //    first tile, raised with an exact O rescale if a later tile holds a scale
@@ -43,9 +45,12 @@
 //
 // Roles (16 warps): 0-7 softmax and epilogue (two warps per TMEM lane
 // quarter, one per 16-column half), 8 TMA producer, 9 and 15 issue the score
-// MMAs (parts 0, 2, 4 and parts 1, 3), 10 issues the PV MMAs, 11-14 stage
-// each tile's scales (raw and as P factors, with the reference scales), clear
-// the rows past a request's end and prepare Q (hi / lo split) per request.
+// MMAs (parts 0, 2, 4 and parts 1, 3), 10 issues the PV MMAs, 11-14 load each
+// request's Q image, stage each tile's scales (raw and as P factors, with the
+// reference scales), clear the rows past a request's end and, for listed
+// tiles, copy the parts the producer's gathers leave.  The kernel is a
+// template on the row source (blocks or listed rows), so that dense decode
+// carries none of the listed code.
 // Shared memory: Q 72 KB, three stages of codes and scales (3 x 33 KB), two
 // of rope (2 x 8 KB), P 32 KB.  Every wait is bounded.
 #include <cuda.h>
