@@ -206,11 +206,13 @@ int decode_partial(const void* q, const void* kv_cache, int kv_dtype, int64_t nu
   p.q_image = ws + ws_total((long long)ctas + batch, num_heads);
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  // Sparse decode on the tensor cores: localise and gather the selected rows,
-  // then decode densely over them (one shard of gathered rows, identity
-  // tables), so that fp8 rows reach the exact e4m3 kernel.  The CUDA-core
-  // kernel and the fp16-operand kernel (DCPMLA_IMPL_TC_F16) keep their own
-  // in-kernel selection.
+  // Sparse decode on the tensor cores: a pre-kernel localises each request's
+  // selections, which are then decoded as one shard of selected rows through
+  // identity tables.  fp8 rows go to the exact e4m3 kernel, which fetches the
+  // listed rows from the cache itself, whole requests per CTA; bf16 rows are
+  // copied into whole blocks for the fp16-operand kernel.  The CUDA-core
+  // kernel and the fp16-operand kernel chosen explicitly (DCPMLA_IMPL_TC_F16)
+  // keep their own in-kernel selection.
   const bool gathered_sparse =
       p.sparse_idx && impl != DCPMLA_IMPL_SIMT && impl != DCPMLA_IMPL_TC_F16;
   if (gathered_sparse) {
