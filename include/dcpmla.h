@@ -143,10 +143,11 @@ int mla_decode_workspace_size(int batch, int num_heads, int num_splits, int topk
  *   out_lse      [batch][num_heads] fp32: natural-log LSE (-inf if none).
  *   workspace, workspace_bytes: at least mla_decode_workspace_size(...).
  *   num_splits   CTAs to spread the work over (0 = automatic: the SM count).
- *                Dense decode splits the shard's tiles evenly over them;
- *                sparse decode on the tensor-core path gives each CTA a
- *                contiguous range of whole requests (at most 32 each, so the
- *                grid is at least ceil(batch / 32) CTAs).
+ *                Dense decode splits the shard's tiles evenly over them, as
+ *                does sparse decode of bf16 rows; sparse decode of fp8 rows
+ *                on the tensor-core path gives each CTA a contiguous range of
+ *                whole requests (at most 32 each, so the grid is at least
+ *                ceil(batch / 32) CTAs).
  *   impl         DCPMLA_IMPL_* (AUTO picks the tensor-core kernel when it
  *                supports the arguments).
  *   stream       cudaStream_t to enqueue on.
